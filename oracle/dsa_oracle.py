@@ -1,0 +1,266 @@
+"""CPU oracle for DSA sparse attention -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module.  The product path (the C-ABI library
+and its Python binding) never calls it and has no CPU fallback.
+
+It is a plain, slow, obviously correct restatement of what the path
+computes, in float64, one query row at a time.  It shares no code with the
+CUDA side: it decodes the storage formats itself (OCP FP8 E4M3 from its
+bit-level definition, bf16 from its bit layout), resolves the paged layout
+itself, and uses numpy only for matmuls, sorting and elementwise math.
+
+What each step follows (page titles and sections of the source pages):
+
+* Paged cache lookup -- "Day-0 Adaptation: Running Trillion-Parameter
+  Models on Domestic AI Accelerators", 3.2 KV Cache Layout: the cache is cut
+  into fixed-size blocks and a block table maps logical to physical blocks;
+  "Engineering Practices for Day-0 Adaptation of Million-Token Context
+  Models on Domestic AI Chips", Four Key Layers 2 (64- or 128-token blocks).
+* Indexer score -- "Day-0 Adaptation for LLMs: Implementing Sparse
+  Attention and Low-Precision Weights", III.1 Index Selection Path (a
+  lightweight scoring network relates each query to historical tokens,
+  scored at higher precision than attention; mixed-precision boundaries in
+  V keep index scoring in BF16/FP32).  The pages leave the scorer's form
+  open; this library takes it as
+      I(t, s) = sum_j w[t, j] * ReLU(qI[t, j] . kI[s]),   s <= pos(t),
+  where kI[s] = kS[s] * e4m3(kI8[s]) is the dequantised indexer key.
+* Top-k -- same page III.1 and the decode sketch (score -> topk(score, k)):
+  the k highest scores, ties to the lower token index; every candidate when
+  a query has at most k of them.
+* Sparse attention -- same page, decode sketch (gather the selected rows,
+  then exact attention over them) and "Day-0 Model Adaptation Depends on
+  the Compute Software Stack", Operator Library Abstraction (query vectors,
+  key-value pairs and index lists in, aggregated context vector out).
+  Written here as plain two-pass softmax: m = max z, p = exp(z - m),
+  o = sum p V / sum p, lse = m + ln(sum p).
+* Split combine -- "Engineering Practices ...", Four Key Layers 3 (partial
+  results over candidate KV blocks followed by a cross-block reduction).
+
+Every function is pinned by tests/test_oracle_pins.py against values fixed
+by hand or by independent arithmetic (exact rationals, torch library
+routines, brute force).
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional, Sequence
+
+import numpy as np
+
+# ----------------------------------------------------------------------------
+# storage formats
+# ----------------------------------------------------------------------------
+
+def _e4m3_table() -> np.ndarray:
+    """Value of every OCP FP8 E4M3 byte: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+    bits; exponent field 0 is subnormal (m * 2^-9); S.1111.111 is NaN; no infinities."""
+    t = np.empty(256, dtype=np.float64)
+    for code in range(256):
+        sign = -1.0 if code & 0x80 else 1.0
+        e = (code >> 3) & 0xF
+        m = code & 0x7
+        if e == 0xF and m == 0x7:
+            t[code] = math.nan
+        elif e == 0:
+            t[code] = sign * m * 2.0 ** -9
+        else:
+            t[code] = sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return t
+
+
+E4M3 = _e4m3_table()
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    return E4M3[np.asarray(codes, dtype=np.uint8).astype(np.int64)]
+
+
+def bf16_decode(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns are the upper half of an fp32 word."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def _real(arr: np.ndarray, fmt: str) -> np.ndarray:
+    if fmt == "f32":
+        return np.asarray(arr, dtype=np.float64)
+    if fmt == "bf16":
+        return bf16_decode(arr)
+    if fmt == "e4m3":
+        return e4m3_decode(arr)
+    raise ValueError(fmt)
+
+
+# ----------------------------------------------------------------------------
+# paged layout
+# ----------------------------------------------------------------------------
+
+def row_location(seq_lens: np.ndarray, cu_q: np.ndarray, row: int):
+    """(sequence, absolute position) of query row `row`: a sequence's rows are its last
+    q_len tokens, so row cu_q[b] + i sits at seq_lens[b] - q_len[b] + i."""
+    b = int(np.searchsorted(cu_q, row, side="right") - 1)
+    q_len = int(cu_q[b + 1] - cu_q[b])
+    pos = int(seq_lens[b]) - q_len + (row - int(cu_q[b]))
+    return b, pos
+
+
+def token_slots(block_table_row: np.ndarray, positions: np.ndarray, page_size: int):
+    """Logical token positions -> (physical block, slot) through the block table."""
+    positions = np.asarray(positions, dtype=np.int64)
+    return block_table_row[positions // page_size].astype(np.int64), positions % page_size
+
+
+def _formats(case):
+    if case.kind == "f32":
+        return dict(q="f32", kv="f32", qI="f32", kI="f32")
+    return dict(q="bf16", kv="bf16", qI="e4m3", kI="e4m3")
+
+
+# ----------------------------------------------------------------------------
+# step 1: indexer scores
+# ----------------------------------------------------------------------------
+
+def indexer_scores_row(case, row: int, chunk: int = 1 << 16) -> np.ndarray:
+    """I[s] for s = 0..pos(row) (fp64):
+    I[s] = sum_j w[row, j] * max(0, sum_d qI[row, j, d] * kI[s, d]),
+    with kI[s] = kS[s] * e4m3(kI8[s]) (kS absent: kI is the fp32 key itself)."""
+    fm = _formats(case)
+    b, pos = row_location(case.seq_lens, case.cu_q, row)
+    n = pos + 1
+    qI = _real(case.qI[row], fm["qI"])                      # [Hi, Di]
+    w = np.asarray(case.w[row], dtype=np.float64)           # [Hi]
+    out = np.empty(n, dtype=np.float64)
+    for lo in range(0, n, chunk):
+        s = np.arange(lo, min(n, lo + chunk))
+        blk, slot = token_slots(case.block_table[b], s, case.page_size)
+        kI = _real(case.kI_pool[blk, slot], fm["kI"])       # [m, Di]
+        if case.kS_pool is not None:
+            kI = kI * np.asarray(case.kS_pool[blk, slot], dtype=np.float64)[:, None]
+        dots = kI @ qI.T                                    # [m, Hi]
+        out[lo: lo + s.size] = np.maximum(dots, 0.0) @ w
+    return out
+
+
+# ----------------------------------------------------------------------------
+# step 2: top-k
+# ----------------------------------------------------------------------------
+
+def topk_row(scores: np.ndarray, k: int) -> np.ndarray:
+    """The k best positions under the order (score descending, position ascending),
+    returned ascending and padded with -1 to length k; all positions when n <= k."""
+    scores = np.asarray(scores, dtype=np.float64)
+    n = scores.size
+    pos = np.arange(n)
+    if n <= k:
+        sel = pos
+    else:
+        order = np.lexsort((pos, -scores))   # last key is primary
+        sel = np.sort(order[:k])
+    out = np.full(k, -1, dtype=np.int32)
+    out[: sel.size] = sel
+    return out
+
+
+# ----------------------------------------------------------------------------
+# step 3: sparse attention over the selected rows
+# ----------------------------------------------------------------------------
+
+def gather_kv(case, b: int, idx: np.ndarray):
+    """Selected latent rows: K[i] = kv[idx_i, :Dqk]; V[i] = kv[idx_i, :Dv] for MLA (the value
+    is the leading part of the shared latent row) or v[idx_i] when V is stored apart.
+    -1 entries are dropped."""
+    fm = _formats(case)
+    idx = np.asarray(idx, dtype=np.int64)
+    idx = idx[idx >= 0]
+    blk, slot = token_slots(case.block_table[b], idx, case.page_size)
+    rows = _real(case.kv_pool[blk, slot], fm["kv"])
+    K = rows[:, : case.Dqk]
+    if case.v_pool is None:
+        V = rows[:, : case.Dv]
+    else:
+        V = _real(case.v_pool[blk, slot], fm["kv"])
+    return K, V
+
+
+def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float):
+    """Exact softmax attention of every head of q [H, D] over the rows K [m, D], V [m, Dv]:
+    two passes (max, then normalised sum).  Empty set: o = 0, lse = -inf."""
+    H = q.shape[0]
+    if K.shape[0] == 0:
+        return np.zeros((H, V.shape[1])), np.full(H, -np.inf)
+    z = scale * (q @ K.T)                                   # [H, m]
+    m = z.max(axis=1, keepdims=True)
+    p = np.exp(z - m)
+    l = p.sum(axis=1, keepdims=True)
+    o = (p @ V) / l
+    lse = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+def sparse_attention_row(case, row: int, idx: np.ndarray):
+    fm = _formats(case)
+    b, _ = row_location(case.seq_lens, case.cu_q, row)
+    q = _real(case.q[row], fm["q"])                         # [H, Dqk]
+    K, V = gather_kv(case, b, idx)
+    return attention(q, K, V, case.softmax_scale)
+
+
+def combine(parts: Sequence, lses: Sequence):
+    """Merge partial results over disjoint key subsets: lse = log sum_i exp(lse_i),
+    o = sum_i exp(lse_i - lse) * o_i (partials with lse_i = -inf contribute nothing)."""
+    L = np.stack([np.asarray(x, dtype=np.float64) for x in lses])     # [S, H]
+    O = np.stack([np.asarray(x, dtype=np.float64) for x in parts])    # [S, H, Dv]
+    mx = L.max(axis=0)
+    safe = np.where(np.isfinite(mx), mx, 0.0)
+    wts = np.where(np.isfinite(L), np.exp(L - safe), 0.0)             # [S, H]
+    tot = wts.sum(axis=0)
+    lse = np.where(tot > 0, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    o = np.einsum("sh,shd->hd", wts, O) / np.where(tot > 0, tot, 1.0)[:, None]
+    return o, lse
+
+
+# ----------------------------------------------------------------------------
+# whole path, row by row
+# ----------------------------------------------------------------------------
+
+def run_rows(case, rows: Iterable[int], idx_override: Optional[dict] = None,
+             want_scores: bool = True, want_attention: bool = True) -> dict:
+    """Scores, top-k and attention of the given query rows.  `idx_override[row]` replaces
+    the oracle's own selection for the attention step (conditional parity on another
+    implementation's index set)."""
+    res = {}
+    for row in rows:
+        row = int(row)
+        r = {}
+        sc = indexer_scores_row(case, row)
+        if want_scores:
+            r["scores"] = sc
+        r["idx"] = topk_row(sc, case.topk)
+        if want_attention:
+            idx = r["idx"] if idx_override is None or row not in idx_override else idx_override[row]
+            r["out"], r["lse"] = sparse_attention_row(case, row, idx)
+        res[row] = r
+    return res
+
+
+def dense_masked_attention(case, row: int, idx: np.ndarray):
+    """Second formulation used only to pin `attention`: logits over every cached position of
+    the row's sequence, -inf outside the selected set, softmax over the full axis."""
+    fm = _formats(case)
+    b, pos = row_location(case.seq_lens, case.cu_q, row)
+    n_all = int(case.seq_lens[b])
+    allpos = np.arange(n_all)
+    blk, slot = token_slots(case.block_table[b], allpos, case.page_size)
+    rows = _real(case.kv_pool[blk, slot], fm["kv"])
+    K = rows[:, : case.Dqk]
+    V = rows[:, : case.Dv] if case.v_pool is None else _real(case.v_pool[blk, slot], fm["kv"])
+    q = _real(case.q[row], fm["q"])
+    logits = case.softmax_scale * (q @ K.T)
+    mask = np.zeros(n_all, dtype=bool)
+    sel = np.asarray(idx, dtype=np.int64)
+    mask[sel[sel >= 0]] = True
+    logits = np.where(mask[None, :], logits, -np.inf)
+    mx = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - mx)
+    return (e / e.sum(axis=1, keepdims=True)) @ V

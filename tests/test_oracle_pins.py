@@ -1,0 +1,329 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself.
+
+Each test checks one oracle function against hand-worked values (tests/golden),
+exact rational arithmetic, a torch library routine, or an independent brute
+force, chosen so that a plausible slip (a dropped scale, a wrong causal bound,
+a reversed tie-break, a transposed operand) fails at least one of them.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+from types import SimpleNamespace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_long_dsa_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _single_row_case(qI, kI, w, kS=None, q=None, kv=None, v=None, topk=4, scale=1.0, page=64):
+    """One sequence whose last token is the only query; tokens laid out contiguously."""
+    qI = np.asarray(qI, np.float32)
+    kI = np.asarray(kI, np.float32)
+    n = kI.shape[0]
+    nb = (n + page - 1) // page
+    def paged(a):
+        a = np.asarray(a, np.float32)
+        out = np.zeros((nb * page,) + a.shape[1:], np.float32)
+        out[:n] = a
+        return out.reshape((nb, page) + a.shape[1:])
+    return SimpleNamespace(
+        kind="f32", page_size=page, seq_lens=np.array([n], np.int32), cu_q=np.array([0, 1], np.int32),
+        block_table=np.arange(nb, dtype=np.int32)[None, :], qI=qI[None], w=np.asarray(w, np.float32)[None],
+        kI_pool=paged(kI), kS_pool=None if kS is None else paged(kS),
+        q=None if q is None else np.asarray(q, np.float32)[None], kv_pool=None if kv is None else paged(kv),
+        v_pool=None if v is None else paged(v), Dqk=None if kv is None else np.asarray(kv).shape[1],
+        Dv=None if v is None else np.asarray(v).shape[1], topk=topk, softmax_scale=scale)
+
+
+# ----------------------------------------------------------------------------- storage formats
+
+def test_e4m3_table_matches_torch():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = oracle.E4M3
+    finite = ~np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), ~finite)
+    assert np.array_equal(ours[finite], ref[finite])
+
+
+def test_e4m3_definition_points():
+    # largest finite, one, smallest subnormal, smallest normal, negative one, zero / minus zero
+    assert oracle.e4m3_decode(np.array([0x7E]))[0] == 448.0
+    assert oracle.e4m3_decode(np.array([0x38]))[0] == 1.0
+    assert oracle.e4m3_decode(np.array([0x01]))[0] == 2.0 ** -9
+    assert oracle.e4m3_decode(np.array([0x08]))[0] == 2.0 ** -6
+    assert oracle.e4m3_decode(np.array([0xB8]))[0] == -1.0
+    assert oracle.e4m3_decode(np.array([0x00]))[0] == 0.0
+    assert math.copysign(1.0, oracle.e4m3_decode(np.array([0x80]))[0]) == -1.0
+
+
+def test_bf16_decode_matches_torch():
+    bits = np.random.default_rng(1).integers(0, 1 << 16, 4096, dtype=np.uint16)
+    bits = bits[((bits >> 7) & 0xFF) != 0xFF]                       # finite only
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.bf16_decode(bits), ref)
+
+
+def test_generator_encoders_match_torch():
+    x = np.random.default_rng(2).standard_normal(20000).astype(np.float32) * 60
+    x = np.concatenate([x, [448.0, -448.0, 2 ** -9, 2 ** -10, 3 * 2 ** -11, 0.0, 240.0, 241.0, 232.0]]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(W.e4m3_encode(x), ref)
+    ref16 = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(W.bf16_encode(x), ref16)
+
+
+# ----------------------------------------------------------------------------- layout
+
+def test_row_location_hand():
+    seq_lens = np.array([10, 3, 7], np.int32)
+    cu_q = np.array([0, 1, 4, 6], np.int32)          # q_lens 1, 3, 2
+    got = [oracle.row_location(seq_lens, cu_q, r) for r in range(6)]
+    assert got == [(0, 9), (1, 0), (1, 1), (1, 2), (2, 5), (2, 6)]
+
+
+def test_token_slots_hand():
+    table = np.array([5, 2, 9], np.int32)
+    blk, slot = oracle.token_slots(table, np.array([0, 63, 64, 130]), 64)
+    assert blk.tolist() == [5, 5, 2, 9] and slot.tolist() == [0, 63, 0, 2]
+
+
+# ----------------------------------------------------------------------------- indexer
+
+@pytest.mark.parametrize("case", _golden("indexer_hand.json")["cases"], ids=lambda c: c["name"])
+def test_indexer_hand(case):
+    c = _single_row_case(case["qI"], case["kI"], case["w"])
+    got = oracle.indexer_scores_row(c, 0)
+    assert got.tolist() == case["scores"]
+
+
+def _fraction_score(wl, row, s):
+    """Exact rational score from torch's own decoders: sum_j w_j * max(0, sum_d q_jd * kS * k_sd)."""
+    b, pos = oracle.row_location(wl.seq_lens, wl.cu_q, row)
+    assert s <= pos
+    blk = int(wl.block_table[b, s // wl.page_size]); slot = s % wl.page_size
+    if wl.kind == "mla":
+        dec = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        q = dec(wl.qI[row]); k = dec(wl.kI_pool[blk, slot]); ks = Fraction(float(wl.kS_pool[blk, slot]))
+    else:
+        q = wl.qI[row].astype(np.float64); k = wl.kI_pool[blk, slot].astype(np.float64); ks = Fraction(1)
+    tot = Fraction(0)
+    for j in range(q.shape[0]):
+        d = sum(Fraction(float(q[j, i])) * ks * Fraction(float(k[i])) for i in range(q.shape[1]))
+        tot += Fraction(float(wl.w[row, j])) * max(d, Fraction(0))
+    return tot
+
+
+def _small_mla(grid, seed=77, seq_lens=(130, 70), q_lens=(3, 2), topk=16):
+    return W.make_workload("pin", kind="mla", seed=seed, seq_lens=list(seq_lens), q_lens=list(q_lens),
+                           topk=topk, grid=grid, H=4, Dqk=40, Dv=32, Hi=3, Di=16)
+
+
+def test_indexer_exact_rationals_random_fp8():
+    wl = _small_mla(grid=False)
+    rng = np.random.default_rng(5)
+    for row in range(wl.total_q):
+        sc = oracle.indexer_scores_row(wl, row)
+        b, pos = oracle.row_location(wl.seq_lens, wl.cu_q, row)
+        assert sc.size == pos + 1                          # causal: s = 0..pos inclusive
+        for s in list(rng.choice(pos + 1, 6, replace=False)) + [pos, 0]:
+            exact = float(_fraction_score(wl, row, int(s)))
+            assert abs(sc[s] - exact) <= 1e-12 * max(1.0, abs(exact))
+
+
+def test_indexer_integer_grid_is_exact():
+    wl = _small_mla(grid=True)
+    for row in range(wl.total_q):
+        sc = oracle.indexer_scores_row(wl, row)
+        for s in range(0, sc.size, 7):
+            assert Fraction(float(sc[s])) == _fraction_score(wl, row, s)
+
+
+def test_indexer_f32_rationals():
+    wl = W.make_workload("pinf", kind="f32", seed=3, seq_lens=[90], q_lens=[5], topk=8, H=2, Dqk=8, Dv=8,
+                         Hi=2, Di=8, shuffle=True)
+    for row in range(wl.total_q):
+        sc = oracle.indexer_scores_row(wl, row)
+        for s in (0, 17, sc.size - 1):
+            exact = float(_fraction_score(wl, row, s))
+            assert abs(sc[s] - exact) <= 1e-12 * max(1.0, abs(exact))
+
+
+def test_indexer_positive_homogeneity_in_key_scale():
+    wl = _small_mla(grid=False)
+    base = oracle.indexer_scores_row(wl, 2)
+    wl.kS_pool = wl.kS_pool * np.float32(4.0)
+    assert np.array_equal(oracle.indexer_scores_row(wl, 2), 4.0 * base)
+
+
+# ----------------------------------------------------------------------------- top-k
+
+@pytest.mark.parametrize("case", _golden("topk_hand.json")["cases"])
+def test_topk_hand(case):
+    assert oracle.topk_row(np.array(case["scores"]), case["k"]).tolist() == case["idx"]
+
+
+def _topk_threshold_scan(scores, k):
+    """Independent selection: tau = k-th largest value (np.partition); keep everything above
+    tau, then the lowest positions equal to tau until k are taken."""
+    n = len(scores)
+    if n <= k:
+        return list(range(n)) + [-1] * (k - n)
+    tau = np.partition(scores, n - k)[n - k]
+    above = [s for s in range(n) if scores[s] > tau]
+    equal = [s for s in range(n) if scores[s] == tau]
+    return sorted(above + equal[: k - len(above)])
+
+
+def test_topk_brute_force_with_ties():
+    rng = np.random.default_rng(11)
+    for trial in range(300):
+        n = int(rng.integers(1, 200))
+        k = int(rng.integers(1, 80))
+        scores = rng.integers(-4, 5, n).astype(np.float64) * (0.5 if trial % 2 else 1.0)
+        assert oracle.topk_row(scores, k).tolist() == _topk_threshold_scan(scores, k)
+
+
+def test_topk_brute_force_distinct():
+    rng = np.random.default_rng(12)
+    for _ in range(100):
+        n = int(rng.integers(1, 5000)); k = int(rng.integers(1, 600))
+        scores = rng.standard_normal(n)
+        assert oracle.topk_row(scores, k).tolist() == _topk_threshold_scan(scores, k)
+
+
+# ----------------------------------------------------------------------------- attention
+
+def test_attention_hand():
+    g = _golden("attention_hand.json")
+    a = g["attention"]
+    o, lse = oracle.attention(np.array(a["q"]), np.array(a["K"])[a["idx"]], np.array(a["V"])[a["idx"]], a["scale"])
+    assert np.allclose(o, a["out"], rtol=0, atol=1e-14) and np.allclose(lse, a["lse"], rtol=0, atol=1e-14)
+    c = g["combine"]
+    o, lse = oracle.combine(c["parts"], c["lses"])
+    assert np.allclose(o, c["out"], rtol=0, atol=1e-14) and np.allclose(lse, c["lse"], rtol=0, atol=1e-14)
+
+
+def _tiny_case(topk, grid=False, seed=20260001):
+    return W.make_workload("t", kind="f32", seed=seed, seq_lens=[96], q_lens=[96], topk=topk,
+                           H=3, Dqk=16, Dv=12, Hi=2, Di=8, shuffle=True, grid=grid, w_dist="uniform")
+
+
+def test_attention_matches_torch_sdpa_with_mask():
+    wl = _tiny_case(topk=10)
+    rng = np.random.default_rng(4)
+    for row in (0, 5, 40, 95):
+        _, pos = oracle.row_location(wl.seq_lens, wl.cu_q, row)
+        idx = np.sort(rng.choice(pos + 1, min(10, pos + 1), replace=False))
+        o, lse = oracle.sparse_attention_row(wl, row, idx)
+        allpos = np.arange(int(wl.seq_lens[0]))
+        blk, slot = wl.block_table[0, allpos // 64], allpos % 64
+        K = torch.from_numpy(wl.kv_pool[blk, slot].astype(np.float64))
+        V = torch.from_numpy(wl.v_pool[blk, slot].astype(np.float64))
+        q = torch.from_numpy(wl.q[row].astype(np.float64))
+        mask = torch.zeros(allpos.size, dtype=torch.bool); mask[torch.from_numpy(idx)] = True
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[:, None, :], K.expand(q.shape[0], -1, -1), V.expand(q.shape[0], -1, -1),
+            attn_mask=mask[None, None, :].expand(q.shape[0], 1, -1), scale=wl.softmax_scale)[:, 0, :]
+        assert np.allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+        logits = wl.softmax_scale * (q @ K.T)[:, torch.from_numpy(idx)]
+        assert np.allclose(lse, torch.logsumexp(logits, dim=1).numpy(), rtol=0, atol=1e-12)
+        dense = oracle.dense_masked_attention(wl, row, idx)
+        assert np.allclose(o, dense, rtol=0, atol=1e-12)
+
+
+def test_full_topk_reproduces_dense_causal_attention():
+    """k >= context: the path (indexer -> top-k -> attention) is dense causal attention."""
+    wl = _tiny_case(topk=128)
+    res = oracle.run_rows(wl, range(wl.total_q))
+    allpos = np.arange(96)
+    blk, slot = wl.block_table[0, allpos // 64], allpos % 64
+    K = torch.from_numpy(wl.kv_pool[blk, slot].astype(np.float64))
+    V = torch.from_numpy(wl.v_pool[blk, slot].astype(np.float64))
+    q = torch.from_numpy(wl.q.astype(np.float64)).permute(1, 0, 2)          # [H, T, D]
+    H = q.shape[0]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q, K.expand(H, -1, -1), V.expand(H, -1, -1), is_causal=True, scale=wl.softmax_scale).permute(1, 0, 2)
+    for row in range(96):
+        assert res[row]["idx"][: row + 1].tolist() == list(range(row + 1))
+        assert np.allclose(res[row]["out"], ref[row].numpy(), rtol=0, atol=1e-12)
+
+
+def test_topk_one_selects_argmax_value():
+    wl = _tiny_case(topk=1)
+    res = oracle.run_rows(wl, [50, 77])
+    for row, r in res.items():
+        sc = r["scores"]
+        best = int(np.flatnonzero(sc == sc.max())[0])
+        assert r["idx"].tolist() == [best]
+        K, V = oracle.gather_kv(wl, 0, np.array([best]))
+        assert np.allclose(r["out"], np.broadcast_to(V[0], r["out"].shape), rtol=0, atol=1e-15)
+
+
+def test_equal_logits_average_values():
+    wl = _tiny_case(topk=12)
+    wl.q = np.zeros_like(wl.q)
+    r = oracle.run_rows(wl, [60])[60]
+    K, V = oracle.gather_kv(wl, 0, r["idx"])
+    assert np.allclose(r["out"], np.broadcast_to(V.mean(axis=0), r["out"].shape), rtol=0, atol=1e-14)
+    assert np.allclose(r["lse"], math.log(12), rtol=0, atol=1e-14)
+
+
+def test_split_and_combine_equals_whole():
+    wl = _tiny_case(topk=40)
+    rng = np.random.default_rng(8)
+    r = oracle.run_rows(wl, [90])[90]
+    idx = r["idx"][r["idx"] >= 0]
+    cut = rng.permutation(idx.size)
+    parts, lses = [], []
+    for sub in (idx[cut[:7]], idx[cut[7:25]], idx[cut[25:]], np.array([], np.int64)):
+        o, l = oracle.sparse_attention_row(wl, 90, sub)
+        parts.append(o); lses.append(l)
+    o, lse = oracle.combine(parts, lses)
+    assert np.allclose(o, r["out"], rtol=0, atol=1e-13) and np.allclose(lse, r["lse"], rtol=0, atol=1e-13)
+
+
+def test_block_table_permutation_invariance():
+    wl = _small_mla(grid=False)
+    ref = oracle.run_rows(wl, range(wl.total_q))
+    perm = np.random.default_rng(9).permutation(wl.num_blocks)     # new physical id of old block
+    inv = np.argsort(perm)
+    wl.kv_pool = wl.kv_pool[inv]; wl.kI_pool = wl.kI_pool[inv]; wl.kS_pool = wl.kS_pool[inv]
+    wl.block_table = perm[wl.block_table].astype(np.int32)
+    got = oracle.run_rows(wl, range(wl.total_q))
+    for row in ref:
+        for key in ("scores", "idx", "out", "lse"):
+            assert np.array_equal(ref[row][key], got[row][key])
+
+
+def test_lse_is_log_normaliser():
+    wl = _tiny_case(topk=20)
+    r = oracle.run_rows(wl, [70])[70]
+    q = wl.q[70].astype(np.float64)
+    K, V = oracle.gather_kv(wl, 0, r["idx"])
+    z = wl.softmax_scale * q @ K.T
+    assert np.allclose(np.exp(z - r["lse"][:, None]).sum(axis=1), 1.0, rtol=0, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- planted long-context case
+
+def test_planted_long_context_selection():
+    """1,048,576-token decode: the 2048 planted positions are exactly the oracle's top-k,
+    with the lowest planted score at least twice the highest other score."""
+    wl = W.decode_1m_planted(attention=False)
+    sc = oracle.indexer_scores_row(wl, 0)
+    idx = oracle.topk_row(sc, 2048)
+    assert np.array_equal(idx, wl.planted)
+    others = np.delete(sc, wl.planted)
+    assert sc[wl.planted].min() > 2.0 * max(others.max(), 0.0)

@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA sparse-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_batch] [--impl ours|reference]
+
+One step = one pass of the whole path (indexer scores -> top-k -> sparse attention) over one
+batch of the workload, through the C ABI.  The default workload is the decode batch (32
+sequences, contexts U[4096, 32768], 128 heads x 576 bf16 MLA latent cache, 64 x 128 e4m3
+indexer, top-k 2048); the metric is query tokens per second.  Prints ONE JSON line (rank 0).
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a device synchronise,
+timed with CUDA events on the launching stream; the max over ranks is reported.  Inputs rotate
+over several device replicas so that more than L2 (126 MB) is touched between two reads of the
+same replica.  Per-stage CUDA events inside the timed region give the dominant kernel's average
+duration for the roofline entry.  `e2e` repeats the timing through the same public calls with
+each step's per-step inputs copied from pinned host memory and the results read back.
+
+Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no data-path collective).
+`--impl reference` times the CPU oracle (the plain fp64 restatement of the method) on a bounded
+sample of the same workload on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------------------------------------- work accounting
+def work_of(wl):
+    """Algorithmic bytes and flops per stage for one step (each cached byte the definition must
+    read counted once; the scores/idx round trip between stages is reported separately)."""
+    T = wl.total_q
+    rows_n = []
+    for b in range(wl.num_seqs):
+        lo, hi = int(wl.cu_q[b]), int(wl.cu_q[b + 1])
+        n0 = int(wl.seq_lens[b]) - (hi - lo)
+        rows_n.append(np.arange(hi - lo) + n0 + 1)
+    n = np.concatenate(rows_n) if rows_n else np.zeros(0)
+    sel = np.minimum(n, wl.topk).astype(np.float64)
+    mla = wl.kind == "mla"
+    kb = (wl.Di * (1 if mla else 4) + (4 if mla else 0))            # indexer key bytes per token
+    row_b = wl.Dqk * (2 if mla else 4) + (0 if mla else wl.Dv * 4)   # latent (+V) bytes per token
+    el = 2 if mla else 4
+    idx_bytes = float(np.sum(wl.seq_lens.astype(np.float64)) * kb + T * wl.Hi * (wl.Di * (1 if mla else 4) + 4))
+    idx_flops = float(np.sum(n) * 2 * wl.Hi * wl.Di)
+    topk_bytes = float(np.sum(n) * 4 + T * wl.topk * 4)
+    attn_rows = float(np.sum(sel))
+    # decode: every row is its own sequence, each selected row is read once per query row
+    attn_bytes = attn_rows * row_b + T * wl.H * (wl.Dqk * el + wl.Dv * el)
+    attn_flops = attn_rows * 2 * wl.H * (wl.Dqk + wl.Dv)
+    return dict(indexer=dict(bytes=idx_bytes, flops=idx_flops), topk=dict(bytes=topk_bytes, flops=0.0),
+                attention=dict(bytes=attn_bytes, flops=attn_flops), tokens=T, selected_rows=attn_rows)
+
+
+# ---------------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls NVML for SM clock and throttle reasons in a background thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, period=0.005):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self.period = period
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return None
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if len(win) < 3:
+            win = self.samples
+            window = "warmup+timed"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        bits = 0
+        for s in win:
+            bits |= s[2]
+        reasons = [name for b, name in self.REASONS.items() if bits & b and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(win), "window": window}
+
+
+# ---------------------------------------------------------------------------------------------- ours
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from sparse_attention_long_dsa_b200 import binding as B
+    from sparse_attention_long_dsa_b200 import workloads as W
+    from sparse_attention_long_dsa_b200.pipeline import DeviceBatch
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    B.load()
+    wl = W.BENCH_WORKLOADS[args.workload](**({} if args.workload == "tiny_f32" else {"seed": _seed(args, rank)}))
+    work = work_of(wl)
+    replicas = []
+    for r in range(args.replicas):
+        replicas.append(DeviceBatch(wl, device=dev))
+    stream = torch.cuda.Stream(device=dev)
+    stages = ("indexer", "topk", "attention")
+
+    def step(db, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        db.indexer(stream)
+        if ev is not None:
+            ev[1].record(stream)
+        db.topk(stream)
+        if ev is not None:
+            ev[2].record(stream)
+        db.attention(stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(replicas[i % len(replicas)])
+    torch.cuda.synchronize(dev)
+    for db in replicas:
+        db.check_status(stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = B.dsa_launch_count()
+    w0 = time.perf_counter()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(replicas[i % len(replicas)], evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.perf_counter()
+    launches = B.dsa_launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    sampler.stop()
+    for db in replicas:
+        db.check_status(stream)
+
+    total_ms = t_start.elapsed_time(t_end)
+    stage_ms = {s: [] for s in stages}
+    for e in evs:
+        for j, s in enumerate(stages):
+            stage_ms[s].append(e[j].elapsed_time(e[j + 1]))
+    stage_avg = {s: float(np.mean(v)) for s, v in stage_ms.items()}
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * work["tokens"] / (ms_per_step / 1e3)
+
+    # e2e: per-step inputs from pinned host memory, results read back, same public calls
+    e2e = run_e2e(args, wl, replicas[0], stream, dev, world)
+
+    peaks, peak_src = load_peaks()
+    dom = max(stage_avg, key=stage_avg.get)
+    roof = roofline_entry(dom, stage_avg[dom], work, peaks, peak_src, args)
+    clocks = sampler.summary(w0, w1)
+    res = {
+        "metric": "sparse-attn decode tokens/s" if wl.kind == "mla" and np.all(wl.q_lens == 1)
+        else "sparse-attn prefill tokens/s",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16+e4m3" if wl.kind == "mla" else "f32", "data": "synthetic",
+        "config": workload_config(wl, args),
+        "stages_ms": stage_avg, "roofline": roof, "e2e": e2e, "gpu_launches": int(launches),
+        "clocks": clocks, "impl": "ours",
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    return res
+
+
+def _seed(args, rank):
+    base = {"decode_batch": 20260002, "prefill_16k": 20260003, "decode_1m_planted": 20260004,
+            "mixed_batch": 20260005}[args.workload]
+    return base + 1000 * rank
+
+
+def workload_config(wl, args):
+    d = {"workload": wl.name, "batch_seqs": wl.num_seqs, "query_rows": wl.total_q,
+         "context": f"{int(wl.seq_lens.min())}..{int(wl.seq_lens.max())}", "topk": wl.topk, "heads": wl.H,
+         "d_qk": wl.Dqk, "d_v": wl.Dv, "indexer": f"{wl.Hi}x{wl.Di} {'e4m3' if wl.kind == 'mla' else 'f32'}",
+         "page": wl.page_size, "l2": f"{args.replicas} rotating device replicas of all inputs (> L2 touched "
+                                     f"between reuses)"}
+    return d
+
+
+def roofline_entry(stage, ms, work, peaks, src, args):
+    w = work[stage]
+    secs = ms / 1e3
+    ach = w["bytes"] / secs / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"kernel": stage, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+            "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback",
+            "algorithmic_bytes_per_launch": w["bytes"], "avg_launch_ms": ms, "traffic": None,
+            "tflops": w["flops"] / secs / 1e12}
+
+
+def run_e2e(args, wl, db, stream, dev, world):
+    import torch
+    per_step = {}
+    for name in ("q", "qI", "w", "block_table", "seq_lens", "cu_q"):
+        t = db.inputs[name]
+        per_step[name] = (torch.empty(t.shape, dtype=t.dtype, pin_memory=True), t)
+        per_step[name][0].copy_(t.cpu())
+    out_h = torch.empty(db.out.shape, dtype=db.out.dtype, pin_memory=True)
+    lse_h = torch.empty(db.lse.shape, dtype=db.lse.dtype, pin_memory=True)
+    h2d = sum(h.numel() * h.element_size() for h, _ in per_step.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+
+    def step():
+        for h, d in per_step.values():
+            d.copy_(h, non_blocking=True)
+        db.run(stream)
+        out_h.copy_(db.out, non_blocking=True)
+        lse_h.copy_(db.lse, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * wl.total_q * args.steps / (ms / 1e3)
+    return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": ms / args.steps}
+
+
+# ---------------------------------------------------------------------------------------------- oracle timing
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(wl, budget_s=15.0, rows=None):
+    """The oracle as it stands, timed on host cores over a bounded sample of rows of the workload."""
+    import oracle
+    order = list(range(wl.total_q)) if rows is None else rows
+    rng = np.random.default_rng(0)
+    if rows is None and len(order) > 64:
+        order = sorted(rng.choice(wl.total_q, 64, replace=False).tolist())
+    done, t0 = 0, time.perf_counter()
+    for r in order:
+        oracle.run_rows(wl, [r])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{done} query rows of {wl.name} (full path per row: scores, top-k, attention), "
+                      f"{dt:.1f} s wall"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from sparse_attention_long_dsa_b200 import workloads as W
+    import oracle
+    wl = W.BENCH_WORKLOADS[args.workload](**({} if args.workload == "tiny_f32" else {"seed": _seed(args, 0)}))
+    rows_per_step = 2 if wl.total_q > 1 else 1
+    rng = np.random.default_rng(1)
+
+    def step(i):
+        rs = [(i * rows_per_step + j) % wl.total_q for j in range(rows_per_step)]
+        oracle.run_rows(wl, rs)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = rows_per_step * args.steps / dt
+    cores = _blas_threads()
+    line = {"metric": "sparse-attn decode tokens/s" if np.all(wl.q_lens == 1) else "sparse-attn prefill tokens/s",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "config": workload_config(wl, args), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows_per_step} query rows of {wl.name} per step (bounded sample)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+# ---------------------------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="decode_batch",
+                    choices=["decode_batch", "prefill_16k", "decode_1m_planted", "mixed_batch", "tiny_f32"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--replicas", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    distributed = world > 1 and args.impl == "ours"
+    if distributed:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        else:
+            res = run_ours(args, rank, world, local_rank)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if distributed:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,182 @@
+/*
+ * dsa.h -- C ABI of libdsa: DSA-style sparse attention on NVIDIA B200 (sm_100a).
+ *
+ * The path has three steps, each one call, all sharing one batch descriptor
+ * (dsa_batch_t) so that index selection and attention resolve tokens through
+ * the same block table ("Day-0 Adaptation: Running Trillion-Parameter Models
+ * on Domestic AI Accelerators", 3.1 Index Selection Operator: selection and
+ * attention share the block-mapping semantics; 3.2 KV Cache Layout: paged
+ * cache, block table from logical to physical blocks):
+ *
+ *   dsa_indexer_scores       I(t,s) = sum_j w[t,j] * ReLU(qI[t,j] . kI[s]) for s <= pos(t)
+ *   dsa_topk                 the k best s per query row (ties -> lower s), ascending
+ *   dsa_sparse_attn_prefill  softmax attention of every head over the selected rows
+ *   dsa_sparse_attn_decode   the same, specialised for one query row per sequence
+ *
+ * ("Day-0 Adaptation for LLMs: Implementing Sparse Attention and Low-Precision
+ * Weights", III.1 Index Selection Path and the decode sketch: score -> topk ->
+ * gather -> attention; III.3 and "Engineering Practices for Day-0 Adaptation of
+ * Million-Token Context Models on Domestic AI Chips", Four Key Layers 3:
+ * separate prefill and decode paths.)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Ownership: the caller owns every buffer.  Pointers inside dsa_batch_t and all
+ *   tensor arguments are DEVICE pointers (cudaMalloc'd or equivalent) unless a
+ *   parameter says otherwise.  The library allocates no memory and keeps no
+ *   state beyond cached device attributes; calls are thread-safe.
+ * Asynchrony: every compute call only enqueues work on `stream` (a cudaStream_t
+ *   passed as void*; NULL is the legacy default stream) and returns without
+ *   synchronising the host.  Outputs are valid once the stream reaches them.
+ * Errors: argument errors are detected on the host before anything is enqueued
+ *   and return DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED / DSA_ERR_WORKSPACE with
+ *   nothing written.  A failed launch returns DSA_ERR_CUDA.  Kernels never spin
+ *   without bound: a device wait that runs out sets a bit in the workspace status
+ *   word, which dsa_read_device_status() reports as DSA_ERR_TIMEOUT.  No C++
+ *   exception crosses this ABI.  dsa_last_error() returns a one-line description
+ *   of the last failure on the calling thread.
+ * Rows: query rows are packed sequence after sequence; sequence b owns rows
+ *   cu_q[b] .. cu_q[b+1]-1, which are its LAST n_b = cu_q[b+1]-cu_q[b] tokens:
+ *   row cu_q[b]+i sits at absolute position pos = seq_lens[b] - n_b + i and may
+ *   attend to positions 0..pos (its own entry is already in the cache).
+ * Paged cache: token s of sequence b lives in physical block
+ *   block_table[b * max_blocks_per_seq + s / page_size], slot s % page_size.
+ *   Only entries for s < seq_lens[b] are read.
+ *
+ * Supported shapes (others return DSA_ERR_UNSUPPORTED):
+ *   MLA path    : bf16 q / latent cache, H = 128, Dqk = 576, Dv = 512, V = the first
+ *                 512 entries of each latent row (v_pool NULL); FP8 e4m3 indexer with
+ *                 Hi = 64, Di = 128 and a per-token fp32 key scale; page_size 64.
+ *   fp32 path   : f32 everything, H <= 16, Dqk <= 128, Dv <= 128 with a separate
+ *                 V cache, Hi <= 16, Di <= 128, no key scale; page_size 64.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,   /* NULL where a buffer is required, bad sizes, misaligned strides */
+  DSA_ERR_UNSUPPORTED = 2,   /* valid request outside the shapes/dtypes listed above */
+  DSA_ERR_WORKSPACE = 3,     /* ws_bytes smaller than dsa_workspace_size() */
+  DSA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  DSA_ERR_DEVICE_CHECK = 5,  /* a kernel found an out-of-range block id or index */
+  DSA_ERR_TIMEOUT = 6        /* a bounded device wait ran out (kernel gave up, outputs invalid) */
+} dsa_status_t;
+
+typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_FP8_E4M3 = 2 } dsa_dtype_t;
+
+typedef enum {
+  DSA_OP_INDEXER = 0,
+  DSA_OP_TOPK = 1,
+  DSA_OP_ATTN_PREFILL = 2,
+  DSA_OP_ATTN_DECODE = 3
+} dsa_op_t;
+
+/* Batch descriptor shared by every call.  The three host integers at the end are
+ * upper bounds the caller already knows; they size grids without a device->host
+ * read.  They must hold: total_q == cu_q[num_seqs], max_q_per_seq >= every n_b,
+ * max_seq_len >= every seq_lens[b]. */
+typedef struct {
+  int32_t num_seqs;            /* B >= 1 */
+  int32_t page_size;           /* tokens per block: 64 */
+  int32_t num_blocks;          /* physical blocks in each pool */
+  int32_t max_blocks_per_seq;  /* row stride of block_table */
+  const int32_t *block_table;  /* device [num_seqs, max_blocks_per_seq], values in [0, num_blocks) */
+  const int32_t *seq_lens;     /* device [num_seqs], cached tokens including the query rows' own */
+  const int32_t *cu_q;         /* device [num_seqs + 1], cu_q[0] = 0, non-decreasing */
+  int32_t total_q;             /* host: cu_q[num_seqs] */
+  int32_t max_q_per_seq;       /* host: >= max_b (cu_q[b+1] - cu_q[b]) */
+  int32_t max_seq_len;         /* host: >= max_b seq_lens[b] */
+} dsa_batch_t;
+
+/* Bytes of workspace `op` needs for this batch.  k = top-k count, H / Dv = attention
+ * heads and value width (ignored by INDEXER and TOPK).  The workspace is caller-owned
+ * device memory, 256-byte aligned, reused freely between calls on one stream; calls
+ * that may run concurrently need separate workspaces. */
+DSA_API dsa_status_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t *b, int32_t k, int32_t H, int32_t Dv,
+                                size_t *bytes);
+
+/* Indexer scores ("Day-0 Adaptation for LLMs ...", III.1 Index Selection Path; V keeps
+ * index scoring at BF16/FP32: products of the FP8 inputs are exact, accumulation and the
+ * result are fp32).
+ *   q_idx   [total_q, Hi, Di] of q_dt (DSA_FP8_E4M3 or DSA_F32)
+ *   w       [total_q, Hi] f32 per-head weights (any sign)
+ *   k_idx_pool [num_blocks, page_size, Di] of k_dt (same dtype as q_dt)
+ *   k_scale_pool [num_blocks, page_size] f32 > 0, required for FP8 keys, NULL for f32
+ *   scores  [total_q, ld_scores] f32 output; ld_scores >= max_seq_len, multiple of 4.
+ * Writes scores[row, s] = kS[s] * sum_j w[row,j] * max(0, sum_d qI[row,j,d] * kI8[s,d])
+ * for s = 0..pos(row); entries s > pos(row) are left untouched. */
+DSA_API dsa_status_t dsa_indexer_scores(const void *q_idx, dsa_dtype_t q_dt, const float *w,
+                                const void *k_idx_pool, dsa_dtype_t k_dt, const float *k_scale_pool,
+                                int32_t Hi, int32_t Di, const dsa_batch_t *b,
+                                float *scores, int64_t ld_scores,
+                                void *ws, size_t ws_bytes, void *stream);
+
+/* Top-k selection ("Day-0 Adaptation for LLMs ...", III.1: top-k over long sequences;
+ * decode sketch idx = topk(score, k)).  For each row, with n = pos(row) + 1 candidates
+ * scores[row, 0..n): if n <= k every position is selected, else the first k positions
+ * of the order (score descending, position ascending).  -0 and +0 compare equal; scores
+ * must be finite.  Output idx [total_q, k] int32: selected positions in ascending
+ * order, padded with -1.  The selection is exact (fp32 keys compared as integers). */
+DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_batch_t *b, int32_t k,
+                      int32_t *idx, void *ws, size_t ws_bytes, void *stream);
+
+/* Sparse attention, prefill / any batch ("Day-0 Adaptation for LLMs ...", decode sketch:
+ * gather the selected KV and run exact attention; "Day-0 Model Adaptation Depends on the
+ * Compute Software Stack", Operator Library Abstraction: query, key-value pairs and index
+ * list in, context vector out).  For every row and head h:
+ *   z_i = softmax_scale * q[row,h,:Dqk] . K[idx_i]   over valid idx_i (>= 0)
+ *   out[row,h,:] = sum_i exp(z_i - m) V[idx_i] / sum_i exp(z_i - m),  m = max z
+ *   lse[row,h]   = m + ln(sum_i exp(z_i - m))            (natural log; -inf if no idx)
+ * K[s] = kv_pool row of token s (first Dqk entries); V[s] = first Dv entries of the
+ * same row when v_pool is NULL, else the v_pool row.
+ *   q       [total_q, H, Dqk] of dt;  kv_pool [num_blocks, page_size, Dqk] of dt
+ *   v_pool  NULL (MLA) or [num_blocks, page_size, Dv] of dt
+ *   idx     [total_q, k] int32 logical positions in [0, seq_len) or -1 (skipped)
+ *   out     [total_q, H, Dv] of dt (bf16 for the MLA path);  lse [total_q, H] f32 or NULL */
+DSA_API dsa_status_t dsa_sparse_attn_prefill(const void *q, dsa_dtype_t dt, const void *kv_pool, const void *v_pool,
+                                     int32_t H, int32_t Dqk, int32_t Dv, float softmax_scale,
+                                     const int32_t *idx, int32_t k, const dsa_batch_t *b,
+                                     void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* Sparse attention, decode: same contract as dsa_sparse_attn_prefill, for batches where
+ * every sequence has exactly one query row (cu_q[b] = b); splits each row's key set over
+ * several CTAs and merges the partial results (log-sum-exp combine), as the pages' prefill
+ * unit does across KV blocks ("Engineering Practices ...", Four Key Layers 3).  A batch
+ * with total_q != num_seqs returns DSA_ERR_INVALID_ARG. */
+DSA_API dsa_status_t dsa_sparse_attn_decode(const void *q, dsa_dtype_t dt, const void *kv_pool, const void *v_pool,
+                                    int32_t H, int32_t Dqk, int32_t Dv, float softmax_scale,
+                                    const int32_t *idx, int32_t k, const dsa_batch_t *b,
+                                    void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, then reads and clears the status word at the start of a
+ * workspace used by the calls above: DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK. */
+DSA_API dsa_status_t dsa_read_device_status(void *ws, void *stream);
+
+DSA_API const char *dsa_status_string(dsa_status_t s);
+DSA_API const char *dsa_last_error(void);
+
+/* Number of kernels this library has launched in the process so far (all devices, all
+ * threads).  Lets a caller count the library's launches over a region of its own code. */
+DSA_API uint64_t dsa_launch_count(void);
+
+/* Library version, "major.minor.patch". */
+DSA_API const char *dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_H_ */

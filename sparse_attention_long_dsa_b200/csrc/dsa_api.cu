@@ -1,0 +1,268 @@
+// C ABI of libdsa: argument validation, workspace sizing and kernel dispatch.
+// Every check runs on the host before anything is enqueued; see include/dsa.h for the contract.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace dsa {
+
+// kernels (defined in the other translation units)
+dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx, void *ws,
+                         cudaStream_t stream, int num_sms);
+size_t topk_workspace_bytes(int total_q, int max_seq_len);
+dsa_status_t indexer_simt_launch(const void *qI, dsa_dtype_t dt, const float *w, const void *kpool,
+                                 const float *kscale, int Hi, int Di, const dsa_batch_t *b, float *scores,
+                                 int64_t ld, cudaStream_t stream);
+dsa_status_t attn_simt_launch(const void *q, dsa_dtype_t dt, const void *kv, const void *v, int H, int Dqk, int Dv,
+                              float scale, const int32_t *idx, int k, const dsa_batch_t *b, void *out, float *lse,
+                              cudaStream_t stream);
+
+static thread_local char g_err[512] = "";
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+void set_error(const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  int num_sms = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+static DeviceInfo g_dev[kMaxDevices];
+static std::mutex g_dev_mu;
+
+// Current device's attributes; fails unless it is an sm_100 part (B200).
+static dsa_status_t current_device(DeviceInfo *out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    set_error("no current CUDA device");
+    return DSA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> g(g_dev_mu);
+  if (g_dev[dev].num_sms == 0) {
+    DeviceInfo d;
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      set_error("cudaDeviceGetAttribute failed");
+      return DSA_ERR_CUDA;
+    }
+    g_dev[dev] = d;
+  }
+  *out = g_dev[dev];
+  if (out->cc_major != 10 || out->cc_minor != 0) {
+    set_error("libdsa is built for sm_100a (B200); current device is sm_%d%d", out->cc_major, out->cc_minor);
+    return DSA_ERR_UNSUPPORTED;
+  }
+  return DSA_OK;
+}
+
+#define CHECK_ARG(cond, ...)          \
+  do {                                \
+    if (!(cond)) {                    \
+      set_error(__VA_ARGS__);         \
+      return DSA_ERR_INVALID_ARG;     \
+    }                                 \
+  } while (0)
+
+#define CHECK_SUP(cond, ...)          \
+  do {                                \
+    if (!(cond)) {                    \
+      set_error(__VA_ARGS__);         \
+      return DSA_ERR_UNSUPPORTED;     \
+    }                                 \
+  } while (0)
+
+static dsa_status_t check_batch(const dsa_batch_t *b) {
+  CHECK_ARG(b != nullptr, "batch descriptor is NULL");
+  CHECK_ARG(b->num_seqs >= 1, "num_seqs must be >= 1 (got %d)", b->num_seqs);
+  CHECK_SUP(b->page_size == 64, "page_size must be 64 (got %d)", b->page_size);
+  CHECK_ARG(b->num_blocks >= 1 && b->max_blocks_per_seq >= 1, "num_blocks and max_blocks_per_seq must be >= 1");
+  CHECK_ARG(b->block_table && b->seq_lens && b->cu_q, "block_table, seq_lens and cu_q are required");
+  CHECK_ARG(b->total_q >= 0, "total_q must be >= 0");
+  CHECK_ARG(b->max_seq_len >= 1 && b->max_q_per_seq >= 0, "max_seq_len must be >= 1");
+  CHECK_ARG(b->max_q_per_seq <= b->max_seq_len, "max_q_per_seq (%d) exceeds max_seq_len (%d)", b->max_q_per_seq,
+            b->max_seq_len);
+  CHECK_ARG((int64_t)b->total_q <= (int64_t)b->num_seqs * b->max_q_per_seq,
+            "total_q (%d) exceeds num_seqs * max_q_per_seq", b->total_q);
+  CHECK_ARG((int64_t)b->max_seq_len <= (int64_t)b->max_blocks_per_seq * b->page_size,
+            "max_seq_len (%d) exceeds max_blocks_per_seq * page_size", b->max_seq_len);
+  return DSA_OK;
+}
+
+static dsa_status_t check_ws(void *ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || ws_bytes < need) {
+    set_error("workspace of %zu bytes given, %zu needed", ws == nullptr ? (size_t)0 : ws_bytes, need);
+    return DSA_ERR_WORKSPACE;
+  }
+  CHECK_ARG(((uintptr_t)ws & 255) == 0, "workspace must be 256-byte aligned");
+  return DSA_OK;
+}
+
+static bool is_mla_attn(dsa_dtype_t dt, int H, int Dqk, int Dv, const void *v) {
+  return dt == DSA_BF16 && H == 128 && Dqk == 576 && Dv == 512 && v == nullptr;
+}
+static bool is_f32_attn(dsa_dtype_t dt, int H, int Dqk, int Dv, const void *v) {
+  return dt == DSA_F32 && H >= 1 && H <= 16 && Dqk >= 1 && Dqk <= 128 && Dv >= 1 && Dv <= 128 && v != nullptr;
+}
+
+static size_t attn_workspace_bytes(const dsa_batch_t *, int, int, int) { return kWsHeader; }
+
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+const char *dsa_version(void) { return "0.1.0"; }
+
+uint64_t dsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *dsa_last_error(void) { return g_err; }
+
+const char *dsa_status_string(dsa_status_t s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case DSA_ERR_WORKSPACE: return "workspace too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_DEVICE_CHECK: return "device-side index check failed";
+    case DSA_ERR_TIMEOUT: return "bounded device wait ran out";
+  }
+  return "unknown status";
+}
+
+dsa_status_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t *b, int32_t k, int32_t H, int32_t Dv,
+                                size_t *bytes) {
+  if (bytes == nullptr) {
+    set_error("bytes is NULL");
+    return DSA_ERR_INVALID_ARG;
+  }
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  switch (op) {
+    case DSA_OP_INDEXER: *bytes = kWsHeader; return DSA_OK;
+    case DSA_OP_TOPK: *bytes = topk_workspace_bytes(b->total_q, b->max_seq_len); return DSA_OK;
+    case DSA_OP_ATTN_PREFILL:
+    case DSA_OP_ATTN_DECODE: *bytes = attn_workspace_bytes(b, k, H, Dv); return DSA_OK;
+  }
+  set_error("unknown op %d", (int)op);
+  return DSA_ERR_INVALID_ARG;
+}
+
+dsa_status_t dsa_indexer_scores(const void *q_idx, dsa_dtype_t q_dt, const float *w, const void *k_idx_pool,
+                                dsa_dtype_t k_dt, const float *k_scale_pool, int32_t Hi, int32_t Di,
+                                const dsa_batch_t *b, float *scores, int64_t ld_scores, void *ws, size_t ws_bytes,
+                                void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  CHECK_ARG(q_idx && w && k_idx_pool && scores, "q_idx, w, k_idx_pool and scores are required");
+  CHECK_ARG(q_dt == k_dt, "query and key dtypes differ");
+  CHECK_ARG(ld_scores >= b->max_seq_len && ld_scores % 4 == 0,
+            "ld_scores (%lld) must be >= max_seq_len and a multiple of 4", (long long)ld_scores);
+  CHECK_ARG(((uintptr_t)scores & 15) == 0, "scores must be 16-byte aligned");
+  const bool mla = q_dt == DSA_FP8_E4M3 && Hi == 64 && Di == 128;
+  const bool f32 = q_dt == DSA_F32 && Hi >= 1 && Hi <= 16 && Di >= 1 && Di <= 128;
+  CHECK_SUP(mla || f32, "indexer supports e4m3 with Hi=64, Di=128 or f32 with Hi<=16, Di<=128");
+  CHECK_ARG(mla ? k_scale_pool != nullptr : k_scale_pool == nullptr,
+            "k_scale_pool is required for e4m3 keys and must be NULL for f32 keys");
+  if ((st = check_ws(ws, ws_bytes, kWsHeader)) != DSA_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;
+  return indexer_simt_launch(q_idx, q_dt, w, k_idx_pool, k_scale_pool, Hi, Di, b, scores, ld_scores,
+                             (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_batch_t *b, int32_t k, int32_t *idx,
+                      void *ws, size_t ws_bytes, void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  CHECK_ARG(scores && idx, "scores and idx are required");
+  CHECK_SUP(k >= 1 && k <= 16384, "k must be in [1, 16384] (got %d)", k);
+  CHECK_ARG(ld_scores >= b->max_seq_len && ld_scores % 4 == 0,
+            "ld_scores (%lld) must be >= max_seq_len and a multiple of 4", (long long)ld_scores);
+  CHECK_ARG(((uintptr_t)scores & 15) == 0, "scores must be 16-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, topk_workspace_bytes(b->total_q, b->max_seq_len))) != DSA_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;
+  return topk_launch(scores, ld_scores, b, k, idx, ws, (cudaStream_t)stream, dev.num_sms);
+}
+
+static dsa_status_t attn_common(bool decode, const void *q, dsa_dtype_t dt, const void *kv_pool, const void *v_pool,
+                                int32_t H, int32_t Dqk, int32_t Dv, float softmax_scale, const int32_t *idx,
+                                int32_t k, const dsa_batch_t *b, void *out, float *lse, void *ws, size_t ws_bytes,
+                                void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  CHECK_ARG(q && kv_pool && idx && out, "q, kv_pool, idx and out are required");
+  CHECK_ARG(k >= 1, "k must be >= 1");
+  CHECK_ARG(softmax_scale == softmax_scale && softmax_scale > 0.f && softmax_scale < 1e30f,
+            "softmax_scale must be finite and positive");
+  const bool mla = is_mla_attn(dt, H, Dqk, Dv, v_pool);
+  const bool f32 = is_f32_attn(dt, H, Dqk, Dv, v_pool);
+  CHECK_SUP(mla || f32,
+            "attention supports bf16 MLA (H=128, Dqk=576, Dv=512, V inside the latent row) or f32 with "
+            "H<=16, Dqk<=128, Dv<=128 and a separate V cache");
+  if (decode) CHECK_ARG(b->total_q == b->num_seqs && b->max_q_per_seq == 1,
+                        "decode needs exactly one query row per sequence");
+  if ((st = check_ws(ws, ws_bytes, attn_workspace_bytes(b, k, H, Dv))) != DSA_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;
+  return attn_simt_launch(q, dt, kv_pool, v_pool, H, Dqk, Dv, softmax_scale, idx, k, b, out, lse,
+                          (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_sparse_attn_prefill(const void *q, dsa_dtype_t dt, const void *kv_pool, const void *v_pool, int32_t H,
+                                     int32_t Dqk, int32_t Dv, float softmax_scale, const int32_t *idx, int32_t k,
+                                     const dsa_batch_t *b, void *out, float *lse, void *ws, size_t ws_bytes,
+                                     void *stream) {
+  return attn_common(false, q, dt, kv_pool, v_pool, H, Dqk, Dv, softmax_scale, idx, k, b, out, lse, ws, ws_bytes,
+                     stream);
+}
+
+dsa_status_t dsa_sparse_attn_decode(const void *q, dsa_dtype_t dt, const void *kv_pool, const void *v_pool, int32_t H,
+                                    int32_t Dqk, int32_t Dv, float softmax_scale, const int32_t *idx, int32_t k,
+                                    const dsa_batch_t *b, void *out, float *lse, void *ws, size_t ws_bytes,
+                                    void *stream) {
+  return attn_common(true, q, dt, kv_pool, v_pool, H, Dqk, Dv, softmax_scale, idx, k, b, out, lse, ws, ws_bytes,
+                     stream);
+}
+
+dsa_status_t dsa_read_device_status(void *ws, void *stream) {
+  if (ws == nullptr) {
+    set_error("workspace is NULL");
+    return DSA_ERR_INVALID_ARG;
+  }
+  uint32_t word = 0;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess ||
+      cudaMemcpy(&word, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(ws, 0, 4) != cudaSuccess) {
+    set_error("reading the device status word failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return DSA_ERR_CUDA;
+  }
+  if (word & kStatusTimeout) {
+    set_error("a bounded device wait ran out (status 0x%x)", word);
+    return DSA_ERR_TIMEOUT;
+  }
+  if (word & kStatusBadIndex) {
+    set_error("a kernel met an out-of-range block id or index (status 0x%x)", word);
+    return DSA_ERR_DEVICE_CHECK;
+  }
+  return DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,378 @@
+// Exact per-row top-k over fp32 indexer scores (radix select in shared memory).
+//
+// Selection order: score descending, token position ascending (the lower position wins a tie;
+// -0 == +0).  Scores are compared as order-preserving u32 keys, so the selection is exact.
+// The k-th key T is found digit by digit (11 + 11 + 10 bits) with shared-memory histograms; every
+// key > T is selected plus the lowest-positioned keys == T until k are taken.  The result is
+// written in ascending position order by a block-wide ordered compaction, so no sort is needed.
+//
+// Rows are grouped by row, buffered in shared memory and read with 16-byte vector loads, the
+// structure the pages credit for their index-selection speed-up ("Engineering Practices for
+// Day-0 Adaptation of Million-Token Context Models on Domestic AI Chips", Four Key Layers 1).
+//
+// Two regimes:
+//   A) n <= kTopkSmemCap candidates: one CTA per row, the row's keys staged once in shared memory,
+//      all digit passes and the ordered write from shared memory.  One launch.
+//   B) longer rows (a million-token decode): the row is split into segments of kTopkSeg keys over
+//      a persistent grid; each digit pass is one launch whose CTAs add segment histograms into a
+//      per-row global histogram, and the last CTA of a row to finish (atomic counter, no waiting)
+//      picks the digit.  Then a count launch and an ordered-write launch.  No CTA ever waits for
+//      another.
+#include "common.cuh"
+
+namespace dsa {
+
+constexpr int kTopkSmemCap = 49152;
+constexpr int kTopkThreadsA = 1024;
+constexpr int kTopkSeg = 8192;
+constexpr int kTopkThreadsB = 512;
+constexpr int kRadixBins = 2048;
+
+struct TopkRowState {
+  uint32_t prefix, pmask, k_rem, done;
+};
+
+// Workspace layout for regime B (after the 256-byte header):
+//   [0]            u32 long-row count
+//   [64 ..)        i32 long-row list [total_q]
+//   state          TopkRowState [total_q]
+//   hist           u32 [total_q][2048]
+//   segcnt         uint2 [total_q][max_segs]   (gt, eq) per segment
+struct TopkWs {
+  uint32_t *count;
+  int32_t *list;
+  TopkRowState *state;
+  uint32_t *hist;
+  uint2 *segcnt;
+  int max_segs;
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline int topk_max_segs(int max_seq_len) { return (max_seq_len + kTopkSeg - 1) / kTopkSeg; }
+
+size_t topk_workspace_bytes(int total_q, int max_seq_len) {
+  size_t bytes = kWsHeader;
+  if (max_seq_len <= kTopkSmemCap) return bytes;
+  size_t off = 64 + align_up((size_t)total_q * 4, 256);
+  off += align_up((size_t)total_q * sizeof(TopkRowState), 256);
+  off += align_up((size_t)total_q * kRadixBins * 4, 256);
+  off += align_up((size_t)total_q * topk_max_segs(max_seq_len) * sizeof(uint2), 256);
+  return bytes + off;
+}
+
+static TopkWs topk_ws_view(void *ws, int total_q, int max_seq_len) {
+  char *p = (char *)ws + kWsHeader;
+  TopkWs w;
+  w.count = (uint32_t *)p;
+  w.list = (int32_t *)(p + 64);
+  size_t off = 64 + align_up((size_t)total_q * 4, 256);
+  w.state = (TopkRowState *)(p + off);
+  off += align_up((size_t)total_q * sizeof(TopkRowState), 256);
+  w.hist = (uint32_t *)(p + off);
+  off += align_up((size_t)total_q * kRadixBins * 4, 256);
+  w.segcnt = (uint2 *)(p + off);
+  w.max_segs = topk_max_segs(max_seq_len);
+  return w;
+}
+
+// Threshold digit: among bins taken in descending order, the bin where the running count first
+// reaches k_rem.  Returns the bin and the count of keys in higher bins.  All threads participate.
+__device__ void find_threshold_bin(const uint32_t *hist, int nbins, uint32_t k_rem, uint32_t *tmp,
+                                   int *s_bin, uint32_t *s_above) {
+  const int per = (nbins + blockDim.x - 1) / blockDim.x;
+  const int d0 = threadIdx.x * per;
+  uint32_t local = 0;
+  for (int d = d0; d < d0 + per && d < nbins; ++d) local += hist[nbins - 1 - d];
+  uint32_t before = block_exclusive_scan(local, tmp, nullptr);
+  uint32_t run = before;
+  for (int d = d0; d < d0 + per && d < nbins; ++d) {
+    uint32_t c = hist[nbins - 1 - d];
+    if (run < k_rem && run + c >= k_rem) {
+      *s_bin = nbins - 1 - d;
+      *s_above = run;
+    }
+    run += c;
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------------------------------------
+// Regime A
+// ------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kTopkThreadsA)
+topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, int k,
+                      int32_t *__restrict__ idx, TopkWs lw, int register_long) {
+  extern __shared__ __align__(16) uint32_t sm[];
+  uint32_t *keys = sm;
+  uint32_t *hist = sm + kTopkSmemCap;
+  uint32_t *tmp = hist + kRadixBins;
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above;
+
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, bs = blockDim.x;
+  int b;
+  const int n = pos_of_row(bv, row, &b) + 1;
+  int32_t *out = idx + (int64_t)row * k;
+
+  if (n > kTopkSmemCap) {
+    // long row: hand it to regime B, initialise its state and histogram
+    if (register_long) {
+      if (tid == 0) {
+        uint32_t slot = atomicAdd(lw.count, 1u);
+        lw.list[slot] = row;
+        lw.state[row] = TopkRowState{0u, 0u, (uint32_t)k, 0u};
+      }
+      for (int i = tid; i < kRadixBins; i += bs) lw.hist[(int64_t)row * kRadixBins + i] = 0u;
+    }
+    return;
+  }
+  if (n <= k) {
+    for (int j = tid; j < k; j += bs) out[j] = j < n ? j : -1;
+    return;
+  }
+
+  const float *src = scores + (int64_t)row * ld;
+  const int n4 = n >> 2;
+  const float4 *src4 = reinterpret_cast<const float4 *>(src);
+  for (int i = tid; i < n4; i += bs) {
+    float4 v = __ldg(src4 + i);
+    uint4 u = make_uint4(ordered_key(v.x), ordered_key(v.y), ordered_key(v.z), ordered_key(v.w));
+    reinterpret_cast<uint4 *>(keys)[i] = u;
+  }
+  for (int i = 4 * n4 + tid; i < n; i += bs) keys[i] = ordered_key(__ldg(src + i));
+  __syncthreads();
+
+  uint32_t prefix = 0u, pmask = 0u, k_rem = (uint32_t)k;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nb = pass == 2 ? 1024 : 2048;
+    for (int i = tid; i < nb; i += bs) hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += bs) {
+      uint32_t u = keys[i];
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    find_threshold_bin(hist, nb, k_rem, tmp, &s_bin, &s_above);
+    prefix |= (uint32_t)s_bin << shift;
+    pmask |= (uint32_t)(nb - 1) << shift;
+    k_rem -= s_above;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;
+
+  // ordered compaction: each thread owns a contiguous range of positions
+  const int per = (n + bs - 1) / bs;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  uint32_t gt = 0, eq = 0;
+  for (int i = lo; i < hi; ++i) {
+    uint32_t u = keys[i];
+    gt += u > T;
+    eq += u == T;
+  }
+  uint32_t eq_before = block_exclusive_scan(eq, tmp, nullptr);
+  uint32_t take_eq = k_rem > eq_before ? min(eq, k_rem - eq_before) : 0u;
+  uint32_t off = block_exclusive_scan(gt + take_eq, tmp, nullptr);
+  uint32_t e = 0;
+  for (int i = lo; i < hi; ++i) {
+    uint32_t u = keys[i];
+    bool sel = u > T;
+    if (u == T) { sel = e < take_eq; ++e; }
+    if (sel && off < (uint32_t)k) out[off++] = i;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Regime B (persistent over (long row, segment) items)
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ bool long_item(const TopkWs &w, const BatchView &bv, int item, int *row, int *seg,
+                                          int *n, int *nseg) {
+  const int r_i = item / w.max_segs;
+  *seg = item % w.max_segs;
+  *row = w.list[r_i];
+  int b;
+  *n = pos_of_row(bv, *row, &b) + 1;
+  *nseg = (*n + kTopkSeg - 1) / kTopkSeg;
+  return *seg < *nseg;
+}
+
+// stage one segment's keys in shared memory; returns its length
+__device__ int stage_segment(const float *__restrict__ scores, int64_t ld, int row, int seg, int n, uint32_t *keys) {
+  const int lo = seg * kTopkSeg;
+  const int len = min(kTopkSeg, n - lo);
+  const float *src = scores + (int64_t)row * ld + lo;
+  const int l4 = len >> 2;
+  for (int i = threadIdx.x; i < l4; i += blockDim.x) {
+    float4 v = __ldg(reinterpret_cast<const float4 *>(src) + i);
+    reinterpret_cast<uint4 *>(keys)[i] =
+        make_uint4(ordered_key(v.x), ordered_key(v.y), ordered_key(v.z), ordered_key(v.w));
+  }
+  for (int i = 4 * l4 + threadIdx.x; i < len; i += blockDim.x) keys[i] = ordered_key(__ldg(src + i));
+  __syncthreads();
+  return len;
+}
+
+__global__ void __launch_bounds__(kTopkThreadsB)
+topk_long_hist_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, TopkWs w, int pass) {
+  __shared__ __align__(16) uint32_t keys[kTopkSeg];
+  __shared__ uint32_t hist[kRadixBins];
+  __shared__ uint32_t tmp[64];
+  __shared__ int s_bin, s_last;
+  __shared__ uint32_t s_above;
+  const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+  const int nb = pass == 2 ? 1024 : 2048;
+  const int items = (int)(*w.count) * w.max_segs;
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    int row, seg, n, nseg;
+    if (!long_item(w, bv, item, &row, &seg, &n, &nseg)) continue;
+    const TopkRowState st = w.state[row];
+    const int len = stage_segment(scores, ld, row, seg, n, keys);
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) hist[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < len; i += blockDim.x) {
+      uint32_t u = keys[i];
+      if ((u & st.pmask) == st.prefix) atomicAdd(&hist[(u >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    uint32_t *gh = w.hist + (int64_t)row * kRadixBins;
+    for (int i = threadIdx.x; i < nb; i += blockDim.x)
+      if (hist[i]) atomicAdd(gh + i, hist[i]);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&w.state[row].done, 1u) == (uint32_t)(nseg - 1);
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        hist[i] = __ldcg(gh + i);
+        gh[i] = 0u;
+      }
+      __syncthreads();
+      find_threshold_bin(hist, nb, st.k_rem, tmp, &s_bin, &s_above);
+      if (threadIdx.x == 0) {
+        TopkRowState ns;
+        ns.prefix = st.prefix | ((uint32_t)s_bin << shift);
+        ns.pmask = st.pmask | ((uint32_t)(nb - 1) << shift);
+        ns.k_rem = st.k_rem - s_above;
+        ns.done = 0u;
+        w.state[row] = ns;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(kTopkThreadsB)
+topk_long_count_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, TopkWs w) {
+  __shared__ __align__(16) uint32_t keys[kTopkSeg];
+  __shared__ uint32_t tmp[64];
+  const int items = (int)(*w.count) * w.max_segs;
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    int row, seg, n, nseg;
+    if (!long_item(w, bv, item, &row, &seg, &n, &nseg)) continue;
+    const uint32_t T = w.state[row].prefix;
+    const int len = stage_segment(scores, ld, row, seg, n, keys);
+    uint32_t gt = 0, eq = 0;
+    for (int i = threadIdx.x; i < len; i += blockDim.x) {
+      gt += keys[i] > T;
+      eq += keys[i] == T;
+    }
+    uint32_t tg, te;
+    block_exclusive_scan(gt, tmp, &tg);
+    block_exclusive_scan(eq, tmp, &te);
+    if (threadIdx.x == 0) w.segcnt[(int64_t)row * w.max_segs + seg] = make_uint2(tg, te);
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(kTopkThreadsB)
+topk_long_write_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, TopkWs w, int k,
+                       int32_t *__restrict__ idx) {
+  __shared__ __align__(16) uint32_t keys[kTopkSeg];
+  __shared__ uint32_t tmp[64];
+  __shared__ uint32_t s_gt_before, s_eq_before;
+  const int items = (int)(*w.count) * w.max_segs;
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    int row, seg, n, nseg;
+    if (!long_item(w, bv, item, &row, &seg, &n, &nseg)) continue;
+    const TopkRowState st = w.state[row];
+    const uint32_t T = st.prefix, k_rem = st.k_rem;
+    // counts of the earlier segments of this row
+    uint32_t g = 0, e = 0;
+    for (int s = threadIdx.x; s < seg; s += blockDim.x) {
+      uint2 c = w.segcnt[(int64_t)row * w.max_segs + s];
+      g += c.x;
+      e += c.y;
+    }
+    uint32_t tg, te;
+    block_exclusive_scan(g, tmp, &tg);
+    block_exclusive_scan(e, tmp, &te);
+    if (threadIdx.x == 0) { s_gt_before = tg; s_eq_before = te; }
+    const int len = stage_segment(scores, ld, row, seg, n, keys);   // syncs
+    const uint32_t seg_gt_before = s_gt_before, seg_eq_before = s_eq_before;
+    const int per = (len + blockDim.x - 1) / blockDim.x;
+    const int lo = min(len, (int)threadIdx.x * per), hi = min(len, lo + per);
+    uint32_t gt = 0, eq = 0;
+    for (int i = lo; i < hi; ++i) {
+      gt += keys[i] > T;
+      eq += keys[i] == T;
+    }
+    const uint32_t eq_before = seg_eq_before + block_exclusive_scan(eq, tmp, nullptr);
+    const uint32_t take_eq = k_rem > eq_before ? min(eq, k_rem - eq_before) : 0u;
+    // selected before this thread = every gt of earlier segments + the eq ones taken there
+    const uint32_t eq_taken_before_seg = min(seg_eq_before, k_rem);
+    uint32_t off = seg_gt_before + eq_taken_before_seg + block_exclusive_scan(gt + take_eq, tmp, nullptr);
+    int32_t *out = idx + (int64_t)row * k;
+    uint32_t c = 0;
+    const int base = seg * kTopkSeg;
+    for (int i = lo; i < hi; ++i) {
+      uint32_t u = keys[i];
+      bool sel = u > T;
+      if (u == T) { sel = c < take_eq; ++c; }
+      if (sel && off < (uint32_t)k) out[off++] = base + i;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// host entry
+// ------------------------------------------------------------------------------------------------
+dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx, void *ws,
+                         cudaStream_t stream, int num_sms) {
+  BatchView bv = view_of(b);
+  const bool has_long = b->max_seq_len > kTopkSmemCap;
+  TopkWs lw{};
+  if (has_long) {
+    lw = topk_ws_view(ws, b->total_q, b->max_seq_len);
+    if (cudaMemsetAsync(lw.count, 0, 4, stream) != cudaSuccess) {
+      set_error("topk: cudaMemsetAsync failed");
+      return DSA_ERR_CUDA;
+    }
+  }
+  const size_t smem = (size_t)(kTopkSmemCap + kRadixBins + 64) * 4;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attr_set = true;
+  }
+  topk_rows_smem_kernel<<<b->total_q, kTopkThreadsA, smem, stream>>>(scores, ld, bv, k, idx, lw, has_long ? 1 : 0);
+  DSA_LAUNCH_CHECK("topk_rows_smem_kernel");
+  if (has_long) {
+    const int grid = max(num_sms * 4, topk_max_segs(b->max_seq_len));   // one segment per CTA per row
+    for (int pass = 0; pass < 3; ++pass) {
+      topk_long_hist_kernel<<<grid, kTopkThreadsB, 0, stream>>>(scores, ld, bv, lw, pass);
+      DSA_LAUNCH_CHECK("topk_long_hist_kernel");
+    }
+    topk_long_count_kernel<<<grid, kTopkThreadsB, 0, stream>>>(scores, ld, bv, lw);
+    DSA_LAUNCH_CHECK("topk_long_count_kernel");
+    topk_long_write_kernel<<<grid, kTopkThreadsB, 0, stream>>>(scores, ld, bv, lw, k, idx);
+    DSA_LAUNCH_CHECK("topk_long_write_kernel");
+  }
+  return DSA_OK;
+}
+
+}  // namespace dsa

@@ -1,0 +1,89 @@
+"""Device-resident batch and the three-call path (indexer -> top-k -> sparse attention).
+
+`DeviceBatch` uploads a host `Workload` (see workloads.py) into device memory with torch
+(plumbing only) and owns the output buffers and one workspace; `run()` enqueues the
+three C-ABI calls on one stream.  Nothing here computes any part of the method.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+
+def _dev(a, device):
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+class DeviceBatch:
+    """One workload resident in HBM plus its outputs.
+
+    scores [total_q, ld] f32, idx [total_q, k] int32, out [total_q, H, Dv] (bf16 or f32),
+    lse [total_q, H] f32.  `decode` picks dsa_sparse_attn_decode (every sequence has one
+    query row) over dsa_sparse_attn_prefill; default: decode when that holds.
+    """
+
+    def __init__(self, wl, device="cuda", decode=None, inputs=None):
+        self.wl = wl
+        self.device = torch.device(device)
+        dv = self.device
+        mla = wl.kind == "mla"
+        self.mla = mla
+        self.dt = B.DSA_BF16 if mla else B.DSA_F32
+        self.idx_dt = B.DSA_FP8_E4M3 if mla else B.DSA_F32
+        if inputs is None:
+            inputs = self.upload_inputs(wl, dv)
+        self.inputs = inputs
+        for k_, v_ in inputs.items():
+            setattr(self, k_, v_)
+        self.ld = int((wl.max_seq_len + 3) // 4 * 4)
+        T = wl.total_q
+        self.batch = B.make_batch(self.block_table, self.seq_lens, self.cu_q, num_blocks=wl.num_blocks,
+                                  page_size=wl.page_size, total_q=T, max_q_per_seq=wl.max_q_per_seq,
+                                  max_seq_len=wl.max_seq_len)
+        self.scores = torch.empty((T, self.ld), dtype=torch.float32, device=dv)
+        self.idx = torch.empty((T, wl.topk), dtype=torch.int32, device=dv)
+        self.out = torch.empty((T, wl.H, wl.Dv), dtype=torch.bfloat16 if mla else torch.float32, device=dv)
+        self.lse = torch.empty((T, wl.H), dtype=torch.float32, device=dv)
+        if decode is None:
+            decode = bool(np.all(wl.q_lens == 1))
+        self.decode = decode
+        op_attn = B.DSA_OP_ATTN_DECODE if decode else B.DSA_OP_ATTN_PREFILL
+        self.ws_bytes = max(B.dsa_workspace_size(B.DSA_OP_INDEXER, self.batch),
+                            B.dsa_workspace_size(B.DSA_OP_TOPK, self.batch, wl.topk),
+                            B.dsa_workspace_size(op_attn, self.batch, wl.topk, wl.H, wl.Dv))
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dv)
+
+    @staticmethod
+    def upload_inputs(wl, dv):
+        """Device copies of every input array of the workload (the cache pools included)."""
+        return dict(
+            q=_dev(wl.q, dv), kv_pool=_dev(wl.kv_pool, dv), v_pool=_dev(wl.v_pool, dv), qI=_dev(wl.qI, dv),
+            kI_pool=_dev(wl.kI_pool, dv), kS_pool=_dev(wl.kS_pool, dv), w=_dev(wl.w, dv),
+            block_table=_dev(wl.block_table.astype(np.int32), dv), seq_lens=_dev(wl.seq_lens.astype(np.int32), dv),
+            cu_q=_dev(wl.cu_q.astype(np.int32), dv))
+
+    # individual steps --------------------------------------------------------------------------
+    def indexer(self, stream=None):
+        wl = self.wl
+        B.dsa_indexer_scores(self.qI, self.idx_dt, self.w, self.kI_pool, self.idx_dt, self.kS_pool, wl.Hi, wl.Di,
+                             self.batch, self.scores, self.ld, self.ws, self.ws_bytes, stream)
+
+    def topk(self, stream=None, scores=None):
+        B.dsa_topk(self.scores if scores is None else scores, self.ld, self.batch, self.wl.topk, self.idx, self.ws,
+                   self.ws_bytes, stream)
+
+    def attention(self, stream=None, idx=None):
+        wl = self.wl
+        fn = B.dsa_sparse_attn_decode if self.decode else B.dsa_sparse_attn_prefill
+        fn(self.q, self.dt, self.kv_pool, self.v_pool, wl.H, wl.Dqk, wl.Dv, wl.softmax_scale,
+           self.idx if idx is None else idx, wl.topk, self.batch, self.out, self.lse, self.ws, self.ws_bytes, stream)
+
+    def run(self, stream=None):
+        self.indexer(stream)
+        self.topk(stream)
+        self.attention(stream)
+
+    def check_status(self, stream=None):
+        B.dsa_read_device_status(self.ws, stream)

@@ -1,0 +1,96 @@
+"""Host-side ABI checks (no GPU): the library loads, exports every declared entry point, and
+rejects bad arguments before touching the device."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from sparse_attention_long_dsa_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for f in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"DSA_API\s+[\w\s\*]+?\b(dsa_\w+)\s*\(", text)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.load()
+    names = _declared()
+    assert set(B.EXPORTS) <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    lib = B.load()
+    for s in range(7):
+        assert lib.dsa_status_string(s)
+    assert B.dsa_version() == "0.1.0"
+
+
+def _batch(**kw):
+    d = dict(num_seqs=2, page_size=64, num_blocks=4, max_blocks_per_seq=2, block_table=1 << 20, seq_lens=1 << 21,
+             cu_q=1 << 22, total_q=3, max_q_per_seq=2, max_seq_len=100)
+    d.update(kw)
+    return B.dsa_batch_t(**d)
+
+
+def test_workspace_size_host_only():
+    b = _batch()
+    assert B.dsa_workspace_size(B.DSA_OP_INDEXER, b) >= 256
+    assert B.dsa_workspace_size(B.DSA_OP_TOPK, b, 2048) >= 256
+    big = _batch(max_seq_len=1 << 20, max_blocks_per_seq=1 << 14, total_q=2)
+    assert B.dsa_workspace_size(B.DSA_OP_TOPK, big, 2048) > 2 * 2048 * 4
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(page_size=128), B.DSA_ERR_UNSUPPORTED),
+    (dict(num_seqs=0), B.DSA_ERR_INVALID_ARG),
+    (dict(block_table=0), B.DSA_ERR_INVALID_ARG),
+    (dict(max_seq_len=129), B.DSA_ERR_INVALID_ARG),        # > max_blocks_per_seq * page_size
+    (dict(total_q=5), B.DSA_ERR_INVALID_ARG),             # > num_seqs * max_q_per_seq
+    (dict(max_q_per_seq=200), B.DSA_ERR_INVALID_ARG),     # > max_seq_len
+])
+def test_batch_validation(bad, status):
+    with pytest.raises(B.DSAError) as e:
+        B.dsa_workspace_size(B.DSA_OP_TOPK, _batch(**bad), 16)
+    assert e.value.status == status
+
+
+def test_compute_calls_reject_before_launch():
+    b = _batch()
+    P = 1 << 24
+    with pytest.raises(B.DSAError) as e:       # unsupported indexer dims
+        B.dsa_indexer_scores(P, B.DSA_FP8_E4M3, P, P, B.DSA_FP8_E4M3, P, 32, 128, b, P, 128, P, 1 << 20, 0)
+    assert e.value.status == B.DSA_ERR_UNSUPPORTED
+    with pytest.raises(B.DSAError) as e:       # ld_scores too small
+        B.dsa_topk(P, 64, b, 16, P, P, 1 << 20, 0)
+    assert e.value.status == B.DSA_ERR_INVALID_ARG
+    with pytest.raises(B.DSAError) as e:       # dtype mix
+        B.dsa_indexer_scores(P, B.DSA_F32, P, P, B.DSA_FP8_E4M3, None, 2, 32, b, P, 128, P, 1 << 20, 0)
+    assert e.value.status == B.DSA_ERR_INVALID_ARG
+    with pytest.raises(B.DSAError) as e:       # attention shape outside both paths
+        B.dsa_sparse_attn_prefill(P, B.DSA_BF16, P, None, 64, 576, 512, 0.1, P, 16, b, P, P, P, 1 << 20, 0)
+    assert e.value.status == B.DSA_ERR_UNSUPPORTED
+    with pytest.raises(B.DSAError) as e:       # misaligned workspace
+        B.dsa_topk(P, 128, b, 16, P, P + 8, 1 << 20, 0)
+    assert e.value.status == B.DSA_ERR_INVALID_ARG
+    with pytest.raises(B.DSAError) as e:       # decode with several rows per sequence
+        B.dsa_sparse_attn_decode(P, B.DSA_BF16, P, None, 128, 576, 512, 0.1, P, 16, b, P, P, P, 1 << 20, 0)
+    assert e.value.status == B.DSA_ERR_INVALID_ARG
+    assert "one query row" in B.load().dsa_last_error().decode()
+
+
+def test_nonfinite_scale_rejected():
+    b = _batch(total_q=2, max_q_per_seq=1)
+    P = 1 << 24
+    with pytest.raises(B.DSAError) as e:
+        B.dsa_sparse_attn_decode(P, B.DSA_BF16, P, None, 128, 576, 512, float("nan"), P, 16, b, P, P, P, 1 << 20, 0)
+    assert e.value.status == B.DSA_ERR_INVALID_ARG

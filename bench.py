@@ -319,16 +319,18 @@ def cpu_baseline(wl, budget_s=15.0, rows=None):
     rng = np.random.default_rng(0)
     if rows is None and len(order) > 64:
         order = sorted(rng.choice(wl.total_q, 64, replace=False).tolist())
-    done, t0 = 0, time.perf_counter()
-    for r in order:
-        oracle.run_rows(wl, [r])
-        done += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
+    done, t0, passes = 0, time.perf_counter(), 0
+    while time.perf_counter() - t0 < budget_s:
+        for r in order:
+            oracle.run_rows(wl, [r])
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        passes += 1
     dt = time.perf_counter() - t0
     return {"value": done / dt, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{done} query rows of {wl.name} (full path per row: scores, top-k, attention), "
-                      f"{dt:.1f} s wall"}
+            "sample": f"{done} query-row evaluations over {len(order)} rows of {wl.name} (full path per row: "
+                      f"scores, top-k, attention), {dt:.1f} s wall"}
 
 
 def run_reference(args, rank, world):

@@ -67,7 +67,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     if force or any(changed for _, changed in results) or not os.path.exists(LIB) or \
             os.path.getmtime(LIB) < _newest(objs):
         tmp = LIB + ".tmp"
-        cmd = [cc, *ARCH, "-shared", "-o", tmp, *objs, "-Xcompiler", "-fPIC", "-lcuda"]
+        cmd = [cc, *ARCH, "-shared", "-o", tmp, *objs, "-Xcompiler", "-fPIC"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

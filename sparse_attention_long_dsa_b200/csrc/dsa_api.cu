@@ -17,6 +17,10 @@ size_t topk_workspace_bytes(int total_q, int max_seq_len);
 dsa_status_t indexer_simt_launch(const void *qI, dsa_dtype_t dt, const float *w, const void *kpool,
                                  const float *kscale, int Hi, int Di, const dsa_batch_t *b, float *scores,
                                  int64_t ld, cudaStream_t stream);
+dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t *kpool, const float *kscale,
+                               const dsa_batch_t *b, float *scores, int64_t ld, void *ws, cudaStream_t stream,
+                               int num_sms);
+size_t indexer_workspace_bytes(int num_seqs, int total_q);
 dsa_status_t attn_simt_launch(const void *q, dsa_dtype_t dt, const void *kv, const void *v, int H, int Dqk, int Dv,
                               float scale, const int32_t *idx, int k, const dsa_batch_t *b, void *out, float *lse,
                               cudaStream_t stream);
@@ -152,7 +156,7 @@ dsa_status_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t *b, int32_t k, in
   dsa_status_t st = check_batch(b);
   if (st != DSA_OK) return st;
   switch (op) {
-    case DSA_OP_INDEXER: *bytes = kWsHeader; return DSA_OK;
+    case DSA_OP_INDEXER: *bytes = indexer_workspace_bytes(b->num_seqs, b->total_q); return DSA_OK;
     case DSA_OP_TOPK: *bytes = topk_workspace_bytes(b->total_q, b->max_seq_len); return DSA_OK;
     case DSA_OP_ATTN_PREFILL:
     case DSA_OP_ATTN_DECODE: *bytes = attn_workspace_bytes(b, k, H, Dv); return DSA_OK;
@@ -177,10 +181,15 @@ dsa_status_t dsa_indexer_scores(const void *q_idx, dsa_dtype_t q_dt, const float
   CHECK_SUP(mla || f32, "indexer supports e4m3 with Hi=64, Di=128 or f32 with Hi<=16, Di<=128");
   CHECK_ARG(mla ? k_scale_pool != nullptr : k_scale_pool == nullptr,
             "k_scale_pool is required for e4m3 keys and must be NULL for f32 keys");
-  if ((st = check_ws(ws, ws_bytes, kWsHeader)) != DSA_OK) return st;
+  CHECK_ARG((((uintptr_t)q_idx | (uintptr_t)w | (uintptr_t)k_idx_pool | (uintptr_t)k_scale_pool) & 15) == 0,
+            "q_idx, w, k_idx_pool and k_scale_pool must be 16-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, indexer_workspace_bytes(b->num_seqs, b->total_q))) != DSA_OK) return st;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
   if (b->total_q == 0) return DSA_OK;
+  if (mla)
+    return indexer_tc_launch((const uint8_t *)q_idx, w, (const uint8_t *)k_idx_pool, k_scale_pool, b, scores,
+                             ld_scores, ws, (cudaStream_t)stream, dev.num_sms);
   return indexer_simt_launch(q_idx, q_dt, w, k_idx_pool, k_scale_pool, Hi, Di, b, scores, ld_scores,
                              (cudaStream_t)stream);
 }

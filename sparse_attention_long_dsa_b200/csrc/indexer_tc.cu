@@ -1,0 +1,425 @@
+// FP8 indexer scores on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+//   scores[row, s] = kS[s] * sum_j w[row, j] * max(0, sum_d qI[row, j, d] * kI8[s, d]),  s <= pos(row)
+//
+// ("Day-0 Adaptation for LLMs: Implementing Sparse Attention and Low-Precision Weights", III.1:
+// the lightweight indexer scores each query against every historical token, at higher precision
+// than attention.  The FP8 products are exact and accumulate in fp32; the scorer's form is the one
+// this library takes for the pages' open "indexer(q, kv_meta)".)  kS is factored out of the ReLU,
+// which is exact because kS > 0 and ReLU is positively homogeneous.
+//
+// Contraction per tile: D[128 keys, 64*R] = K[128 keys, 128] x Q[64*R, 128]^T with R <= 4 query
+// rows of one sequence sharing the keys (prefill / chunked prefill) or R = 1 (decode).  Keys are the
+// M dimension so that each TMEM lane holds one key and the weighted ReLU sum over heads is a
+// per-thread reduction with no shuffles.  A 128-key tile is two 64-token pages fetched by TMA through
+// the block table (128-byte swizzle, the layout the MMA descriptor reads).
+//
+// Warp roles (192 threads, persistent, one CTA per SM):
+//   warp 0       TMA producer: query rows + weights of a row group, then key tiles into an 8-stage ring
+//   warp 1       allocates 512 TMEM columns; lane 0 issues 4 MMAs (K = 32 each) per tile into one of two
+//                256-column accumulators and commits them to the ring / accumulator barriers
+//   warps 2..5   epilogue: tcgen05.ld 64 heads per row, ReLU, weight, sum, key scale, causal store
+// Work units are (row group, key tile) pairs in group order, split evenly over the CTAs; a one-CTA
+// plan kernel enumerates the groups and their tile counts in the workspace first.
+#include "tc.cuh"
+
+namespace dsa {
+
+constexpr int kIdxTile = 128;
+constexpr int kIdxRows = 4;
+constexpr int kIdxStages = 8;
+constexpr int kIdxThreads = 192;
+constexpr int kIdxHi = 64, kIdxDi = 128;
+constexpr uint32_t kIdxTileBytes = kIdxTile * kIdxDi;         // 16 KB
+constexpr uint32_t kIdxPageBytes = 64 * kIdxDi;               // 8 KB
+constexpr uint32_t kIdxBSlotBytes = kIdxRows * kIdxHi * kIdxDi;  // 32 KB
+constexpr uint32_t kIdxWSlotBytes = kIdxRows * kIdxHi * 4;       // 1 KB
+
+// ------------------------------------------------------------------------------------------------ plan
+// workspace (after the header): int32 [0] = G, [1] = U, then arrays
+struct IdxPlanView {
+  int32_t *hdr;
+  int32_t *seq_goff;      // [num_seqs + 1]
+  int32_t *g_row0;        // [total_q]
+  int32_t *g_nrows;       // [total_q]
+  int32_t *g_seq;         // [total_q]
+  int32_t *tile_prefix;   // [total_q + 1]
+};
+
+static size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t indexer_workspace_bytes(int num_seqs, int total_q) {
+  return kWsHeader + 256 + al256((size_t)(num_seqs + 1) * 4) + 3 * al256((size_t)total_q * 4) +
+         al256((size_t)(total_q + 1) * 4);
+}
+
+static IdxPlanView plan_view(void *ws, int num_seqs, int total_q) {
+  char *p = (char *)ws + kWsHeader;
+  IdxPlanView v;
+  v.hdr = (int32_t *)p;
+  p += 256;
+  v.seq_goff = (int32_t *)p;
+  p += al256((size_t)(num_seqs + 1) * 4);
+  v.g_row0 = (int32_t *)p;
+  p += al256((size_t)total_q * 4);
+  v.g_nrows = (int32_t *)p;
+  p += al256((size_t)total_q * 4);
+  v.g_seq = (int32_t *)p;
+  p += al256((size_t)total_q * 4);
+  v.tile_prefix = (int32_t *)p;
+  return v;
+}
+
+__global__ void __launch_bounds__(1024) indexer_plan_kernel(BatchView bv, IdxPlanView pv) {
+  __shared__ uint32_t tmp[64];
+  __shared__ uint32_t s_carry;
+  const int tid = threadIdx.x;
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  // groups per sequence -> seq_goff (exclusive prefix)
+  for (int base = 0; base < bv.num_seqs; base += blockDim.x) {
+    const int b = base + tid;
+    uint32_t g = 0;
+    if (b < bv.num_seqs) {
+      const int nb = __ldg(bv.cu_q + b + 1) - __ldg(bv.cu_q + b);
+      g = (nb + kIdxRows - 1) / kIdxRows;
+    }
+    uint32_t tot;
+    const uint32_t ex = block_exclusive_scan(g, tmp, &tot);
+    if (b < bv.num_seqs) pv.seq_goff[b] = (int)(s_carry + ex);
+    __syncthreads();
+    if (tid == 0) s_carry += tot;
+    __syncthreads();
+  }
+  const int G = (int)s_carry;
+  if (tid == 0) pv.seq_goff[bv.num_seqs] = G;
+  __syncthreads();
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  // per group: rows, sequence, tile count -> tile_prefix
+  for (int base = 0; base < G; base += blockDim.x) {
+    const int gi = base + tid;
+    uint32_t tiles = 0;
+    if (gi < G) {
+      int lo = 0, hi = bv.num_seqs - 1;            // last b with seq_goff[b] <= gi
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pv.seq_goff[mid] <= gi) lo = mid; else hi = mid - 1;
+      }
+      const int b = lo;
+      const int g = gi - pv.seq_goff[b];
+      const int c0 = __ldg(bv.cu_q + b), nb = __ldg(bv.cu_q + b + 1) - c0;
+      const int nrows = min(kIdxRows, nb - g * kIdxRows);
+      const int pos_last = __ldg(bv.seq_lens + b) - nb + g * kIdxRows + nrows - 1;
+      tiles = (uint32_t)(pos_last / kIdxTile + 1);
+      pv.g_row0[gi] = c0 + g * kIdxRows;
+      pv.g_nrows[gi] = nrows;
+      pv.g_seq[gi] = b;
+    }
+    uint32_t tot;
+    const uint32_t ex = block_exclusive_scan(tiles, tmp, &tot);
+    if (gi < G) pv.tile_prefix[gi] = (int)(s_carry + ex);
+    __syncthreads();
+    if (tid == 0) s_carry += tot;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    pv.tile_prefix[G] = (int)s_carry;
+    pv.hdr[0] = G;
+    pv.hdr[1] = (int)s_carry;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------ main
+struct IdxSmem {
+  uint64_t full[kIdxStages], empty[kIdxStages];
+  uint64_t bfull[2], bempty[2];
+  uint64_t tfull[2], tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// position of unit u: group index and tile within the group
+__device__ __forceinline__ void unit_locate(const int32_t *tile_prefix, int G, int u, int *gi, int *t) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(tile_prefix + mid) <= u) lo = mid; else hi = mid - 1;
+  }
+  *gi = lo;
+  *t = u - __ldg(tile_prefix + lo);
+}
+
+__global__ void __launch_bounds__(kIdxThreads, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                  const float *__restrict__ kscale, const float *__restrict__ w, BatchView bv, IdxPlanView pv,
+                  float *__restrict__ scores, int64_t ld, uint32_t *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sA = smem;                                             // kIdxStages x 16 KB
+  uint8_t *sB = sA + kIdxStages * kIdxTileBytes;                  // 2 x 32 KB
+  float *sW = (float *)(sB + 2 * kIdxBSlotBytes);                 // 2 x 1 KB
+  IdxSmem *S = (IdxSmem *)((uint8_t *)sW + 2 * kIdxWSlotBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = pv.hdr[0], U = pv.hdr[1];
+  const int u0 = (int)(((int64_t)blockIdx.x * U) / gridDim.x);
+  const int u1 = (int)(((int64_t)(blockIdx.x + 1) * U) / gridDim.x);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kIdxStages; ++i) {
+      tc::mbar_init(tc::smem_u32(&S->full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(tc::smem_u32(&S->bfull[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->bempty[i]), 1 + 4);
+      tc::mbar_init(tc::smem_u32(&S->tfull[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->tempty[i]), 4);
+    }
+    tc::mbar_init(tc::smem_u32(&S->drain), 1);
+    S->abort = 0;
+    tc::fence_barrier_init();
+    tc::prefetch_tmap(&tm_k);
+    tc::prefetch_tmap(&tm_q);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(&S->tmem_base), 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = S->tmem_base;
+  volatile int *abort = &S->abort;
+
+  if (u0 < u1) {
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      int gi, t;
+      unit_locate(pv.tile_prefix, G, u0, &gi, &t);
+      int stage = 0;
+      uint32_t phase = 0;
+      int bslot = 0, nb_groups = 0;
+      uint32_t issued = 0, last_par = 0;       // per stage: issued at least once / parity of last issue
+      uint32_t b_issued = 0, b_last_par = 0;
+      int cur = -1;
+      for (int u = u0; u < u1; ++u) {
+        if (gi != cur) {
+          bslot = nb_groups & 1;
+          const uint32_t use = (uint32_t)(nb_groups >> 1);
+          if (!tc::mbar_wait(tc::smem_u32(&S->bempty[bslot]), (use & 1u) ^ 1u, abort, status)) break;
+          const int row0 = pv.g_row0[gi], nr = pv.g_nrows[gi];
+          const uint32_t bar = tc::smem_u32(&S->bfull[bslot]);
+          tc::mbar_expect_tx(bar, (uint32_t)nr * (kIdxHi * kIdxDi + kIdxHi * 4));
+          for (int q = 0; q < nr; ++q) {
+            tc::tma_load_2d(tc::smem_u32(sB + bslot * kIdxBSlotBytes + q * kIdxHi * kIdxDi), &tm_q, 0,
+                            (row0 + q) * kIdxHi, bar);
+            tc::bulk_load(tc::smem_u32(sW + bslot * (kIdxWSlotBytes / 4) + q * kIdxHi), w + (int64_t)(row0 + q) * kIdxHi,
+                          kIdxHi * 4, bar);
+          }
+          b_issued |= 1u << bslot;
+          b_last_par = (b_last_par & ~(1u << bslot)) | ((use & 1u) << bslot);
+          ++nb_groups;
+          cur = gi;
+        }
+        if (!tc::mbar_wait(tc::smem_u32(&S->empty[stage]), phase ^ 1u, abort, status)) break;
+        const int b = pv.g_seq[gi];
+        const int nrw = pv.g_nrows[gi];
+        const int nbq = __ldg(bv.cu_q + b + 1) - __ldg(bv.cu_q + b);
+        const int pos_last = __ldg(bv.seq_lens + b) - nbq + (pv.g_row0[gi] - __ldg(bv.cu_q + b)) + nrw - 1;
+        const int pages = pos_last / 64 + 1;
+        const int p0 = 2 * t, p1 = 2 * t + 1;
+        const int32_t *btr = bv.block_table + (int64_t)b * bv.max_blocks_per_seq;
+        int blk0 = __ldg(btr + p0);
+        int blk1 = p1 < pages ? __ldg(btr + p1) : -1;
+        if ((unsigned)blk0 >= (unsigned)bv.num_blocks) { set_status(status, kStatusBadIndex); blk0 = -1; }
+        if (p1 < pages && (unsigned)blk1 >= (unsigned)bv.num_blocks) { set_status(status, kStatusBadIndex); blk1 = -1; }
+        const uint32_t bar = tc::smem_u32(&S->full[stage]);
+        const uint32_t bytes = (blk0 >= 0 ? kIdxPageBytes : 0u) + (blk1 >= 0 ? kIdxPageBytes : 0u);
+        if (bytes) {
+          tc::mbar_expect_tx(bar, bytes);
+          if (blk0 >= 0) tc::tma_load_2d(tc::smem_u32(sA + stage * kIdxTileBytes), &tm_k, 0, blk0 * 64, bar);
+          if (blk1 >= 0)
+            tc::tma_load_2d(tc::smem_u32(sA + stage * kIdxTileBytes + kIdxPageBytes), &tm_k, 0, blk1 * 64, bar);
+        } else {
+          tc::mbar_arrive(bar);
+        }
+        issued |= 1u << stage;
+        last_par = (last_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kIdxStages) { stage = 0; phase ^= 1u; }
+        if (++t == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) { ++gi; t = 0; }
+      }
+      // never leave with copies in flight: wait for the last fill of every stage / slot
+      for (int s = 0; s < kIdxStages; ++s)
+        if (issued & (1u << s)) {
+          volatile int no_abort = 0;
+          tc::mbar_wait(tc::smem_u32(&S->full[s]), (last_par >> s) & 1u, &no_abort, status);
+        }
+      for (int s = 0; s < 2; ++s)
+        if (b_issued & (1u << s)) {
+          volatile int no_abort = 0;
+          tc::mbar_wait(tc::smem_u32(&S->bfull[s]), (b_last_par >> s) & 1u, &no_abort, status);
+        }
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------------ MMA issuer
+      int gi, t;
+      unit_locate(pv.tile_prefix, G, u0, &gi, &t);
+      int stage = 0, acc = 0, nb_groups = 0, bslot = 0, cur = -1;
+      uint32_t phase = 0, acc_phase = 0;
+      for (int u = u0; u < u1; ++u) {
+        if (gi != cur) {
+          bslot = nb_groups & 1;
+          if (!tc::mbar_wait(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort, status)) break;
+          ++nb_groups;
+          cur = gi;
+        }
+        if (!tc::mbar_wait(tc::smem_u32(&S->tempty[acc]), acc_phase ^ 1u, abort, status)) break;
+        tc::fence_after_sync();
+        if (!tc::mbar_wait(tc::smem_u32(&S->full[stage]), phase, abort, status)) break;
+        const int nr = pv.g_nrows[gi];
+        const uint32_t idesc = tc::make_idesc(0, 0, 128, 64 * nr, false, false);
+        const uint32_t a0 = tc::smem_u32(sA + stage * kIdxTileBytes);
+        const uint32_t b0 = tc::smem_u32(sB + bslot * kIdxBSlotBytes);
+#pragma unroll
+        for (int k = 0; k < kIdxDi / 32; ++k) {
+          tc::mma_f8f6f4(tmem + acc * 256, tc::desc_sw128(a0 + 32 * k, 1024), tc::desc_sw128(b0 + 32 * k, 1024), idesc,
+                         k > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(tc::smem_u32(&S->empty[stage]));
+        tc::mma_commit(tc::smem_u32(&S->tfull[acc]));
+        const bool last_of_group = (t + 1 == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) || (u + 1 == u1);
+        if (last_of_group) tc::mma_commit(tc::smem_u32(&S->bempty[bslot]));
+        if (++stage == kIdxStages) { stage = 0; phase ^= 1u; }
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++t == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) { ++gi; t = 0; }
+      }
+      // every MMA issued by this thread has completed before TMEM is released
+      tc::mma_commit(tc::smem_u32(&S->drain));
+      volatile int no_abort = 0;
+      tc::mbar_wait(tc::smem_u32(&S->drain), 0, &no_abort, status);
+    } else if (warp >= 2) {
+      // ------------------------------------------------------------------ epilogue
+      const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+      const int key_local = quad * 32 + lane;
+      int gi, t;
+      unit_locate(pv.tile_prefix, G, u0, &gi, &t);
+      int acc = 0, nb_groups = 0, bslot = 0, cur = -1;
+      uint32_t acc_phase = 0;
+      int b = 0, row0 = 0, nr = 0, pos0 = 0;
+      for (int u = u0; u < u1; ++u) {
+        if (gi != cur) {
+          bslot = nb_groups & 1;
+          if (!tc::mbar_wait(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort, status)) break;
+          ++nb_groups;
+          cur = gi;
+          b = pv.g_seq[gi];
+          row0 = pv.g_row0[gi];
+          nr = pv.g_nrows[gi];
+          const int c0 = __ldg(bv.cu_q + b);
+          pos0 = __ldg(bv.seq_lens + b) - (__ldg(bv.cu_q + b + 1) - c0) + (row0 - c0);
+        }
+        const int s = t * kIdxTile + key_local;
+        float ks = 0.f;
+        if (s <= pos0 + nr - 1) {
+          const int blk = __ldg(bv.block_table + (int64_t)b * bv.max_blocks_per_seq + (s >> 6));
+          if ((unsigned)blk < (unsigned)bv.num_blocks) ks = __ldg(kscale + (int64_t)blk * 64 + (s & 63));
+        }
+        if (!tc::mbar_wait(tc::smem_u32(&S->tfull[acc]), acc_phase, abort, status)) break;
+        tc::fence_after_sync();
+        const float *wq = sW + bslot * (kIdxWSlotBytes / 4);
+        const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + acc * 256;
+        for (int q = 0; q < nr; ++q) {
+          float v0[32], v1[32];
+          tc::tmem_ld32(tbase + q * 64, v0);
+          tc::tmem_ld32(tbase + q * 64 + 32, v1);
+          tc::tmem_wait_ld();
+          const float *wr = wq + q * kIdxHi;
+          float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+          for (int h = 0; h < 32; h += 2) {
+            a0 = fmaf(wr[h], fmaxf(v0[h], 0.f), a0);
+            a1 = fmaf(wr[h + 1], fmaxf(v0[h + 1], 0.f), a1);
+          }
+#pragma unroll
+          for (int h = 0; h < 32; h += 2) {
+            a0 = fmaf(wr[32 + h], fmaxf(v1[h], 0.f), a0);
+            a1 = fmaf(wr[33 + h], fmaxf(v1[h + 1], 0.f), a1);
+          }
+          if (s <= pos0 + q) scores[(int64_t)(row0 + q) * ld + s] = (a0 + a1) * ks;
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->tempty[acc]));
+        const bool last_of_group = (t + 1 == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) || (u + 1 == u1);
+        if (last_of_group && lane == 0) tc::mbar_arrive(tc::smem_u32(&S->bempty[bslot]));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++t == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) { ++gi; t = 0; }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------ host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// 2-D byte matrix [rows, 128] read in boxes of 64 rows x 128 bytes with the 128-byte swizzle
+static bool make_rows128_map(CUtensorMap *m, const void *base, uint64_t rows) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, 64};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static size_t indexer_tc_smem() {
+  return 1024 + kIdxStages * kIdxTileBytes + 2 * kIdxBSlotBytes + 2 * kIdxWSlotBytes + sizeof(IdxSmem);
+}
+
+dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t *kpool, const float *kscale,
+                               const dsa_batch_t *b, float *scores, int64_t ld, void *ws, cudaStream_t stream,
+                               int num_sms) {
+  BatchView bv = view_of(b);
+  IdxPlanView pv = plan_view(ws, b->num_seqs, b->total_q);
+  CUtensorMap tm_k, tm_q;
+  if (!make_rows128_map(&tm_k, kpool, (uint64_t)b->num_blocks * 64) ||
+      !make_rows128_map(&tm_q, qI, (uint64_t)b->total_q * kIdxHi)) {
+    set_error("indexer: cuTensorMapEncodeTiled failed");
+    return DSA_ERR_CUDA;
+  }
+  indexer_plan_kernel<<<1, 1024, 0, stream>>>(bv, pv);
+  DSA_LAUNCH_CHECK("indexer_plan_kernel");
+  const size_t smem = indexer_tc_smem();
+  cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  indexer_tc_kernel<<<num_sms, kIdxThreads, smem, stream>>>(tm_k, tm_q, kscale, w, bv, pv, scores, ld,
+                                                             (uint32_t *)ws);
+  DSA_LAUNCH_CHECK("indexer_tc_kernel");
+  return DSA_OK;
+}
+
+}  // namespace dsa

@@ -1,0 +1,658 @@
+// Sparse MLA attention on tcgen05 tensor cores, one CTA pair (cluster of 2) per query row.
+//
+// For one query row with 128 heads, latent rows of 576 bf16 (the first 512 are also the values) and
+// up to k selected token positions:
+//   z[h, i] = scale * q[h, :] . K[idx_i],   o[h, :] = sum_i softmax_i(z[h, :]) V[idx_i],   lse[h]
+// ("Day-0 Adaptation for LLMs: Implementing Sparse Attention and Low-Precision Weights", decode sketch:
+// gather the selected KV, exact attention over it; "Engineering Practices for Day-0 Adaptation of
+// Million-Token Context Models on Domestic AI Chips", Four Key Layers 3: prefill processes query
+// tokens in parallel units, decode prefetches the next KV block with asynchronous copies while the
+// current one is computed, partial results are merged by a cross-block reduction.)
+//
+// Work split of a CTA pair (rank r = 0, 1), chunks of 128 selected tokens:
+//   * QK^T  : M = 128 heads (rank r holds heads 64r..64r+63 of q in smem), N = 128 tokens (rank r
+//             gathers tokens 64r..64r+63 of the chunk, all 576 dims), K = 576.  S lands in TMEM of
+//             both CTAs: each CTA gets its 64 heads x 128 tokens.
+//   * softmax: each CTA's 4 softmax warps own one (head, 64-token half) per thread: running max shared
+//             with the partner thread through smem, exp2, P (bf16) into smem.  O is rescaled in TMEM
+//             only when the running max grows by more than 2^8 (exact: the final division uses the
+//             same reference max).
+//   * P V   : M = 128 heads, N = 512 values as two N = 256 MMAs (rank r supplies values 256r..256r+255
+//             of every token), K = 128 tokens.  O (64 heads x 512 fp32) stays in TMEM, 256 columns.
+// Every MMA is issued by one thread of rank 0 for the pair (cta_group::2).  Tokens are gathered with
+// 16-byte cp.async through the block table straight into the 128-byte-swizzled operand layout, into a
+// ring of 16 KB slots in exactly the order the MMAs consume them; rank 1's slot completions are
+// relayed to rank 0's barriers by one thread.  Token positions that are -1 (or out of range) are
+// zero-filled and masked.
+//
+// Units: prefill = one row (all its chunks); decode = (row, split) pairs whose partial (o, lse) are
+// merged by attn_combine_kernel.  Rows are taken longest-first (reverse order) round-robin over pairs.
+#include <algorithm>
+
+#include "tc.cuh"
+
+namespace dsa {
+
+constexpr int kAttH = 128, kAttD = 576, kAttDv = 512;
+constexpr int kAttChunk = 128;
+constexpr int kAttSlots = 8;
+constexpr int kAttThreads = 320;                 // warps 0-3 softmax, 4-7 gather, 8 MMA, 9 relay
+constexpr uint32_t kAttSlotBytes = 16384;
+constexpr uint32_t kAttQBytes = 9 * 8192;
+constexpr uint32_t kAttPBytes = 16384;
+constexpr uint32_t kTmemO = 0, kTmemS = 256;     // O: 256 columns; S: two buffers of 64 columns
+constexpr float kRescaleLog2 = 8.0f;
+
+struct AttSmem {
+  uint64_t slot_full[kAttSlots];    // local: 128 gather threads (cp.async completion)
+  uint64_t pair_full[kAttSlots];    // rank 0: 2 relays
+  uint64_t slot_empty[kAttSlots];   // MMA commit to both CTAs
+  uint64_t q_full, pair_q_full, q_empty;
+  uint64_t s_full[2];               // MMA commit to both CTAs
+  uint64_t p_full;                  // rank 0: 8 softmax warps (4 per CTA)
+  uint64_t pv_done;                 // MMA commit to both CTAs, once per chunk
+  uint64_t o_empty;                 // rank 0: 8 softmax warps after the epilogue read O
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  float xm[2][128];
+  float xl[128];
+  int32_t phys[2][kAttChunk];
+};
+
+struct AttArgs {
+  const __nv_bfloat16 *q;       // [T, 128, 576]
+  const __nv_bfloat16 *kv;      // [NB*64, 576]
+  const int32_t *idx;           // [T, k]
+  int k;
+  BatchView bv;
+  const int32_t *neff;          // [T] 1 + last valid idx position
+  int T, splits;                // splits = 1: prefill units (one per row)
+  float scale_log2;             // softmax_scale * log2(e)
+  __nv_bfloat16 *out;           // [T, 128, 512] (splits == 1)
+  float *lse;                   // [T, 128] or nullptr (splits == 1)
+  float *part_o;                // [T*splits, 128, 512] (splits > 1)
+  float *part_lse;              // [T*splits, 128]
+  uint32_t *status;
+};
+
+__device__ __forceinline__ void unit_of(const AttArgs &a, int u, int *row, int *cb, int *ce) {
+  if (a.splits == 1) {
+    *row = a.T - 1 - u;
+    const int n = __ldg(a.neff + *row);
+    *cb = 0;
+    *ce = (n + kAttChunk - 1) / kAttChunk;
+  } else {
+    *row = u / a.splits;
+    const int s = u % a.splits;
+    const int n = __ldg(a.neff + *row);
+    const int nch = (n + kAttChunk - 1) / kAttChunk;
+    *cb = (s * nch) / a.splits;
+    *ce = ((s + 1) * nch) / a.splits;
+  }
+}
+
+__device__ __forceinline__ int num_units(const AttArgs &a) { return a.T * a.splits; }
+
+// ------------------------------------------------------------------------------------------------ plan
+// neff[row] = 1 + largest j with a usable idx[row, j] (0 if none); flags positions outside [0, seq_len)
+__global__ void attn_plan_kernel(const int32_t *__restrict__ idx, int k, BatchView bv, int T, int32_t *neff,
+                                 uint32_t *status) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  int b;
+  pos_of_row(bv, warp, &b);
+  const int seq_len = __ldg(bv.seq_lens + b);
+  int last = -1;
+  bool bad = false;
+  const int32_t *ir = idx + (int64_t)warp * k;
+  for (int j = lane; j < k; j += 32) {
+    const int s = __ldg(ir + j);
+    if (s >= 0 && s < seq_len) last = j;
+    else if (s >= seq_len) bad = true;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    neff[warp] = last + 1;
+    if (bad) set_status(status, kStatusBadIndex);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------ main
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn_mla_kernel(const AttArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sQ = smem;
+  uint8_t *sRing = sQ + kAttQBytes;
+  uint8_t *sP = sRing + kAttSlots * kAttSlotBytes;
+  AttSmem *S = (AttSmem *)(sP + kAttPBytes);
+
+  const uint32_t rank = tc::cluster_ctarank();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int U = num_units(a);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kAttSlots; ++i) {
+      tc::mbar_init(tc::smem_u32(&S->slot_full[i]), 128);
+      tc::mbar_init(tc::smem_u32(&S->pair_full[i]), 2);
+      tc::mbar_init(tc::smem_u32(&S->slot_empty[i]), 1);
+    }
+    tc::mbar_init(tc::smem_u32(&S->q_full), 128);
+    tc::mbar_init(tc::smem_u32(&S->pair_q_full), 2);
+    tc::mbar_init(tc::smem_u32(&S->q_empty), 1);
+    tc::mbar_init(tc::smem_u32(&S->s_full[0]), 1);
+    tc::mbar_init(tc::smem_u32(&S->s_full[1]), 1);
+    tc::mbar_init(tc::smem_u32(&S->p_full), 8);
+    tc::mbar_init(tc::smem_u32(&S->pv_done), 1);
+    tc::mbar_init(tc::smem_u32(&S->o_empty), 8);
+    tc::mbar_init(tc::smem_u32(&S->drain), 1);
+    S->abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 8) {
+    tc::tmem_alloc2(tc::smem_u32(&S->tmem_base), 512);
+    tc::tmem_relinquish2();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::cluster_sync();
+  tc::fence_after_sync();
+  const uint32_t tmem = S->tmem_base;
+  volatile int *abort = &S->abort;
+  uint32_t *status = a.status;
+
+  if (warp >= 4 && warp < 8) {
+    // ====================================================================== gather (128 threads)
+    // Loops holding the named barrier never break: after a timeout every wait returns at once and the
+    // copies are skipped, so all 128 threads still meet at the same barriers and reach the teardown.
+    const int t = threadIdx.x - 128;
+    int slot = 0;
+    uint32_t sphase = 0, v = 0;
+    for (int u = pair; u < U; u += npairs) {
+      int row, cb, ce;
+      unit_of(a, u, &row, &cb, &ce);
+      const int nch = ce - cb;
+      if (nch <= 0) continue;
+      int b;
+      pos_of_row(a.bv, row, &b);
+      const int seq_len = __ldg(a.bv.seq_lens + b);
+      const int32_t *btr = a.bv.block_table + (int64_t)b * a.bv.max_blocks_per_seq;
+      // ---- q: this CTA's 64 heads, [9 dim blocks][64 heads][128 B], 128-byte swizzle
+      bool ok = v == 0 || tc::mbar_wait_cl(tc::smem_u32(&S->q_empty), (v - 1) & 1u, abort, status);
+      if (ok) {
+        const __nv_bfloat16 *qr = a.q + ((int64_t)row * kAttH + 64 * rank) * kAttD;
+        const uint32_t qbase = tc::smem_u32(sQ);
+        for (int id = t; id < 64 * 72; id += 128) {
+          const int h = id / 72, rem = id % 72, d = rem >> 3, c = rem & 7;
+          tc::cp_async16(qbase + d * 8192 + h * 128 + ((c ^ (h & 7)) << 4), qr + (int64_t)h * kAttD + d * 64 + c * 8,
+                         16);
+        }
+      }
+      tc::cp_async_arrive_noinc(tc::smem_u32(&S->q_full));
+      for (int i = 0; i <= nch; ++i) {
+        if (i < nch) {
+          // token positions of chunk i -> physical rows (-1: masked)
+          tc::named_bar_sync(1, 128);
+          {
+            const int j = (cb + i) * kAttChunk + t;
+            int32_t pr = -1;
+            if (j < a.k) {
+              const int s = __ldg(a.idx + (int64_t)row * a.k + j);
+              if (s >= 0 && s < seq_len) {
+                const int blk = __ldg(btr + (s >> 6));
+                if ((unsigned)blk < (unsigned)a.bv.num_blocks) pr = blk * 64 + (s & 63);
+                else set_status(status, kStatusBadIndex);
+              }
+            }
+            S->phys[i & 1][t] = pr;
+          }
+          tc::named_bar_sync(1, 128);
+          // QK slots: own 64 tokens, dim blocks (2s, 2s+1)
+          for (int sl = 0; sl < 5; ++sl) {
+            if (tc::mbar_wait_cl(tc::smem_u32(&S->slot_empty[slot]), sphase ^ 1u, abort, status)) {
+              const uint32_t base = tc::smem_u32(sRing + slot * kAttSlotBytes);
+#pragma unroll
+              for (int m = 0; m < 8; ++m) {
+                const int id = t + 128 * m;
+                const int kr = id >> 4, blk = (id >> 3) & 1, c = id & 7;
+                const int d = 2 * sl + blk;
+                if (d < 9) {
+                  const int32_t pr = S->phys[i & 1][64 * rank + kr];
+                  const __nv_bfloat16 *src = pr >= 0 ? a.kv + (int64_t)pr * kAttD + d * 64 + c * 8 : a.kv;
+                  tc::cp_async16(base + blk * 8192 + kr * 128 + ((c ^ (kr & 7)) << 4), src, pr >= 0 ? 16u : 0u);
+                }
+              }
+            }
+            tc::cp_async_arrive_noinc(tc::smem_u32(&S->slot_full[slot]));
+            if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
+          }
+        }
+        if (i > 0) {
+          // PV slots of chunk i-1: value blocks (4r + 2p, 4r + 2p + 1) of token half kh
+          const int pc = (i - 1) & 1;
+          for (int p = 0; p < 2; ++p)
+            for (int kh = 0; kh < 2; ++kh) {
+              if (tc::mbar_wait_cl(tc::smem_u32(&S->slot_empty[slot]), sphase ^ 1u, abort, status)) {
+                const uint32_t base = tc::smem_u32(sRing + slot * kAttSlotBytes);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                  const int id = t + 128 * m;
+                  const int kr = id >> 4, blk = (id >> 3) & 1, c = id & 7;
+                  const int d = 4 * rank + 2 * p + blk;
+                  const int32_t pr = S->phys[pc][64 * kh + kr];
+                  const __nv_bfloat16 *src = pr >= 0 ? a.kv + (int64_t)pr * kAttD + d * 64 + c * 8 : a.kv;
+                  tc::cp_async16(base + blk * 8192 + kr * 128 + ((c ^ (kr & 7)) << 4), src, pr >= 0 ? 16u : 0u);
+                }
+              }
+              tc::cp_async_arrive_noinc(tc::smem_u32(&S->slot_full[slot]));
+              if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
+            }
+        }
+      }
+      ++v;
+    }
+    tc::cp_async_wait_all();
+  } else if (warp == 9) {
+    // ====================================================================== relay (lane 0)
+    if (lane == 0) {
+      const uint32_t peer_pair_full = tc::map_to_rank(tc::smem_u32(&S->pair_full[0]), 0);
+      const uint32_t peer_pair_q = tc::map_to_rank(tc::smem_u32(&S->pair_q_full), 0);
+      int slot = 0;
+      uint32_t sphase = 0, v = 0;
+      bool ok = true;
+      for (int u = pair; u < U && ok; u += npairs) {
+        int row, cb, ce;
+        unit_of(a, u, &row, &cb, &ce);
+        const int nch = ce - cb;
+        if (nch <= 0) continue;
+        if (!tc::mbar_wait(tc::smem_u32(&S->q_full), v & 1u, abort, status)) break;
+        tc::fence_proxy_async();
+        tc::mbar_arrive_cluster(peer_pair_q);
+        const int fills = 9 * nch;
+        for (int f = 0; f < fills; ++f) {
+          if (!tc::mbar_wait(tc::smem_u32(&S->slot_full[slot]), sphase, abort, status)) { ok = false; break; }
+          tc::fence_proxy_async();
+          tc::mbar_arrive_cluster(peer_pair_full + slot * 8);
+          if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
+        }
+        ++v;
+      }
+    }
+  } else if (warp == 8) {
+    // ====================================================================== MMA issuer (rank 0, lane 0)
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc_qk = tc::make_idesc(1, 1, 128, 128, false, false);
+      const uint32_t idesc_pv = tc::make_idesc(1, 1, 128, 256, false, true);
+      const uint16_t both = 3;
+      const uint32_t qbase = tc::smem_u32(sQ), pbase = tc::smem_u32(sP);
+      int slot = 0;
+      uint32_t sphase = 0, v = 0, g = 0;       // g: chunks issued so far (all units)
+      bool ok = true;
+      auto pv = [&](int c, uint32_t gc) -> bool {
+        if (!tc::mbar_wait_cl(tc::smem_u32(&S->p_full), gc & 1u, abort, status)) return false;
+        if (c == 0 && v > 0 && !tc::mbar_wait_cl(tc::smem_u32(&S->o_empty), (v - 1) & 1u, abort, status)) return false;
+        tc::fence_after_sync();
+        for (int p = 0; p < 2; ++p)
+          for (int kh = 0; kh < 2; ++kh) {
+            if (!tc::mbar_wait_cl(tc::smem_u32(&S->pair_full[slot]), sphase, abort, status)) return false;
+            tc::fence_after_sync();
+            const uint32_t base = tc::smem_u32(sRing + slot * kAttSlotBytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = tc::desc_sw128(pbase + kh * 8192 + kk * 32, 1024);
+              const uint64_t bd = tc::desc_sw128_lbo(base + kk * 2048, 8192, 1024);
+              tc::mma_bf16_pair(tmem + kTmemO + 128 * p, ad, bd, idesc_pv, (c == 0 && kh == 0 && kk == 0) ? 0u : 1u);
+            }
+            tc::mma_commit_pair(tc::smem_u32(&S->slot_empty[slot]), both);
+            if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
+          }
+        tc::mma_commit_pair(tc::smem_u32(&S->pv_done), both);
+        return true;
+      };
+      for (int u = pair; u < U && ok; u += npairs) {
+        int row, cb, ce;
+        unit_of(a, u, &row, &cb, &ce);
+        const int nch = ce - cb;
+        if (nch <= 0) continue;
+        if (!tc::mbar_wait_cl(tc::smem_u32(&S->pair_q_full), v & 1u, abort, status)) break;
+        tc::fence_after_sync();
+        const uint32_t g0 = g;
+        for (int i = 0; i < nch && ok; ++i) {
+          const uint32_t sb = tmem + kTmemS + 64 * (g & 1u);
+          for (int sl = 0; sl < 5; ++sl) {
+            if (!tc::mbar_wait_cl(tc::smem_u32(&S->pair_full[slot]), sphase, abort, status)) { ok = false; break; }
+            tc::fence_after_sync();
+            const uint32_t base = tc::smem_u32(sRing + slot * kAttSlotBytes);
+            for (int blk = 0; blk < 2; ++blk) {
+              const int d = 2 * sl + blk;
+              if (d >= 9) break;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = tc::desc_sw128(qbase + d * 8192 + kk * 32, 1024);
+                const uint64_t bd = tc::desc_sw128(base + blk * 8192 + kk * 32, 1024);
+                tc::mma_bf16_pair(sb, ad, bd, idesc_qk, (d == 0 && kk == 0) ? 0u : 1u);
+              }
+            }
+            tc::mma_commit_pair(tc::smem_u32(&S->slot_empty[slot]), both);
+            if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
+          }
+          if (!ok) break;
+          tc::mma_commit_pair(tc::smem_u32(&S->s_full[g & 1u]), both);
+          if (i == nch - 1) tc::mma_commit_pair(tc::smem_u32(&S->q_empty), both);
+          ++g;
+          if (i > 0 && !pv(i - 1, g0 + i - 1)) { ok = false; break; }
+        }
+        if (ok && !pv(nch - 1, g0 + nch - 1)) ok = false;
+        ++v;
+      }
+      tc::mma_commit_pair_local(tc::smem_u32(&S->drain));
+      volatile int no_abort = 0;
+      tc::mbar_wait(tc::smem_u32(&S->drain), 0, &no_abort, status);
+    }
+  } else {
+    // ====================================================================== softmax + epilogue (128 threads)
+    // Like the gather role, these loops never break (they hold named barrier 2): after a timeout the
+    // waits return at once and the remaining chunks run through without touching TMEM or memory.
+    const int L = threadIdx.x;                 // TMEM lane
+    const int h = L & 63, half = L >> 6;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t p_full_r0 = tc::map_to_rank(tc::smem_u32(&S->p_full), 0);
+    const uint32_t o_empty_r0 = tc::map_to_rank(tc::smem_u32(&S->o_empty), 0);
+    uint32_t g = 0, v = 0;
+    for (int u = pair; u < U; u += npairs) {
+      int row, cb, ce;
+      unit_of(a, u, &row, &cb, &ce);
+      const int nch = ce - cb;
+      const int head = 64 * (int)rank + h;
+      if (nch <= 0) {
+        // nothing selected: o = 0, lse = -inf
+        if (a.splits == 1) {
+          __nv_bfloat16 *o = a.out + ((int64_t)row * kAttH + head) * kAttDv + 256 * half;
+          for (int c = 0; c < 256; c += 8) *reinterpret_cast<uint4 *>(o + c) = make_uint4(0, 0, 0, 0);
+          if (a.lse && half == 0) a.lse[(int64_t)row * kAttH + head] = -INFINITY;
+        } else {
+          float *o = a.part_o + ((int64_t)u * kAttH + head) * kAttDv + 256 * half;
+          for (int c = 0; c < 256; c += 4) *reinterpret_cast<float4 *>(o + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (half == 0) a.part_lse[(int64_t)u * kAttH + head] = -INFINITY;
+        }
+        continue;
+      }
+      int b;
+      pos_of_row(a.bv, row, &b);
+      const int seq_len = __ldg(a.bv.seq_lens + b);
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int i = 0; i < nch; ++i, ++g) {
+        // validity of this thread's 64 tokens
+        uint64_t valid = 0;
+        {
+          const int j0 = (cb + i) * kAttChunk + 64 * half;
+          const int32_t *ir = a.idx + (int64_t)row * a.k;
+#pragma unroll 8
+          for (int t2 = 0; t2 < 64; ++t2) {
+            const int j = j0 + t2;
+            const int s = j < a.k ? __ldg(ir + j) : -1;
+            if (s >= 0 && s < seq_len) valid |= 1ull << t2;
+          }
+        }
+        const bool have_s = tc::mbar_wait_cl(tc::smem_u32(&S->s_full[g & 1u]), (g >> 1) & 1u, abort, status);
+        tc::fence_after_sync();
+        float sv[64];
+        {
+          float t0[32], t1[32];
+          const uint32_t sa = tmem + lane_base + kTmemS + 64 * (g & 1u);
+          tc::tmem_ld32(sa, t0);
+          tc::tmem_ld32(sa + 32, t1);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            sv[c] = t0[c];
+            sv[32 + c] = t1[c];
+          }
+        }
+        if (!have_s) valid = 0;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          sv[c] = ((valid >> c) & 1ull) ? sv[c] * a.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sv[c]);
+        }
+        const float mloc = fmaxf(m_run, mx);
+        S->xm[g & 1u][L] = mloc;
+        tc::named_bar_sync(2, 128);
+        const float m_new = fmaxf(mloc, S->xm[g & 1u][L ^ 64]);
+        // PV of the previous chunk must be finished before O is touched or P is overwritten
+        bool pv_ok = true;
+        if (i > 0) {
+          pv_ok = tc::mbar_wait_cl(tc::smem_u32(&S->pv_done), (g - 1) & 1u, abort, status);
+          tc::fence_after_sync();
+        }
+        if (i == 0) {
+          m_run = m_new;
+        } else if (m_new > m_run + kRescaleLog2) {
+          const float alpha = tc::ex2(m_run - m_new);
+          if (pv_ok) {
+            for (int cc = 0; cc < 8; ++cc) {
+              float ov[32];
+              tc::tmem_ld32(tmem + lane_base + kTmemO + 32 * cc, ov);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+              tc::tmem_st32(tmem + lane_base + kTmemO + 32 * cc, ov);
+            }
+            tc::tmem_wait_st();
+          }
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        // P = exp2(z - m) in bf16, into the 128-byte-swizzled A operand (row h, tokens of this half)
+        if (pv_ok) {
+          uint8_t *prow = sP + half * 8192 + h * 128;
+          float lsum = 0.f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int t0 = 8 * c + 2 * e;
+              const float p0 = ((valid >> t0) & 1ull) ? tc::ex2(sv[t0] - m_run) : 0.f;
+              const float p1 = ((valid >> (t0 + 1)) & 1ull) ? tc::ex2(sv[t0 + 1] - m_run) : 0.f;
+              const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+              const float2 pr = __bfloat1622float2(pb);
+              lsum += pr.x + pr.y;
+              w4[e] = *reinterpret_cast<const uint32_t *>(&pb);
+            }
+            *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+          l_run += lsum;
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive_cluster(p_full_r0);
+      }
+      // ---- epilogue: wait for the last P V, normalise, store
+      const bool o_ok = tc::mbar_wait_cl(tc::smem_u32(&S->pv_done), (g - 1) & 1u, abort, status);
+      tc::fence_after_sync();
+      S->xl[L] = l_run;
+      tc::named_bar_sync(2, 128);
+      const float l_tot = l_run + S->xl[L ^ 64];
+      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const float lse_v = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+      if (o_ok) {
+        if (a.splits == 1) {
+          __nv_bfloat16 *o = a.out + ((int64_t)row * kAttH + head) * kAttDv + 256 * half;
+          for (int cc = 0; cc < 8; ++cc) {
+            float ov[32];
+            tc::tmem_ld32(tmem + lane_base + kTmemO + 32 * cc, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 w;
+              __nv_bfloat162 b0 = __floats2bfloat162_rn(ov[e] * inv, ov[e + 1] * inv);
+              __nv_bfloat162 b1 = __floats2bfloat162_rn(ov[e + 2] * inv, ov[e + 3] * inv);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(ov[e + 4] * inv, ov[e + 5] * inv);
+              __nv_bfloat162 b3 = __floats2bfloat162_rn(ov[e + 6] * inv, ov[e + 7] * inv);
+              w.x = *reinterpret_cast<uint32_t *>(&b0);
+              w.y = *reinterpret_cast<uint32_t *>(&b1);
+              w.z = *reinterpret_cast<uint32_t *>(&b2);
+              w.w = *reinterpret_cast<uint32_t *>(&b3);
+              *reinterpret_cast<uint4 *>(o + 32 * cc + e) = w;
+            }
+          }
+          if (a.lse && half == 0) a.lse[(int64_t)row * kAttH + head] = lse_v;
+        } else {
+          float *o = a.part_o + ((int64_t)u * kAttH + head) * kAttDv + 256 * half;
+          for (int cc = 0; cc < 8; ++cc) {
+            float ov[32];
+            tc::tmem_ld32(tmem + lane_base + kTmemO + 32 * cc, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4 *>(o + 32 * cc + e) =
+                  make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv, ov[e + 3] * inv);
+          }
+          if (half == 0) a.part_lse[(int64_t)u * kAttH + head] = lse_v;
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive_cluster(o_empty_r0);
+      ++v;
+    }
+  }
+
+  // ---- teardown: every role is done; MMAs drained; peers done with our barriers and TMEM
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::cluster_sync();
+  if (warp == 8) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc2(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------ combine
+// out[row, h, :] = sum_s exp(lse_s - lse) o_s,  lse = log sum_s exp(lse_s)   (splits of one row)
+__global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restrict__ part_o,
+                                                           const float *__restrict__ part_lse, int splits,
+                                                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+  const int row = blockIdx.x, h = blockIdx.y;
+  float mx = -INFINITY;
+  for (int s = 0; s < splits; ++s) mx = fmaxf(mx, __ldg(part_lse + ((int64_t)row * splits + s) * kAttH + h));
+  float tot = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float l = __ldg(part_lse + ((int64_t)row * splits + s) * kAttH + h);
+    tot += l == -INFINITY ? 0.f : __expf(l - mx);
+  }
+  const int dv = threadIdx.x * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tot > 0.f) {
+    for (int s = 0; s < splits; ++s) {
+      const float l = __ldg(part_lse + ((int64_t)row * splits + s) * kAttH + h);
+      if (l == -INFINITY) continue;
+      const float wgt = __expf(l - mx) / tot;
+      const float4 o = __ldg(reinterpret_cast<const float4 *>(part_o + (((int64_t)row * splits + s) * kAttH + h) * kAttDv + dv));
+      acc.x += wgt * o.x;
+      acc.y += wgt * o.y;
+      acc.z += wgt * o.z;
+      acc.w += wgt * o.w;
+    }
+  }
+  __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x, acc.y), b1 = __floats2bfloat162_rn(acc.z, acc.w);
+  uint2 w;
+  w.x = *reinterpret_cast<uint32_t *>(&b0);
+  w.y = *reinterpret_cast<uint32_t *>(&b1);
+  *reinterpret_cast<uint2 *>(out + ((int64_t)row * kAttH + h) * kAttDv + dv) = w;
+  if (lse && threadIdx.x == 0) lse[(int64_t)row * kAttH + h] = tot > 0.f ? mx + __logf(tot) : -INFINITY;
+}
+
+// ------------------------------------------------------------------------------------------------ host
+static size_t al256b(size_t x) { return (x + 255) / 256 * 256; }
+
+// Decode splits are sized for the B200's 148 SMs (74 CTA pairs); the same figure sizes the workspace.
+constexpr int kAttPairsForSplits = 74;
+
+int attn_decode_splits(int T, int k) {
+  const int pairs = kAttPairsForSplits;
+  const int chunks = (k + kAttChunk - 1) / kAttChunk;
+  int s = T > 0 ? pairs / T : 1;
+  return s < 1 ? 1 : (s > chunks ? chunks : s);
+}
+
+size_t attn_workspace_bytes(int T, int k, bool decode) {
+  size_t bytes = kWsHeader + al256b((size_t)T * 4);
+  if (decode) {
+    const int s = attn_decode_splits(T, k);
+    if (s > 1) bytes += al256b((size_t)T * s * kAttH * kAttDv * 4) + al256b((size_t)T * s * kAttH * 4);
+  }
+  return bytes;
+}
+
+static size_t attn_smem_bytes() { return 1024 + kAttQBytes + kAttSlots * kAttSlotBytes + kAttPBytes + sizeof(AttSmem); }
+
+dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, int k, float softmax_scale,
+                             const dsa_batch_t *b, void *out, float *lse, void *ws, bool decode, cudaStream_t stream,
+                             int num_sms) {
+  AttArgs a{};
+  a.q = (const __nv_bfloat16 *)q;
+  a.kv = (const __nv_bfloat16 *)kv;
+  a.idx = idx;
+  a.k = k;
+  a.bv = view_of(b);
+  a.T = b->total_q;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.status = (uint32_t *)ws;
+  char *p = (char *)ws + kWsHeader;
+  a.neff = (const int32_t *)p;
+  int32_t *neff = (int32_t *)p;
+  p += al256b((size_t)a.T * 4);
+  a.splits = decode ? attn_decode_splits(a.T, k) : 1;
+  if (a.splits > 1) {
+    a.part_o = (float *)p;
+    p += al256b((size_t)a.T * a.splits * kAttH * kAttDv * 4);
+    a.part_lse = (float *)p;
+  } else {
+    a.out = (__nv_bfloat16 *)out;
+    a.lse = lse;
+  }
+  attn_plan_kernel<<<(a.T + 3) / 4, 128, 0, stream>>>(idx, k, a.bv, a.T, neff, a.status);
+  DSA_LAUNCH_CHECK("attn_plan_kernel");
+  const size_t smem = attn_smem_bytes();
+  cudaFuncSetAttribute(attn_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // persistent grid: as many CTA pairs as can be resident at once
+  static int max_pairs = 0;
+  if (max_pairs == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.gridDim = dim3(num_sms & ~1);
+    cfg.blockDim = dim3(kAttThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_mla_kernel, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = num_sms / 2;
+    }
+    max_pairs = std::min(n, num_sms / 2);
+  }
+  const int units = a.T * a.splits;
+  const int pairs = std::min(max_pairs, units);
+  attn_mla_kernel<<<2 * pairs, kAttThreads, smem, stream>>>(a);
+  DSA_LAUNCH_CHECK("attn_mla_kernel");
+  if (a.splits > 1) {
+    attn_combine_kernel<<<dim3(a.T, kAttH), 128, 0, stream>>>(a.part_o, a.part_lse, a.splits, (__nv_bfloat16 *)out,
+                                                               lse);
+    DSA_LAUNCH_CHECK("attn_combine_kernel");
+  }
+  return DSA_OK;
+}
+
+}  // namespace dsa

@@ -21,6 +21,10 @@ dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t 
                                const dsa_batch_t *b, float *scores, int64_t ld, void *ws, cudaStream_t stream,
                                int num_sms);
 size_t indexer_workspace_bytes(int num_seqs, int total_q);
+dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, int k, float softmax_scale,
+                             const dsa_batch_t *b, void *out, float *lse, void *ws, bool decode, cudaStream_t stream,
+                             int num_sms);
+size_t attn_workspace_bytes(int T, int k, bool decode);
 dsa_status_t attn_simt_launch(const void *q, dsa_dtype_t dt, const void *kv, const void *v, int H, int Dqk, int Dv,
                               float scale, const int32_t *idx, int k, const dsa_batch_t *b, void *out, float *lse,
                               cudaStream_t stream);
@@ -120,7 +124,9 @@ static bool is_f32_attn(dsa_dtype_t dt, int H, int Dqk, int Dv, const void *v) {
   return dt == DSA_F32 && H >= 1 && H <= 16 && Dqk >= 1 && Dqk <= 128 && Dv >= 1 && Dv <= 128 && v != nullptr;
 }
 
-static size_t attn_workspace_bytes(const dsa_batch_t *, int, int, int) { return kWsHeader; }
+static size_t attn_ws_bytes(const dsa_batch_t *b, int k, int H, int Dv, bool decode) {
+  return H == 128 && Dv == 512 ? attn_workspace_bytes(b->total_q, k, decode) : kWsHeader;
+}
 
 }  // namespace dsa
 
@@ -158,8 +164,8 @@ dsa_status_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t *b, int32_t k, in
   switch (op) {
     case DSA_OP_INDEXER: *bytes = indexer_workspace_bytes(b->num_seqs, b->total_q); return DSA_OK;
     case DSA_OP_TOPK: *bytes = topk_workspace_bytes(b->total_q, b->max_seq_len); return DSA_OK;
-    case DSA_OP_ATTN_PREFILL:
-    case DSA_OP_ATTN_DECODE: *bytes = attn_workspace_bytes(b, k, H, Dv); return DSA_OK;
+    case DSA_OP_ATTN_PREFILL: *bytes = attn_ws_bytes(b, k, H, Dv, false); return DSA_OK;
+    case DSA_OP_ATTN_DECODE: *bytes = attn_ws_bytes(b, k, H, Dv, true); return DSA_OK;
   }
   set_error("unknown op %d", (int)op);
   return DSA_ERR_INVALID_ARG;
@@ -227,10 +233,15 @@ static dsa_status_t attn_common(bool decode, const void *q, dsa_dtype_t dt, cons
             "H<=16, Dqk<=128, Dv<=128 and a separate V cache");
   if (decode) CHECK_ARG(b->total_q == b->num_seqs && b->max_q_per_seq == 1,
                         "decode needs exactly one query row per sequence");
-  if ((st = check_ws(ws, ws_bytes, attn_workspace_bytes(b, k, H, Dv))) != DSA_OK) return st;
+  CHECK_ARG((((uintptr_t)q | (uintptr_t)kv_pool | (uintptr_t)out) & 15) == 0,
+            "q, kv_pool and out must be 16-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, attn_ws_bytes(b, k, H, Dv, decode))) != DSA_OK) return st;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
   if (b->total_q == 0) return DSA_OK;
+  if (mla)
+    return attn_mla_launch(q, kv_pool, idx, k, softmax_scale, b, out, lse, ws, decode, (cudaStream_t)stream,
+                           dev.num_sms);
   return attn_simt_launch(q, dt, kv_pool, v_pool, H, Dqk, Dv, softmax_scale, idx, k, b, out, lse,
                           (cudaStream_t)stream);
 }

@@ -18,12 +18,6 @@ template <typename TQ>
 __device__ __forceinline__ float load_val(const TQ *p, int64_t i);
 template <>
 __device__ __forceinline__ float load_val<float>(const float *p, int64_t i) { return __ldg(p + i); }
-template <>
-__device__ __forceinline__ float load_val<uint8_t>(const uint8_t *p, int64_t i) { return e4m3_to_float(__ldg(p + i)); }
-template <>
-__device__ __forceinline__ float load_val<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
-  return __bfloat162float(p[i]);
-}
 
 template <typename TQ>
 __global__ void __launch_bounds__(kIdxSimtTile)
@@ -69,10 +63,6 @@ template <typename T>
 __device__ __forceinline__ void store_val(T *p, int64_t i, float v);
 template <>
 __device__ __forceinline__ void store_val<float>(float *p, int64_t i, float v) { p[i] = v; }
-template <>
-__device__ __forceinline__ void store_val<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float v) {
-  p[i] = __float2bfloat16_rn(v);
-}
 
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -186,15 +176,10 @@ dsa_status_t indexer_simt_launch(const void *qI, dsa_dtype_t dt, const float *w,
   BatchView bv = view_of(b);
   dim3 grid(b->total_q, (b->max_seq_len + kIdxSimtTile - 1) / kIdxSimtTile);
   size_t smem = (size_t)(Hi * Di + Hi) * 4;
-  if (dt == DSA_F32) {
-    cudaFuncSetAttribute(indexer_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    indexer_simt_kernel<float><<<grid, kIdxSimtTile, smem, stream>>>((const float *)qI, w, (const float *)kpool,
-                                                                     kscale, Hi, Di, bv, scores, ld);
-  } else {
-    cudaFuncSetAttribute(indexer_simt_kernel<uint8_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    indexer_simt_kernel<uint8_t><<<grid, kIdxSimtTile, smem, stream>>>(
-        (const uint8_t *)qI, w, (const uint8_t *)kpool, kscale, Hi, Di, bv, scores, ld);
-  }
+  (void)dt;   // the e4m3 indexer runs on the tensor cores (indexer_tc.cu)
+  cudaFuncSetAttribute(indexer_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  indexer_simt_kernel<float><<<grid, kIdxSimtTile, smem, stream>>>((const float *)qI, w, (const float *)kpool,
+                                                                   kscale, Hi, Di, bv, scores, ld);
   DSA_LAUNCH_CHECK("indexer_simt_kernel");
   return DSA_OK;
 }
@@ -206,16 +191,10 @@ dsa_status_t attn_simt_launch(const void *q, dsa_dtype_t dt, const void *kv, con
   dim3 grid(b->total_q, (H + kAttnSimtHG - 1) / kAttnSimtHG);
   size_t smem = (size_t)(kAttnSimtHG * Dqk + kAttnSimtChunk * (Dqk + 1) + kAttnSimtChunk * Dv +
                          kAttnSimtHG * kAttnSimtChunk) * 4;
-  if (dt == DSA_F32) {
-    cudaFuncSetAttribute(attn_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_simt_kernel<float><<<grid, 256, smem, stream>>>((const float *)q, (const float *)kv, (const float *)v, H,
-                                                         Dqk, Dv, scale, idx, k, bv, (float *)out, lse);
-  } else {
-    cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_simt_kernel<__nv_bfloat16><<<grid, 256, smem, stream>>>(
-        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kv, (const __nv_bfloat16 *)v, H, Dqk, Dv, scale, idx, k,
-        bv, (__nv_bfloat16 *)out, lse);
-  }
+  (void)dt;   // the bf16 MLA path runs on the tensor cores (attn_mla_tc.cu)
+  cudaFuncSetAttribute(attn_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  attn_simt_kernel<float><<<grid, 256, smem, stream>>>((const float *)q, (const float *)kv, (const float *)v, H, Dqk,
+                                                       Dv, scale, idx, k, bv, (float *)out, lse);
   DSA_LAUNCH_CHECK("attn_simt_kernel");
   return DSA_OK;
 }

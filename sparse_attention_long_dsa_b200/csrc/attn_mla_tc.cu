@@ -56,7 +56,7 @@ struct AttSmem {
   uint32_t tmem_base;
   int abort;
   float xm[2][128];
-  float xl[128];
+  float xl[2][128];
   int32_t phys[2][kAttChunk];
 };
 
@@ -383,7 +383,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
       int b;
       pos_of_row(a.bv, row, &b);
       const int seq_len = __ldg(a.bv.seq_lens + b);
-      float m_run = -INFINITY, l_run = 0.f;
+      float m_run = -INFINITY, l_run = 0.f, l_exact = 0.f;
       for (int i = 0; i < nch; ++i, ++g) {
         // validity of this thread's 64 tokens
         uint64_t valid = 0;
@@ -429,28 +429,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
           pv_ok = tc::mbar_wait_cl(tc::smem_u32(&S->pv_done), (g - 1) & 1u, abort, status);
           tc::fence_after_sync();
         }
+        pv_ok = __all_sync(0xffffffffu, pv_ok);
         if (i == 0) {
           m_run = m_new;
-        } else if (m_new > m_run + kRescaleLog2) {
-          const float alpha = tc::ex2(m_run - m_new);
-          if (pv_ok) {
-            for (int cc = 0; cc < 8; ++cc) {
-              float ov[32];
-              tc::tmem_ld32(tmem + lane_base + kTmemO + 32 * cc, ov);
-              tc::tmem_wait_ld();
+        } else {
+          // TMEM loads/stores are warp-collective: the warp rescales if any of its rows needs it,
+          // rows that do not keep their reference max (alpha = 1)
+          const bool want = m_new > m_run + kRescaleLog2;
+          if (__any_sync(0xffffffffu, want)) {
+            const float alpha = want ? tc::ex2(m_run - m_new) : 1.f;
+            if (pv_ok) {
+              for (int cc = 0; cc < 8; ++cc) {
+                float ov[32];
+                tc::tmem_ld32(tmem + lane_base + kTmemO + 32 * cc, ov);
+                tc::tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-              tc::tmem_st32(tmem + lane_base + kTmemO + 32 * cc, ov);
+                for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+                tc::tmem_st32(tmem + lane_base + kTmemO + 32 * cc, ov);
+              }
+              tc::tmem_wait_st();
             }
-            tc::tmem_wait_st();
+            if (want) {
+              l_run *= alpha;
+              l_exact *= alpha;
+              m_run = m_new;
+            }
           }
-          l_run *= alpha;
-          m_run = m_new;
         }
-        // P = exp2(z - m) in bf16, into the 128-byte-swizzled A operand (row h, tokens of this half)
+        // P = exp2(z - m) in bf16, into the 128-byte-swizzled A operand (row h, tokens of this half).
+        // l_run sums the rounded P (what the MMA multiplies) and normalises O; l_exact sums the
+        // unrounded values and gives lse.
         if (pv_ok) {
           uint8_t *prow = sP + half * 8192 + h * 128;
-          float lsum = 0.f;
+          float lsum = 0.f, lex = 0.f;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t w4[4];
@@ -462,11 +473,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
               const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
               const float2 pr = __bfloat1622float2(pb);
               lsum += pr.x + pr.y;
+              lex += p0 + p1;
               w4[e] = *reinterpret_cast<const uint32_t *>(&pb);
             }
             *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
           l_run += lsum;
+          l_exact += lex;
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
@@ -474,13 +487,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
         if (lane == 0) tc::mbar_arrive_cluster(p_full_r0);
       }
       // ---- epilogue: wait for the last P V, normalise, store
-      const bool o_ok = tc::mbar_wait_cl(tc::smem_u32(&S->pv_done), (g - 1) & 1u, abort, status);
+      const bool o_ok =
+          __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->pv_done), (g - 1) & 1u, abort, status));
       tc::fence_after_sync();
-      S->xl[L] = l_run;
+      S->xl[0][L] = l_run;
+      S->xl[1][L] = l_exact;
       tc::named_bar_sync(2, 128);
-      const float l_tot = l_run + S->xl[L ^ 64];
+      const float l_tot = l_run + S->xl[0][L ^ 64];
+      const float l_ex = l_exact + S->xl[1][L ^ 64];
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      const float lse_v = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+      const float lse_v = l_ex > 0.f ? (m_run + __log2f(l_ex)) * 0.69314718055994531f : -INFINITY;
       if (o_ok) {
         if (a.splits == 1) {
           __nv_bfloat16 *o = a.out + ((int64_t)row * kAttH + head) * kAttDv + 256 * half;

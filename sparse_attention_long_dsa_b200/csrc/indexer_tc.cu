@@ -311,7 +311,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       for (int u = u0; u < u1; ++u) {
         if (gi != cur) {
           bslot = nb_groups & 1;
-          if (!tc::mbar_wait(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort, status)) break;
+          if (!__all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort, status))) break;
           ++nb_groups;
           cur = gi;
           b = pv.g_seq[gi];
@@ -326,7 +326,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           const int blk = __ldg(bv.block_table + (int64_t)b * bv.max_blocks_per_seq + (s >> 6));
           if ((unsigned)blk < (unsigned)bv.num_blocks) ks = __ldg(kscale + (int64_t)blk * 64 + (s & 63));
         }
-        if (!tc::mbar_wait(tc::smem_u32(&S->tfull[acc]), acc_phase, abort, status)) break;
+        // the TMEM loads below are warp-collective: leave the loop together or not at all
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->tfull[acc]), acc_phase, abort, status))) break;
         tc::fence_after_sync();
         const float *wq = sW + bslot * (kIdxWSlotBytes / 4);
         const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + acc * 256;

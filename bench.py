@@ -217,7 +217,8 @@ def run_ours(args, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     dom = max(stage_avg, key=stage_avg.get)
-    roof = roofline_entry(dom, stage_avg[dom], work, peaks, peak_src, args)
+    decode = bool(np.all(wl.q_lens == 1))
+    roof = roofline_entry(dom, stage_avg[dom], work, peaks, peak_src, args, decode)
     clocks = sampler.summary(w0, w1)
     res = {
         "metric": "sparse-attn decode tokens/s" if wl.kind == "mla" and np.all(wl.q_lens == 1)
@@ -249,15 +250,25 @@ def workload_config(wl, args):
     return d
 
 
-def roofline_entry(stage, ms, work, peaks, src, args):
+def roofline_entry(stage, ms, work, peaks, src, args, decode):
+    """Decode stages are HBM-bound (bytes / HBM copy bandwidth); prefill attention and indexer are
+    tensor-bound (flops / dense peak: bf16 for attention, 2x bf16 for the FP8 indexer)."""
     w = work[stage]
     secs = ms / 1e3
-    ach = w["bytes"] / secs / 1e9
-    peak = peaks["hbm_gbs"]
-    return {"kernel": stage, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-            "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback",
-            "algorithmic_bytes_per_launch": w["bytes"], "avg_launch_ms": ms, "traffic": None,
-            "tflops": w["flops"] / secs / 1e12}
+    tag = f"{src} (MEASURED_PEAKS.json)" if src == "measured" else "fallback"
+    if decode or stage == "topk":
+        ach = w["bytes"] / secs / 1e9
+        peak = peaks["hbm_gbs"]
+        return {"kernel": stage, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "peak_source": f"{tag} hbm_gbs", "algorithmic_bytes_per_launch": w["bytes"],
+                "avg_launch_ms": ms, "traffic": None, "tflops": w["flops"] / secs / 1e12}
+    ach = w["flops"] / secs / 1e12
+    fp8 = stage == "indexer"
+    peak = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
+    return {"kernel": stage, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+            "peak_source": f"{tag} bf16_tflops_sustained" + (" x2 (fp8 = 2x bf16 dense ratio)" if fp8 else ""),
+            "algorithmic_flops_per_launch": w["flops"], "avg_launch_ms": ms, "traffic": None,
+            "gbs": w["bytes"] / secs / 1e9}
 
 
 def run_e2e(args, wl, db, stream, dev, world):

@@ -28,6 +28,8 @@
 // Units: prefill = one row (all its chunks); decode = (row, split) pairs whose partial (o, lse) are
 // merged by attn_combine_kernel.  Rows are taken longest-first (reverse order) round-robin over pairs.
 #include <algorithm>
+#include <cstdio>
+#include <cstdlib>
 
 #include "tc.cuh"
 
@@ -95,7 +97,8 @@ __device__ __forceinline__ void unit_of(const AttArgs &a, int u, int *row, int *
 __device__ __forceinline__ int num_units(const AttArgs &a) { return a.T * a.splits; }
 
 // ------------------------------------------------------------------------------------------------ plan
-// neff[row] = 1 + largest j with a usable idx[row, j] (0 if none); flags positions outside [0, seq_len)
+// neff[row] = 1 + largest j with a usable idx[row, j] (0 if none); flags positions outside [0, seq_len).
+// One warp per row; every lane reads 16-byte vectors, all of them issued before any is used.
 __global__ void attn_plan_kernel(const int32_t *__restrict__ idx, int k, BatchView bv, int T, int32_t *neff,
                                  uint32_t *status) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
@@ -106,10 +109,33 @@ __global__ void attn_plan_kernel(const int32_t *__restrict__ idx, int k, BatchVi
   int last = -1;
   bool bad = false;
   const int32_t *ir = idx + (int64_t)warp * k;
-  for (int j = lane; j < k; j += 32) {
-    const int s = __ldg(ir + j);
-    if (s >= 0 && s < seq_len) last = j;
-    else if (s >= seq_len) bad = true;
+  const bool vec = (k & 3) == 0 && (((uintptr_t)ir) & 15) == 0;
+  if (vec) {
+    const int k4 = k >> 2;
+    for (int base = 0; base < k4; base += 32 * 8) {
+      int4 v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j4 = base + e * 32 + lane;
+        v[e] = j4 < k4 ? __ldg(reinterpret_cast<const int4 *>(ir) + j4) : make_int4(-1, -1, -1, -1);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = 4 * (base + e * 32 + lane);
+        const int vals[4] = {v[e].x, v[e].y, v[e].z, v[e].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (vals[c] >= 0 && vals[c] < seq_len) last = max(last, j + c);
+          else if (vals[c] >= seq_len) bad = true;
+        }
+      }
+    }
+  } else {
+    for (int j = lane; j < k; j += 32) {
+      const int s = __ldg(ir + j);
+      if (s >= 0 && s < seq_len) last = j;
+      else if (s >= seq_len) bad = true;
+    }
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
@@ -658,6 +684,7 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
       n = num_sms / 2;
     }
     max_pairs = std::min(n, num_sms / 2);
+    if (getenv("DSA_VERBOSE")) fprintf(stderr, "[libdsa] attention: %d resident CTA pairs\n", max_pairs);
   }
   const int units = a.T * a.splits;
   const int pairs = std::min(max_pairs, units);

@@ -44,6 +44,7 @@ constexpr uint32_t kAttQBytes = 9 * 8192;
 constexpr uint32_t kAttPBytes = 16384;
 constexpr uint32_t kTmemO = 0, kTmemS = 256;     // O: 256 columns; S: two buffers of 64 columns
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kPrefetchAhead = 2;              // chunks of L2 prefetch ahead of the gather
 
 struct AttSmem {
   uint64_t slot_full[kAttSlots];    // local: 128 gather threads (cp.async completion)
@@ -55,8 +56,10 @@ struct AttSmem {
   uint64_t pv_done;                 // MMA commit to both CTAs, once per chunk
   uint64_t o_empty;                 // rank 0: 8 softmax warps after the epilogue read O
   uint64_t drain;
+  uint64_t mask_full[4], mask_empty[4];   // validity masks of upcoming chunks (gather -> softmax)
   uint32_t tmem_base;
   int abort;
+  uint64_t mask[4][2];
   float xm[2][128];
   float xl[2][128];
   int32_t phys[2][kAttChunk];
@@ -175,6 +178,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
     tc::mbar_init(tc::smem_u32(&S->pv_done), 1);
     tc::mbar_init(tc::smem_u32(&S->o_empty), 8);
     tc::mbar_init(tc::smem_u32(&S->drain), 1);
+    for (int i = 0; i < 4; ++i) {
+      tc::mbar_init(tc::smem_u32(&S->mask_full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->mask_empty[i]), 4);
+    }
     S->abort = 0;
     tc::fence_barrier_init();
   }
@@ -196,7 +203,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
     // copies are skipped, so all 128 threads still meet at the same barriers and reach the teardown.
     const int t = threadIdx.x - 128;
     int slot = 0;
-    uint32_t sphase = 0, v = 0;
+    uint32_t sphase = 0, v = 0, gch = 0;
+    // L2 prefetch cursor, kPrefetchAhead chunks ahead of the chunk being gathered: each CTA prefetches the
+    // full latent rows of its own 64 tokens of the chunk (and the next unit's q when the cursor enters it)
+    int pf_u = pair, pf_c = 0, pf_row = -1, pf_cb = 0, pf_nch = 0, pf_seq = 0;
+    const int32_t *pf_btr = nullptr;
+    auto pf_enter = [&](int uu) -> bool {      // position the cursor at chunk 0 of the first non-empty unit >= uu
+      for (; uu < U; uu += npairs) {
+        int r2, cb2, ce2;
+        unit_of(a, uu, &r2, &cb2, &ce2);
+        if (ce2 > cb2) {
+          int b2;
+          pos_of_row(a.bv, r2, &b2);
+          pf_u = uu; pf_c = 0; pf_row = r2; pf_cb = cb2; pf_nch = ce2 - cb2;
+          pf_seq = __ldg(a.bv.seq_lens + b2);
+          pf_btr = a.bv.block_table + (int64_t)b2 * a.bv.max_blocks_per_seq;
+          if (t < 64) {
+            const __nv_bfloat16 *qr = a.q + ((int64_t)r2 * kAttH + 64 * rank + t) * kAttD;
+            tc::prefetch_l2(qr, kAttD * 2);
+          }
+          return true;
+        }
+      }
+      pf_u = U;
+      return false;
+    };
+    auto pf_step = [&]() {                     // prefetch the cursor's chunk, then advance it
+      if (pf_u >= U) return;
+      if (t < 64) {
+        const int j = (pf_cb + pf_c) * kAttChunk + 64 * (int)rank + t;
+        if (j < a.k) {
+          const int s = __ldg(a.idx + (int64_t)pf_row * a.k + j);
+          if (s >= 0 && s < pf_seq) {
+            const int blk = __ldg(pf_btr + (s >> 6));
+            if ((unsigned)blk < (unsigned)a.bv.num_blocks) tc::prefetch_l2(a.kv + ((int64_t)blk * 64 + (s & 63)) * kAttD, kAttD * 2);
+          }
+        }
+      }
+      if (++pf_c == pf_nch) pf_enter(pf_u + npairs);
+    };
+    pf_enter(pair);
+    for (int d = 0; d < kPrefetchAhead; ++d) pf_step();
     for (int u = pair; u < U; u += npairs) {
       int row, cb, ce;
       unit_of(a, u, &row, &cb, &ce);
@@ -220,7 +267,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
       tc::cp_async_arrive_noinc(tc::smem_u32(&S->q_full));
       for (int i = 0; i <= nch; ++i) {
         if (i < nch) {
-          // token positions of chunk i -> physical rows (-1: masked)
+          // token positions of chunk i -> physical rows (-1: masked); the validity mask goes to the softmax
+          pf_step();
+          const uint32_t mslot = gch & 3u;
+          const bool m_ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->mask_empty[mslot]),
+                                                                  ((gch >> 2) & 1u) ^ 1u, abort, status));
           tc::named_bar_sync(1, 128);
           {
             const int j = (cb + i) * kAttChunk + t;
@@ -234,8 +285,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
               }
             }
             S->phys[i & 1][t] = pr;
+            const unsigned bits = __ballot_sync(0xffffffffu, pr >= 0);
+            if (lane == 0 && m_ok) reinterpret_cast<uint32_t *>(S->mask[mslot])[t >> 5] = bits;
           }
           tc::named_bar_sync(1, 128);
+          if (t == 0) tc::mbar_arrive(tc::smem_u32(&S->mask_full[mslot]));
+          ++gch;
           // QK slots: own 64 tokens, dim blocks (2s, 2s+1)
           for (int sl = 0; sl < 5; ++sl) {
             if (tc::mbar_wait_cl(tc::smem_u32(&S->slot_empty[slot]), sphase ^ 1u, abort, status)) {
@@ -411,18 +466,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
       const int seq_len = __ldg(a.bv.seq_lens + b);
       float m_run = -INFINITY, l_run = 0.f, l_exact = 0.f;
       for (int i = 0; i < nch; ++i, ++g) {
-        // validity of this thread's 64 tokens
-        uint64_t valid = 0;
-        {
-          const int j0 = (cb + i) * kAttChunk + 64 * half;
-          const int32_t *ir = a.idx + (int64_t)row * a.k;
-#pragma unroll 8
-          for (int t2 = 0; t2 < 64; ++t2) {
-            const int j = j0 + t2;
-            const int s = j < a.k ? __ldg(ir + j) : -1;
-            if (s >= 0 && s < seq_len) valid |= 1ull << t2;
-          }
-        }
+        // validity of this thread's 64 tokens, published by the gather warps
+        const uint32_t mslot = g & 3u;
+        const bool m_ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->mask_full[mslot]),
+                                                                (g >> 2) & 1u, abort, status));
+        uint64_t valid = m_ok ? S->mask[mslot][half] : 0ull;
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->mask_empty[mslot]));
         const bool have_s = tc::mbar_wait_cl(tc::smem_u32(&S->s_full[g & 1u]), (g >> 1) & 1u, abort, status);
         tc::fence_after_sync();
         float sv[64];

@@ -160,7 +160,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   uint8_t *sA = smem;                                             // kIdxStages x 16 KB
   uint8_t *sB = sA + kIdxStages * kIdxTileBytes;                  // 2 x 32 KB
   float *sW = (float *)(sB + 2 * kIdxBSlotBytes);                 // 2 x 1 KB
-  IdxSmem *S = (IdxSmem *)((uint8_t *)sW + 2 * kIdxWSlotBytes);
+  float *sKS = sW + 2 * (kIdxWSlotBytes / 4);                     // kIdxStages x 128 key scales
+  IdxSmem *S = (IdxSmem *)(sKS + kIdxStages * kIdxTile);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = pv.hdr[0], U = pv.hdr[1];
@@ -170,7 +171,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   if (threadIdx.x == 0) {
     for (int i = 0; i < kIdxStages; ++i) {
       tc::mbar_init(tc::smem_u32(&S->full[i]), 1);
-      tc::mbar_init(tc::smem_u32(&S->empty[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->empty[i]), 1 + 4);      // MMA commit + 4 epilogue warps (key scales)
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(tc::smem_u32(&S->bfull[i]), 1);
@@ -195,73 +196,102 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   volatile int *abort = &S->abort;
 
   if (u0 < u1) {
-    if (warp == 0 && lane == 0) {
-      // ------------------------------------------------------------------ TMA producer
-      int gi, t;
-      unit_locate(pv.tile_prefix, G, u0, &gi, &t);
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer (whole warp)
+      // The 32 lanes look up the block-table entries of the next 32 tiles at once, so the lookups cost
+      // one memory round trip per 32 tiles; lane 0 then issues the copies in order.
       int stage = 0;
       uint32_t phase = 0;
-      int bslot = 0, nb_groups = 0;
+      int nb_groups = 0, cur = -1;
       uint32_t issued = 0, last_par = 0;       // per stage: issued at least once / parity of last issue
       uint32_t b_issued = 0, b_last_par = 0;
-      int cur = -1;
-      for (int u = u0; u < u1; ++u) {
-        if (gi != cur) {
-          bslot = nb_groups & 1;
-          const uint32_t use = (uint32_t)(nb_groups >> 1);
-          if (!tc::mbar_wait(tc::smem_u32(&S->bempty[bslot]), (use & 1u) ^ 1u, abort, status)) break;
-          const int row0 = pv.g_row0[gi], nr = pv.g_nrows[gi];
-          const uint32_t bar = tc::smem_u32(&S->bfull[bslot]);
-          tc::mbar_expect_tx(bar, (uint32_t)nr * (kIdxHi * kIdxDi + kIdxHi * 4));
-          for (int q = 0; q < nr; ++q) {
-            tc::tma_load_2d(tc::smem_u32(sB + bslot * kIdxBSlotBytes + q * kIdxHi * kIdxDi), &tm_q, 0,
-                            (row0 + q) * kIdxHi, bar);
-            tc::bulk_load(tc::smem_u32(sW + bslot * (kIdxWSlotBytes / 4) + q * kIdxHi), w + (int64_t)(row0 + q) * kIdxHi,
-                          kIdxHi * 4, bar);
+      bool ok = true;
+      for (int ub = u0; ub < u1 && ok; ub += 32) {
+        // ---- lane l describes unit ub + l
+        const int u = ub + lane;
+        int gi = 0, t = 0, blk0 = -1, blk1 = -1;
+        if (u < u1) {
+          unit_locate(pv.tile_prefix, G, u, &gi, &t);
+          const int b = pv.g_seq[gi];
+          const int c0 = __ldg(bv.cu_q + b), nbq = __ldg(bv.cu_q + b + 1) - c0;
+          const int pos_last = __ldg(bv.seq_lens + b) - nbq + (pv.g_row0[gi] - c0) + pv.g_nrows[gi] - 1;
+          const int pages = pos_last / 64 + 1;
+          const int32_t *btr = bv.block_table + (int64_t)b * bv.max_blocks_per_seq;
+          blk0 = __ldg(btr + 2 * t);
+          if (2 * t + 1 < pages) blk1 = __ldg(btr + 2 * t + 1);
+          if ((unsigned)blk0 >= (unsigned)bv.num_blocks) { set_status(status, kStatusBadIndex); blk0 = -1; }
+          if (2 * t + 1 < pages && (unsigned)blk1 >= (unsigned)bv.num_blocks) {
+            set_status(status, kStatusBadIndex);
+            blk1 = -1;
           }
-          b_issued |= 1u << bslot;
-          b_last_par = (b_last_par & ~(1u << bslot)) | ((use & 1u) << bslot);
-          ++nb_groups;
-          cur = gi;
         }
-        if (!tc::mbar_wait(tc::smem_u32(&S->empty[stage]), phase ^ 1u, abort, status)) break;
-        const int b = pv.g_seq[gi];
-        const int nrw = pv.g_nrows[gi];
-        const int nbq = __ldg(bv.cu_q + b + 1) - __ldg(bv.cu_q + b);
-        const int pos_last = __ldg(bv.seq_lens + b) - nbq + (pv.g_row0[gi] - __ldg(bv.cu_q + b)) + nrw - 1;
-        const int pages = pos_last / 64 + 1;
-        const int p0 = 2 * t, p1 = 2 * t + 1;
-        const int32_t *btr = bv.block_table + (int64_t)b * bv.max_blocks_per_seq;
-        int blk0 = __ldg(btr + p0);
-        int blk1 = p1 < pages ? __ldg(btr + p1) : -1;
-        if ((unsigned)blk0 >= (unsigned)bv.num_blocks) { set_status(status, kStatusBadIndex); blk0 = -1; }
-        if (p1 < pages && (unsigned)blk1 >= (unsigned)bv.num_blocks) { set_status(status, kStatusBadIndex); blk1 = -1; }
-        const uint32_t bar = tc::smem_u32(&S->full[stage]);
-        const uint32_t bytes = (blk0 >= 0 ? kIdxPageBytes : 0u) + (blk1 >= 0 ? kIdxPageBytes : 0u);
-        if (bytes) {
-          tc::mbar_expect_tx(bar, bytes);
-          if (blk0 >= 0) tc::tma_load_2d(tc::smem_u32(sA + stage * kIdxTileBytes), &tm_k, 0, blk0 * 64, bar);
-          if (blk1 >= 0)
-            tc::tma_load_2d(tc::smem_u32(sA + stage * kIdxTileBytes + kIdxPageBytes), &tm_k, 0, blk1 * 64, bar);
-        } else {
-          tc::mbar_arrive(bar);
+        const int n = min(32, u1 - ub);
+        for (int j = 0; j < n; ++j) {
+          const int gj = __shfl_sync(0xffffffffu, gi, j);
+          const int b0 = __shfl_sync(0xffffffffu, blk0, j);
+          const int b1 = __shfl_sync(0xffffffffu, blk1, j);
+          if (lane == 0) {
+            if (gj != cur) {
+              const int bslot = nb_groups & 1;
+              const uint32_t use = (uint32_t)(nb_groups >> 1);
+              ok = tc::mbar_wait(tc::smem_u32(&S->bempty[bslot]), (use & 1u) ^ 1u, abort, status);
+              if (ok) {
+                const int row0 = pv.g_row0[gj], nr = pv.g_nrows[gj];
+                const uint32_t bar = tc::smem_u32(&S->bfull[bslot]);
+                tc::mbar_expect_tx(bar, (uint32_t)nr * (kIdxHi * kIdxDi + kIdxHi * 4));
+                for (int q = 0; q < nr; ++q) {
+                  tc::tma_load_2d(tc::smem_u32(sB + bslot * kIdxBSlotBytes + q * kIdxHi * kIdxDi), &tm_q, 0,
+                                  (row0 + q) * kIdxHi, bar);
+                  tc::bulk_load(tc::smem_u32(sW + bslot * (kIdxWSlotBytes / 4) + q * kIdxHi),
+                                w + (int64_t)(row0 + q) * kIdxHi, kIdxHi * 4, bar);
+                }
+                b_issued |= 1u << bslot;
+                b_last_par = (b_last_par & ~(1u << bslot)) | ((use & 1u) << bslot);
+              }
+              ++nb_groups;
+              cur = gj;
+            }
+            if (ok) ok = tc::mbar_wait(tc::smem_u32(&S->empty[stage]), phase ^ 1u, abort, status);
+            if (ok) {
+              const uint32_t bar = tc::smem_u32(&S->full[stage]);
+              const uint32_t bytes = (b0 >= 0 ? kIdxPageBytes + 256u : 0u) + (b1 >= 0 ? kIdxPageBytes + 256u : 0u);
+              if (bytes) {
+                tc::mbar_expect_tx(bar, bytes);
+                const uint32_t a_dst = tc::smem_u32(sA + stage * kIdxTileBytes);
+                const uint32_t k_dst = tc::smem_u32(sKS + stage * kIdxTile);
+                if (b0 >= 0) {
+                  tc::tma_load_2d(a_dst, &tm_k, 0, b0 * 64, bar);
+                  tc::bulk_load(k_dst, kscale + (int64_t)b0 * 64, 256, bar);
+                }
+                if (b1 >= 0) {
+                  tc::tma_load_2d(a_dst + kIdxPageBytes, &tm_k, 0, b1 * 64, bar);
+                  tc::bulk_load(k_dst + 256, kscale + (int64_t)b1 * 64, 256, bar);
+                }
+              } else {
+                tc::mbar_arrive(bar);
+              }
+              issued |= 1u << stage;
+              last_par = (last_par & ~(1u << stage)) | (phase << stage);
+              if (++stage == kIdxStages) { stage = 0; phase ^= 1u; }
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
         }
-        issued |= 1u << stage;
-        last_par = (last_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == kIdxStages) { stage = 0; phase ^= 1u; }
-        if (++t == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) { ++gi; t = 0; }
       }
       // never leave with copies in flight: wait for the last fill of every stage / slot
-      for (int s = 0; s < kIdxStages; ++s)
-        if (issued & (1u << s)) {
-          volatile int no_abort = 0;
-          tc::mbar_wait(tc::smem_u32(&S->full[s]), (last_par >> s) & 1u, &no_abort, status);
-        }
-      for (int s = 0; s < 2; ++s)
-        if (b_issued & (1u << s)) {
-          volatile int no_abort = 0;
-          tc::mbar_wait(tc::smem_u32(&S->bfull[s]), (b_last_par >> s) & 1u, &no_abort, status);
-        }
+      if (lane == 0) {
+        for (int s2 = 0; s2 < kIdxStages; ++s2)
+          if (issued & (1u << s2)) {
+            volatile int no_abort = 0;
+            tc::mbar_wait(tc::smem_u32(&S->full[s2]), (last_par >> s2) & 1u, &no_abort, status);
+          }
+        for (int s2 = 0; s2 < 2; ++s2)
+          if (b_issued & (1u << s2)) {
+            volatile int no_abort = 0;
+            tc::mbar_wait(tc::smem_u32(&S->bfull[s2]), (b_last_par >> s2) & 1u, &no_abort, status);
+          }
+      }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------------ MMA issuer
       int gi, t;
@@ -321,14 +351,16 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           pos0 = __ldg(bv.seq_lens + b) - (__ldg(bv.cu_q + b + 1) - c0) + (row0 - c0);
         }
         const int s = t * kIdxTile + key_local;
-        float ks = 0.f;
-        if (s <= pos0 + nr - 1) {
-          const int blk = __ldg(bv.block_table + (int64_t)b * bv.max_blocks_per_seq + (s >> 6));
-          if ((unsigned)blk < (unsigned)bv.num_blocks) ks = __ldg(kscale + (int64_t)blk * 64 + (s & 63));
-        }
         // the TMEM loads below are warp-collective: leave the loop together or not at all
         if (!__all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->tfull[acc]), acc_phase, abort, status))) break;
         tc::fence_after_sync();
+        // the tile's key scales arrived with it; the stage's fill has completed (the MMA consumed it), the
+        // wait below returns at once and orders the bulk copy before these reads
+        const int stage = (u - u0) % kIdxStages;
+        tc::mbar_wait(tc::smem_u32(&S->full[stage]), (uint32_t)((u - u0) / kIdxStages) & 1u, abort, status);
+        const float ks = sKS[stage * kIdxTile + key_local];
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->empty[stage]));
         const float *wq = sW + bslot * (kIdxWSlotBytes / 4);
         const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + acc * 256;
         for (int q = 0; q < nr; ++q) {
@@ -399,7 +431,8 @@ static bool make_rows128_map(CUtensorMap *m, const void *base, uint64_t rows) {
 }
 
 static size_t indexer_tc_smem() {
-  return 1024 + kIdxStages * kIdxTileBytes + 2 * kIdxBSlotBytes + 2 * kIdxWSlotBytes + sizeof(IdxSmem);
+  return 1024 + kIdxStages * kIdxTileBytes + 2 * kIdxBSlotBytes + 2 * kIdxWSlotBytes + kIdxStages * kIdxTile * 4 +
+         sizeof(IdxSmem);
 }
 
 dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t *kpool, const float *kscale,

@@ -47,7 +47,7 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr int kPrefetchAhead = 2;              // chunks of L2 prefetch ahead of the gather
 
 struct AttSmem {
-  uint64_t slot_full[kAttSlots];    // local: 128 gather threads (cp.async completion)
+  uint64_t slot_full[kAttSlots];    // local: TMA transaction bytes (one expect_tx per fill)
   uint64_t pair_full[kAttSlots];    // rank 0: 2 relays
   uint64_t slot_empty[kAttSlots];   // MMA commit to both CTAs
   uint64_t q_full, pair_q_full, q_empty;
@@ -150,7 +150,8 @@ __global__ void attn_plan_kernel(const int32_t *__restrict__ idx, int k, BatchVi
 }
 
 // ------------------------------------------------------------------------------------------------ main
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn_mla_kernel(const AttArgs a) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
+    attn_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv, const AttArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sQ = smem;
@@ -165,11 +166,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kAttSlots; ++i) {
-      tc::mbar_init(tc::smem_u32(&S->slot_full[i]), 128);
+      tc::mbar_init(tc::smem_u32(&S->slot_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&S->pair_full[i]), 2);
       tc::mbar_init(tc::smem_u32(&S->slot_empty[i]), 1);
     }
-    tc::mbar_init(tc::smem_u32(&S->q_full), 128);
+    tc::mbar_init(tc::smem_u32(&S->q_full), 1);
     tc::mbar_init(tc::smem_u32(&S->pair_q_full), 2);
     tc::mbar_init(tc::smem_u32(&S->q_empty), 1);
     tc::mbar_init(tc::smem_u32(&S->s_full[0]), 1);
@@ -199,10 +200,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
 
   if (warp >= 4 && warp < 8) {
     // ====================================================================== gather (128 threads)
-    // Loops holding the named barrier never break: after a timeout every wait returns at once and the
-    // copies are skipped, so all 128 threads still meet at the same barriers and reach the teardown.
-    const int t = threadIdx.x - 128;
-    int slot = 0;
+    // q arrives by one tiled TMA per dim block; selected latent rows by TMA gather4 (4 rows x 128 bytes per
+    // instruction, 128-byte swizzle applied by the copy engine).  Each 16 KB ring slot is filled by one of
+    // the four gather warps (one gather4 per lane), round-robin over slots.  Loops holding the named
+    // barrier never break: after a timeout every wait returns at once and the copies are skipped, so all
+    // 128 threads still meet at the same barriers and reach the teardown.
+    const int t = threadIdx.x - 128, pw = t >> 5;
+    const int oob_row = a.bv.num_blocks * 64;           // outside the map: the copy engine fills zeros
+    int slot = 0, fill = 0;
     uint32_t sphase = 0, v = 0, gch = 0;
     // L2 prefetch cursor, kPrefetchAhead chunks ahead of the chunk being gathered: each CTA prefetches the
     // full latent rows of its own 64 tokens of the chunk (and the next unit's q when the cursor enters it)
@@ -242,6 +247,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
       }
       if (++pf_c == pf_nch) pf_enter(pf_u + npairs);
     };
+    // fill one ring slot with 32 gather4 copies: lane -> (dim block d(lane), tokens 4*(lane%16) + [0,4) of
+    // the 64 tokens starting at chunk token key0); blocks with d < 0 are skipped
+    auto fill_slot = [&](int chunk_parity, int key0, int d0, int d1) {
+      const bool mine = (fill & 3) == pw;
+      if (mine) {
+        const int nblk = d1 >= 0 ? 2 : 1;
+        bool ok = true;
+        if (lane == 0) {
+          ok = tc::mbar_wait_cl(tc::smem_u32(&S->slot_empty[slot]), sphase ^ 1u, abort, status);
+          if (ok) tc::mbar_expect_tx(tc::smem_u32(&S->slot_full[slot]), (uint32_t)nblk * 64 * 128);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        const int blk = lane >> 4, g4 = lane & 15;
+        if (ok && blk < nblk) {
+          const int d = blk ? d1 : d0;
+          const int32_t *ph = S->phys[chunk_parity] + key0 + 4 * g4;
+          int r[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) r[e] = ph[e] >= 0 ? ph[e] : oob_row;
+          tc::tma_gather4(tc::smem_u32(sRing + slot * kAttSlotBytes + blk * 8192 + 4 * g4 * 128), &tm_kv, d * 64, r[0],
+                          r[1], r[2], r[3], tc::smem_u32(&S->slot_full[slot]));
+        }
+      }
+      ++fill;
+      if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
+    };
     pf_enter(pair);
     for (int d = 0; d < kPrefetchAhead; ++d) pf_step();
     for (int u = pair; u < U; u += npairs) {
@@ -254,17 +285,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
       const int seq_len = __ldg(a.bv.seq_lens + b);
       const int32_t *btr = a.bv.block_table + (int64_t)b * a.bv.max_blocks_per_seq;
       // ---- q: this CTA's 64 heads, [9 dim blocks][64 heads][128 B], 128-byte swizzle
-      bool ok = v == 0 || tc::mbar_wait_cl(tc::smem_u32(&S->q_empty), (v - 1) & 1u, abort, status);
-      if (ok) {
-        const __nv_bfloat16 *qr = a.q + ((int64_t)row * kAttH + 64 * rank) * kAttD;
-        const uint32_t qbase = tc::smem_u32(sQ);
-        for (int id = t; id < 64 * 72; id += 128) {
-          const int h = id / 72, rem = id % 72, d = rem >> 3, c = rem & 7;
-          tc::cp_async16(qbase + d * 8192 + h * 128 + ((c ^ (h & 7)) << 4), qr + (int64_t)h * kAttD + d * 64 + c * 8,
-                         16);
+      if (t == 0) {
+        const bool ok = v == 0 || tc::mbar_wait_cl(tc::smem_u32(&S->q_empty), (v - 1) & 1u, abort, status);
+        if (ok) {
+          const uint32_t bar = tc::smem_u32(&S->q_full);
+          tc::mbar_expect_tx(bar, kAttQBytes);
+          for (int d = 0; d < 9; ++d)
+            tc::tma_load_2d(tc::smem_u32(sQ + d * 8192), &tm_q, d * 64, row * kAttH + 64 * (int)rank, bar);
         }
       }
-      tc::cp_async_arrive_noinc(tc::smem_u32(&S->q_full));
       for (int i = 0; i <= nch; ++i) {
         if (i < nch) {
           // token positions of chunk i -> physical rows (-1: masked); the validity mask goes to the softmax
@@ -291,51 +320,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1) attn
           tc::named_bar_sync(1, 128);
           if (t == 0) tc::mbar_arrive(tc::smem_u32(&S->mask_full[mslot]));
           ++gch;
-          // QK slots: own 64 tokens, dim blocks (2s, 2s+1)
-          for (int sl = 0; sl < 5; ++sl) {
-            if (tc::mbar_wait_cl(tc::smem_u32(&S->slot_empty[slot]), sphase ^ 1u, abort, status)) {
-              const uint32_t base = tc::smem_u32(sRing + slot * kAttSlotBytes);
-#pragma unroll
-              for (int m = 0; m < 8; ++m) {
-                const int id = t + 128 * m;
-                const int kr = id >> 4, blk = (id >> 3) & 1, c = id & 7;
-                const int d = 2 * sl + blk;
-                if (d < 9) {
-                  const int32_t pr = S->phys[i & 1][64 * rank + kr];
-                  const __nv_bfloat16 *src = pr >= 0 ? a.kv + (int64_t)pr * kAttD + d * 64 + c * 8 : a.kv;
-                  tc::cp_async16(base + blk * 8192 + kr * 128 + ((c ^ (kr & 7)) << 4), src, pr >= 0 ? 16u : 0u);
-                }
-              }
-            }
-            tc::cp_async_arrive_noinc(tc::smem_u32(&S->slot_full[slot]));
-            if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
-          }
+          // QK slots: this CTA's 64 tokens, dim blocks (2s, 2s+1)
+          for (int sl = 0; sl < 5; ++sl) fill_slot(i & 1, 64 * (int)rank, 2 * sl, 2 * sl + 1 < 9 ? 2 * sl + 1 : -1);
         }
         if (i > 0) {
           // PV slots of chunk i-1: value blocks (4r + 2p, 4r + 2p + 1) of token half kh
-          const int pc = (i - 1) & 1;
           for (int p = 0; p < 2; ++p)
-            for (int kh = 0; kh < 2; ++kh) {
-              if (tc::mbar_wait_cl(tc::smem_u32(&S->slot_empty[slot]), sphase ^ 1u, abort, status)) {
-                const uint32_t base = tc::smem_u32(sRing + slot * kAttSlotBytes);
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                  const int id = t + 128 * m;
-                  const int kr = id >> 4, blk = (id >> 3) & 1, c = id & 7;
-                  const int d = 4 * rank + 2 * p + blk;
-                  const int32_t pr = S->phys[pc][64 * kh + kr];
-                  const __nv_bfloat16 *src = pr >= 0 ? a.kv + (int64_t)pr * kAttD + d * 64 + c * 8 : a.kv;
-                  tc::cp_async16(base + blk * 8192 + kr * 128 + ((c ^ (kr & 7)) << 4), src, pr >= 0 ? 16u : 0u);
-                }
-              }
-              tc::cp_async_arrive_noinc(tc::smem_u32(&S->slot_full[slot]));
-              if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
-            }
+            for (int kh = 0; kh < 2; ++kh) fill_slot((i - 1) & 1, 64 * kh, 4 * (int)rank + 2 * p, 4 * (int)rank + 2 * p + 1);
         }
       }
       ++v;
     }
-    tc::cp_async_wait_all();
   } else if (warp == 9) {
     // ====================================================================== relay (lane 0)
     if (lane == 0) {
@@ -683,6 +678,24 @@ size_t attn_workspace_bytes(int T, int k, bool decode) {
   return bytes;
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+// bf16 matrix [rows, 576] read in boxes of `box_rows` rows x 64 columns (128 bytes) with the 128-byte swizzle
+static bool make_bf16_rows_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kAttD, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kAttD * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static size_t attn_smem_bytes() { return 1024 + kAttQBytes + kAttSlots * kAttSlotBytes + kAttPBytes + sizeof(AttSmem); }
 
 dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, int k, float softmax_scale,
@@ -709,6 +722,12 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
   } else {
     a.out = (__nv_bfloat16 *)out;
     a.lse = lse;
+  }
+  CUtensorMap tm_q, tm_kv;
+  if (!make_bf16_rows_map(&tm_q, q, (uint64_t)a.T * kAttH, 64) ||
+      !make_bf16_rows_map(&tm_kv, kv, (uint64_t)b->num_blocks * 64, 1)) {
+    set_error("attention: cuTensorMapEncodeTiled failed");
+    return DSA_ERR_CUDA;
   }
   attn_plan_kernel<<<(a.T + 3) / 4, 128, 0, stream>>>(idx, k, a.bv, a.T, neff, a.status);
   DSA_LAUNCH_CHECK("attn_plan_kernel");
@@ -738,7 +757,7 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
   }
   const int units = a.T * a.splits;
   const int pairs = std::min(max_pairs, units);
-  attn_mla_kernel<<<2 * pairs, kAttThreads, smem, stream>>>(a);
+  attn_mla_kernel<<<2 * pairs, kAttThreads, smem, stream>>>(tm_q, tm_kv, a);
   DSA_LAUNCH_CHECK("attn_mla_kernel");
   if (a.splits > 1) {
     attn_combine_kernel<<<dim3(a.T, kAttH), 128, 0, stream>>>(a.part_o, a.part_lse, a.splits, (__nv_bfloat16 *)out,

@@ -151,20 +151,9 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
     const int nb = pass == 2 ? 1024 : 2048;
     for (int i = tid; i < nb; i += bs) hist[i] = 0u;
     __syncthreads();
-    if (pass == 0) {
-      // the leading digit of float keys crowds into a few bins: combine equal bins within a warp first
-      const int n_pad = (n + bs - 1) / bs * bs;
-      for (int i = tid; i < n_pad; i += bs) {
-        const uint32_t u = i < n ? keys[i] : 0u;
-        const uint32_t bin = i < n ? (u >> shift) & (nb - 1) : 0xFFFFFFFFu;
-        const unsigned same = __match_any_sync(0xffffffffu, bin);
-        if (i < n && (threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
-      }
-    } else {
-      for (int i = tid; i < n; i += bs) {
-        uint32_t u = keys[i];
-        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & (nb - 1)], 1u);
-      }
+    for (int i = tid; i < n; i += bs) {
+      uint32_t u = keys[i];
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & (nb - 1)], 1u);
     }
     __syncthreads();
     find_threshold_bin(hist, nb, k_rem, tmp, &s_bin, &s_above);

@@ -14,8 +14,9 @@
 // per-thread reduction with no shuffles.  A 128-key tile is two 64-token pages fetched by TMA through
 // the block table (128-byte swizzle, the layout the MMA descriptor reads).
 //
-// Warp roles (192 threads, persistent, one CTA per SM):
-//   warp 0       TMA producer: query rows + weights of a row group, then key tiles into an 8-stage ring
+// Warp roles (288 threads, persistent, one CTA per SM):
+//   warps 0,6-8  TMA producers: key tiles into an 8-stage ring (round-robin over the four warps); warp 0
+//                also loads the query rows + weights of each row group
 //   warp 1       allocates 512 TMEM columns; lane 0 issues 4 MMAs (K = 32 each) per tile into one of two
 //                256-column accumulators and commits them to the ring / accumulator barriers
 //   warps 2..5   epilogue: tcgen05.ld 64 heads per row, ReLU, weight, sum, key scale, causal store
@@ -28,7 +29,7 @@ namespace dsa {
 constexpr int kIdxTile = 128;
 constexpr int kIdxRows = 4;
 constexpr int kIdxStages = 8;
-constexpr int kIdxThreads = 192;
+constexpr int kIdxThreads = 288;                  // warps 0, 6-8 TMA, 1 MMA, 2-5 epilogue
 constexpr int kIdxHi = 64, kIdxDi = 128;
 constexpr uint32_t kIdxTileBytes = kIdxTile * kIdxDi;         // 16 KB
 constexpr uint32_t kIdxPageBytes = 64 * kIdxDi;               // 8 KB
@@ -196,21 +197,47 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   volatile int *abort = &S->abort;
 
   if (u0 < u1) {
-    if (warp == 0) {
-      // ------------------------------------------------------------------ TMA producer (whole warp)
-      // The 32 lanes look up the block-table entries of the next 32 tiles at once, so the lookups cost
-      // one memory round trip per 32 tiles; lane 0 then issues the copies in order.
-      int stage = 0;
-      uint32_t phase = 0;
-      int nb_groups = 0, cur = -1;
-      uint32_t issued = 0, last_par = 0;       // per stage: issued at least once / parity of last issue
+    if (warp == 0 || warp >= 6) {
+      // ------------------------------------------------------------------ TMA producers (4 warps)
+      // Key tiles are spread over four producer warps (a tile's stage is fixed by its position, so each
+      // warp owns two of the eight stages): the copy engine takes several warps' copies at once.  Each
+      // warp looks up the block-table entries of its next 32 tiles in one memory round trip.  Warp 0 also
+      // loads the query rows + weights of every row group, in order.
+      const int pw = warp == 0 ? 0 : warp - 5;              // 0..3
+      uint32_t issued = 0, last_par = 0;                    // stages this warp filled / parity of last fill
       uint32_t b_issued = 0, b_last_par = 0;
       bool ok = true;
-      for (int ub = u0; ub < u1 && ok; ub += 32) {
-        // ---- lane l describes unit ub + l
-        const int u = ub + lane;
+      // ---- row-group (B operand) loads, warp 0: all groups of the range in order, ahead of the tiles
+      auto load_group = [&](int gj, int nbg) -> bool {
+        const int bslot = nbg & 1;
+        const uint32_t use = (uint32_t)(nbg >> 1);
+        if (!tc::mbar_wait(tc::smem_u32(&S->bempty[bslot]), (use & 1u) ^ 1u, abort, status)) return false;
+        const int row0 = pv.g_row0[gj], nr = pv.g_nrows[gj];
+        const uint32_t bar = tc::smem_u32(&S->bfull[bslot]);
+        tc::mbar_expect_tx(bar, (uint32_t)nr * (kIdxHi * kIdxDi + kIdxHi * 4));
+        for (int q = 0; q < nr; ++q) {
+          tc::tma_load_2d(tc::smem_u32(sB + bslot * kIdxBSlotBytes + q * kIdxHi * kIdxDi), &tm_q, 0, (row0 + q) * kIdxHi,
+                          bar);
+          tc::bulk_load(tc::smem_u32(sW + bslot * (kIdxWSlotBytes / 4) + q * kIdxHi), w + (int64_t)(row0 + q) * kIdxHi,
+                        kIdxHi * 4, bar);
+        }
+        b_issued |= 1u << bslot;
+        b_last_par = (b_last_par & ~(1u << bslot)) | ((use & 1u) << bslot);
+        return true;
+      };
+      int g_next = 0, g_cur = -1, g_count = 0, g_last = -1;   // warp 0: groups loaded so far
+      if (pw == 0) {
+        int t0;
+        unit_locate(pv.tile_prefix, G, u0, &g_next, &t0);
+        unit_locate(pv.tile_prefix, G, u1 - 1, &g_last, &t0);
+      }
+      const int mine = (u1 - u0 - pw + 3) / 4;              // tiles of this warp: u0 + pw + 4 m
+      for (int mb = 0; mb < mine && ok; mb += 32) {
+        // ---- lane l describes tile m = mb + l of this warp
+        const int m = mb + lane;
+        const int u = u0 + pw + 4 * m;
         int gi = 0, t = 0, blk0 = -1, blk1 = -1;
-        if (u < u1) {
+        if (m < mine) {
           unit_locate(pv.tile_prefix, G, u, &gi, &t);
           const int b = pv.g_seq[gi];
           const int c0 = __ldg(bv.cu_q + b), nbq = __ldg(bv.cu_q + b + 1) - c0;
@@ -225,32 +252,22 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             blk1 = -1;
           }
         }
-        const int n = min(32, u1 - ub);
+        const int n = min(32, mine - mb);
         for (int j = 0; j < n; ++j) {
           const int gj = __shfl_sync(0xffffffffu, gi, j);
           const int b0 = __shfl_sync(0xffffffffu, blk0, j);
           const int b1 = __shfl_sync(0xffffffffu, blk1, j);
           if (lane == 0) {
-            if (gj != cur) {
-              const int bslot = nb_groups & 1;
-              const uint32_t use = (uint32_t)(nb_groups >> 1);
-              ok = tc::mbar_wait(tc::smem_u32(&S->bempty[bslot]), (use & 1u) ^ 1u, abort, status);
-              if (ok) {
-                const int row0 = pv.g_row0[gj], nr = pv.g_nrows[gj];
-                const uint32_t bar = tc::smem_u32(&S->bfull[bslot]);
-                tc::mbar_expect_tx(bar, (uint32_t)nr * (kIdxHi * kIdxDi + kIdxHi * 4));
-                for (int q = 0; q < nr; ++q) {
-                  tc::tma_load_2d(tc::smem_u32(sB + bslot * kIdxBSlotBytes + q * kIdxHi * kIdxDi), &tm_q, 0,
-                                  (row0 + q) * kIdxHi, bar);
-                  tc::bulk_load(tc::smem_u32(sW + bslot * (kIdxWSlotBytes / 4) + q * kIdxHi),
-                                w + (int64_t)(row0 + q) * kIdxHi, kIdxHi * 4, bar);
-                }
-                b_issued |= 1u << bslot;
-                b_last_par = (b_last_par & ~(1u << bslot)) | ((use & 1u) << bslot);
+            // warp 0 keeps the group loads at least up to the group of its current tile
+            if (pw == 0)
+              while (ok && g_cur < gj) {
+                ok = load_group(g_next, g_count);
+                g_cur = g_next++;
+                ++g_count;
               }
-              ++nb_groups;
-              cur = gj;
-            }
+            const int q = (mb + j) * 4 + pw;                // position of the tile in this CTA's range
+            const int stage = q % kIdxStages;
+            const uint32_t phase = (uint32_t)(q / kIdxStages) & 1u;
             if (ok) ok = tc::mbar_wait(tc::smem_u32(&S->empty[stage]), phase ^ 1u, abort, status);
             if (ok) {
               const uint32_t bar = tc::smem_u32(&S->full[stage]);
@@ -272,14 +289,19 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
               }
               issued |= 1u << stage;
               last_par = (last_par & ~(1u << stage)) | (phase << stage);
-              if (++stage == kIdxStages) { stage = 0; phase ^= 1u; }
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
         }
       }
-      // never leave with copies in flight: wait for the last fill of every stage / slot
+      if (lane == 0 && pw == 0)      // groups of the range not reached by warp 0's own tiles
+        while (ok && g_cur < g_last) {
+          ok = load_group(g_next, g_count);
+          g_cur = g_next++;
+          ++g_count;
+        }
+      // never leave with copies in flight: wait for the last fill of every stage / slot this warp issued
       if (lane == 0) {
         for (int s2 = 0; s2 < kIdxStages; ++s2)
           if (issued & (1u << s2)) {
@@ -329,7 +351,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       tc::mma_commit(tc::smem_u32(&S->drain));
       volatile int no_abort = 0;
       tc::mbar_wait(tc::smem_u32(&S->drain), 0, &no_abort, status);
-    } else if (warp >= 2) {
+    } else if (warp >= 2 && warp < 6) {
       // ------------------------------------------------------------------ epilogue
       const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
       const int key_local = quad * 32 + lane;

@@ -134,6 +134,20 @@ DSA_API dsa_status_t dsa_indexer_scores(const void *q_idx, dsa_dtype_t q_dt, con
 DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_batch_t *b, int32_t k,
                       int32_t *idx, void *ws, size_t ws_bytes, void *stream);
 
+/* Allocation-free top-k.  There is no counterpart in the pages: this entry point exists for callers
+ * that cannot allocate device memory for a workspace -- code that runs where cudaMalloc is not allowed
+ * or not wanted (a plugin or custom operator handed only a stream, a framework whose memory is owned
+ * by its own pool, a latency-critical path that must not trigger an allocation and its implicit device
+ * synchronisation).  Same selection and output as dsa_topk, but its scratch is a fixed device array
+ * inside the library (about 2.3 MB per device, held until the process exits) instead of a caller
+ * workspace.  Limits: total_q <= 256 rows and max_seq_len <= 1,048,576 candidates; larger batches return
+ * DSA_ERR_UNSUPPORTED with nothing enqueued.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) and caches it; make that first call outside any stream capture.  All
+ * calls share the one array, so calls whose GPU work overlaps (different streams, concurrent host
+ * threads) race on it; serialise them on one stream.  Allocates nothing: no cudaMalloc/cudaFree. */
+DSA_API dsa_status_t dsa_topk_noalloc(const float *scores, int64_t ld_scores, const dsa_batch_t *b, int32_t k,
+                                      int32_t *idx, void *stream);
+
 /* Sparse attention, prefill / any batch ("Day-0 Adaptation for LLMs ...", decode sketch:
  * gather the selected KV and run exact attention; "Day-0 Model Adaptation Depends on the
  * Compute Software Stack", Operator Library Abstraction: query, key-value pairs and index

@@ -21,7 +21,7 @@ DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_ATTN_PREFILL, DSA_OP_ATTN_DECODE = 0, 1, 2, 
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn_prefill",
            "dsa_sparse_attn_decode", "dsa_read_device_status", "dsa_status_string", "dsa_last_error",
-           "dsa_version", "dsa_launch_count")
+           "dsa_version", "dsa_launch_count", "dsa_topk_noalloc")
 
 
 class dsa_batch_t(ctypes.Structure):
@@ -63,6 +63,7 @@ def load(path: str = LIB_PATH):
         "dsa_workspace_size": [I32, B, I32, I32, I32, ctypes.POINTER(SZ)],
         "dsa_indexer_scores": [P, I32, P, P, I32, P, I32, I32, B, P, I64, P, SZ, P],
         "dsa_topk": [P, I64, B, I32, P, P, SZ, P],
+        "dsa_topk_noalloc": [P, I64, B, I32, P, P],
         "dsa_sparse_attn_prefill": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
         "dsa_sparse_attn_decode": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
         "dsa_read_device_status": [P, P],
@@ -131,6 +132,12 @@ def dsa_indexer_scores(q_idx, q_dt: int, w, k_idx_pool, k_dt: int, k_scale_pool,
 def dsa_topk(scores, ld_scores: int, batch: dsa_batch_t, k: int, idx, ws, ws_bytes: int, stream=None):
     _check(load().dsa_topk(_ptr(scores), ld_scores, ctypes.byref(batch), k, _ptr(idx), _ptr(ws), ws_bytes,
                            _stream(stream)), "dsa_topk")
+
+
+def dsa_topk_noalloc(scores, ld_scores: int, batch: dsa_batch_t, k: int, idx, stream=None):
+    """Top-k with the library's built-in scratch instead of a caller workspace (no device allocation)."""
+    _check(load().dsa_topk_noalloc(_ptr(scores), ld_scores, ctypes.byref(batch), k, _ptr(idx), _stream(stream)),
+           "dsa_topk_noalloc")
 
 
 def dsa_sparse_attn_prefill(q, dt: int, kv_pool, v_pool, H: int, Dqk: int, Dv: int, softmax_scale: float, idx,

@@ -14,6 +14,8 @@ namespace dsa {
 dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx, void *ws,
                          cudaStream_t stream, int num_sms);
 size_t topk_workspace_bytes(int total_q, int max_seq_len);
+dsa_status_t topk_noalloc_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx,
+                                 cudaStream_t stream, int num_sms);
 dsa_status_t indexer_simt_launch(const void *qI, dsa_dtype_t dt, const float *w, const void *kpool,
                                  const float *kscale, int Hi, int Di, const dsa_batch_t *b, float *scores,
                                  int64_t ld, cudaStream_t stream);
@@ -214,6 +216,21 @@ dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_batch_t 
   if ((st = current_device(&dev)) != DSA_OK) return st;
   if (b->total_q == 0) return DSA_OK;
   return topk_launch(scores, ld_scores, b, k, idx, ws, (cudaStream_t)stream, dev.num_sms);
+}
+
+dsa_status_t dsa_topk_noalloc(const float *scores, int64_t ld_scores, const dsa_batch_t *b, int32_t k,
+                              int32_t *idx, void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  CHECK_ARG(scores && idx, "scores and idx are required");
+  CHECK_SUP(k >= 1 && k <= 16384, "k must be in [1, 16384] (got %d)", k);
+  CHECK_ARG(ld_scores >= b->max_seq_len && ld_scores % 4 == 0,
+            "ld_scores (%lld) must be >= max_seq_len and a multiple of 4", (long long)ld_scores);
+  CHECK_ARG(((uintptr_t)scores & 15) == 0, "scores must be 16-byte aligned");
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;
+  return topk_noalloc_launch(scores, ld_scores, b, k, idx, (cudaStream_t)stream, dev.num_sms);
 }
 
 static dsa_status_t attn_common(bool decode, const void *q, dsa_dtype_t dt, const void *kv_pool, const void *v_pool,

@@ -18,6 +18,8 @@
 //      per-row global histogram, and the last CTA of a row to finish (atomic counter, no waiting)
 //      picks the digit.  Then a count launch and an ordered-write launch.  No CTA ever waits for
 //      another.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace dsa {
@@ -354,11 +356,7 @@ dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, 
     }
   }
   const size_t smem = (size_t)(kTopkSmemCap + kRadixBins + 64) * 4;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr_set = true;
-  }
+  cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   topk_rows_smem_kernel<<<b->total_q, kTopkThreadsA, smem, stream>>>(scores, ld, bv, k, idx, lw, has_long ? 1 : 0);
   DSA_LAUNCH_CHECK("topk_rows_smem_kernel");
   if (has_long) {
@@ -373,6 +371,61 @@ dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, 
     DSA_LAUNCH_CHECK("topk_long_write_kernel");
   }
   return DSA_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free variant.  Its scratch (long-row histograms, row states, segment counts and the status
+// header) is one file-scope device array, sized for at most kNoAllocMaxRows query rows and rows of at
+// most kNoAllocMaxSeqLen candidates.  Every device that loads the library holds it until the process
+// exits.  Host code must not hand the array's host-side name to a kernel: it is only a stand-in there,
+// so the device address is looked up with cudaGetSymbolAddress once per device and cached.
+// ------------------------------------------------------------------------------------------------
+constexpr int kNoAllocMaxRows = 256;
+constexpr int kNoAllocMaxSeqLen = 1 << 20;
+constexpr size_t al256c(size_t x) { return (x + 255) / 256 * 256; }
+constexpr size_t kNoAllocBytes =
+    kWsHeader + 64 + al256c((size_t)kNoAllocMaxRows * 4) + al256c((size_t)kNoAllocMaxRows * sizeof(TopkRowState)) +
+    al256c((size_t)kNoAllocMaxRows * kRadixBins * 4) +
+    al256c((size_t)kNoAllocMaxRows * ((kNoAllocMaxSeqLen + kTopkSeg - 1) / kTopkSeg) * sizeof(uint2));
+
+static __device__ __align__(256) unsigned char g_topk_scratch[kNoAllocBytes];
+
+static void *g_topk_scratch_addr[64];
+static std::mutex g_topk_scratch_mu;
+
+// device address of the scratch array on the current device (looked up on first use per device)
+static dsa_status_t topk_scratch_address(void **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    set_error("dsa_topk_noalloc: no current CUDA device");
+    return DSA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> g(g_topk_scratch_mu);
+  if (g_topk_scratch_addr[dev] == nullptr) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_topk_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      set_error("dsa_topk_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+      return DSA_ERR_CUDA;
+    }
+    g_topk_scratch_addr[dev] = p;
+  }
+  *out = g_topk_scratch_addr[dev];
+  return DSA_OK;
+}
+
+dsa_status_t topk_noalloc_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx,
+                                 cudaStream_t stream, int num_sms) {
+  if (b->total_q > kNoAllocMaxRows || b->max_seq_len > kNoAllocMaxSeqLen ||
+      topk_workspace_bytes(b->total_q, b->max_seq_len) > kNoAllocBytes) {
+    set_error("dsa_topk_noalloc: batch exceeds the built-in scratch (at most %d rows of at most %d candidates; "
+              "got %d rows, max_seq_len %d)", kNoAllocMaxRows, kNoAllocMaxSeqLen, b->total_q, b->max_seq_len);
+    return DSA_ERR_UNSUPPORTED;
+  }
+  void *scratch = nullptr;
+  dsa_status_t st = topk_scratch_address(&scratch);
+  if (st != DSA_OK) return st;
+  return topk_launch(scores, ld, b, k, idx, scratch, stream, num_sms);
 }
 
 }  // namespace dsa

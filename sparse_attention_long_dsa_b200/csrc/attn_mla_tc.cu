@@ -9,21 +9,23 @@
 // tokens in parallel units, decode prefetches the next KV block with asynchronous copies while the
 // current one is computed, partial results are merged by a cross-block reduction.)
 //
-// Work split of a CTA pair (rank r = 0, 1), chunks of 128 selected tokens:
-//   * QK^T  : M = 128 heads (rank r holds heads 64r..64r+63 of q in smem), N = 128 tokens (rank r
-//             gathers tokens 64r..64r+63 of the chunk, all 576 dims), K = 576.  S lands in TMEM of
-//             both CTAs: each CTA gets its 64 heads x 128 tokens.
-//   * softmax: each CTA's 4 softmax warps own one (head, 64-token half) per thread: running max shared
-//             with the partner thread through smem, exp2, P (bf16) into smem.  O is rescaled in TMEM
-//             only when the running max grows by more than 2^8 (exact: the final division uses the
-//             same reference max).
-//   * P V   : M = 128 heads, N = 512 values as two N = 256 MMAs (rank r supplies values 256r..256r+255
-//             of every token), K = 128 tokens.  O (64 heads x 512 fp32) stays in TMEM, 256 columns.
-// Every MMA is issued by one thread of rank 0 for the pair (cta_group::2).  Tokens are gathered with
-// 16-byte cp.async through the block table straight into the 128-byte-swizzled operand layout, into a
-// ring of 16 KB slots in exactly the order the MMAs consume them; rank 1's slot completions are
-// relayed to rank 0's barriers by one thread.  Token positions that are -1 (or out of range) are
-// zero-filled and masked.
+// Work split of a CTA pair (rank r = 0, 1) over chunks of 96 selected tokens:
+//   * each CTA gathers ITS 48 tokens of the chunk (tokens 48r..48r+47), all 576 dims, into a chunk buffer
+//     [9 dim blocks][48 tokens][128 B] (128-byte swizzle), by TMA gather4 through the block table;
+//   * QK^T  : M = 128 heads (rank r holds heads 64r..64r+63 of q), N = 96 tokens (48 from each CTA),
+//             K = 576; each CTA gets S for its 64 heads x all 96 tokens in TMEM;
+//   * swap  : the values each CTA needs for P V are 256 of the 512 value dims of all 96 tokens; its own
+//             tokens already hold them, the peer's tokens are fetched from the peer's chunk buffer over
+//             distributed shared memory (dim blocks 0-3 of rank 1's tokens <-> dim blocks 4-7 of rank 0's
+//             tokens, in place), so every token row crosses the copy engine once per pair;
+//   * softmax: 4 warps per CTA, one (head, 48-token half) per thread, running max shared with the partner
+//             thread, exp2, P (bf16) into smem; O is rescaled in TMEM only when the running max grows by
+//             more than 2^8 (exact: the final division uses the same reference max);
+//   * P V   : M = 128 heads, N = 512 values as two N = 256 MMAs (rank r supplies values 256r..256r+255),
+//             K = 96 tokens; O (64 heads x 512 fp32 per CTA) stays in TMEM, 256 columns.
+// Every MMA is issued by one thread of rank 0 for the pair (cta_group::2).  Chunk buffers are double
+// buffered; rank 1's buffer completions are relayed to rank 0's barriers by one thread.  Token positions
+// that are -1 (or out of range) are zero-filled by the copy engine and masked.
 //
 // Units: prefill = one row (all its chunks); decode = (row, split) pairs whose partial (o, lse) are
 // merged by attn_combine_kernel.  Rows are taken longest-first (reverse order) round-robin over pairs.
@@ -36,30 +38,32 @@
 namespace dsa {
 
 constexpr int kAttH = 128, kAttD = 576, kAttDv = 512;
-constexpr int kAttChunk = 128;
-constexpr int kAttSlots = 8;
+constexpr int kAttChunk = 96;                    // tokens per chunk (48 per CTA)
+constexpr int kAttHalf = kAttChunk / 2;
 constexpr int kAttThreads = 320;                 // warps 0-3 softmax, 4-7 gather, 8 MMA, 9 relay
-constexpr uint32_t kAttSlotBytes = 16384;
+constexpr uint32_t kAttBlkBytes = kAttHalf * 128;                // one dim block of a CTA's 48 tokens: 6 KB
+constexpr uint32_t kAttBufBytes = 9 * kAttBlkBytes;              // 54 KB
 constexpr uint32_t kAttQBytes = 9 * 8192;
-constexpr uint32_t kAttPBytes = 16384;
-constexpr uint32_t kTmemO = 0, kTmemS = 256;     // O: 256 columns; S: two buffers of 64 columns
+constexpr uint32_t kAttPBytes = 16384;           // [2 token blocks of 64][64 heads][128 B]
+constexpr uint32_t kTmemO = 0, kTmemS = 256;     // O: 256 columns; S: two buffers of 48 columns
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kPrefetchAhead = 2;              // chunks of L2 prefetch ahead of the gather
+constexpr int kPrefetchAhead = 2;                // chunks of L2 prefetch ahead of the gather
 
 struct AttSmem {
-  uint64_t slot_full[kAttSlots];    // local: TMA transaction bytes (one expect_tx per fill)
-  uint64_t pair_full[kAttSlots];    // rank 0: 2 relays
-  uint64_t slot_empty[kAttSlots];   // MMA commit to both CTAs
+  uint64_t buf_full[2];             // local: TMA bytes of this CTA's half of a chunk (4 producer warps)
+  uint64_t pair_full[2];            // rank 0: 2 relays
+  uint64_t buf_empty[2];            // MMA commit to both CTAs after P V of the chunk
   uint64_t q_full, pair_q_full, q_empty;
   uint64_t s_full[2];               // MMA commit to both CTAs
-  uint64_t p_full;                  // rank 0: 8 softmax warps (4 per CTA)
+  uint64_t xchg[2];                 // the peer's 4 softmax warps finished reading this CTA's buffer
+  uint64_t p_full;                  // rank 0: 8 softmax warps (swap written + P written)
   uint64_t pv_done;                 // MMA commit to both CTAs, once per chunk
   uint64_t o_empty;                 // rank 0: 8 softmax warps after the epilogue read O
   uint64_t drain;
   uint64_t mask_full[4], mask_empty[4];   // validity masks of upcoming chunks (gather -> softmax)
   uint32_t tmem_base;
   int abort;
-  uint64_t mask[4][2];
+  uint32_t mask[4][4];              // 3 ballot words per chunk (tokens 0-31, 32-63, 64-95)
   float xm[2][128];
   float xl[2][128];
   int32_t phys[2][kAttChunk];
@@ -154,9 +158,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     attn_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv, const AttArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *sQ = smem;
-  uint8_t *sRing = sQ + kAttQBytes;
-  uint8_t *sP = sRing + kAttSlots * kAttSlotBytes;
+  uint8_t *sQ = smem;                                  // [9 dim blocks][64 heads][128 B]
+  uint8_t *sBuf = sQ + kAttQBytes;                     // 2 x [9 dim blocks][48 tokens][128 B]
+  uint8_t *sP = sBuf + 2 * kAttBufBytes;               // [2 token blocks][64 heads][128 B]
   AttSmem *S = (AttSmem *)(sP + kAttPBytes);
 
   const uint32_t rank = tc::cluster_ctarank();
@@ -165,16 +169,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
   const int U = num_units(a);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kAttSlots; ++i) {
-      tc::mbar_init(tc::smem_u32(&S->slot_full[i]), 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(tc::smem_u32(&S->buf_full[i]), 4);
       tc::mbar_init(tc::smem_u32(&S->pair_full[i]), 2);
-      tc::mbar_init(tc::smem_u32(&S->slot_empty[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->buf_empty[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->s_full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->xchg[i]), 4);
     }
     tc::mbar_init(tc::smem_u32(&S->q_full), 1);
     tc::mbar_init(tc::smem_u32(&S->pair_q_full), 2);
     tc::mbar_init(tc::smem_u32(&S->q_empty), 1);
-    tc::mbar_init(tc::smem_u32(&S->s_full[0]), 1);
-    tc::mbar_init(tc::smem_u32(&S->s_full[1]), 1);
     tc::mbar_init(tc::smem_u32(&S->p_full), 8);
     tc::mbar_init(tc::smem_u32(&S->pv_done), 1);
     tc::mbar_init(tc::smem_u32(&S->o_empty), 8);
@@ -185,6 +189,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     }
     S->abort = 0;
     tc::fence_barrier_init();
+    tc::prefetch_tmap(&tm_q);
+    tc::prefetch_tmap(&tm_kv);
   }
   if (warp == 8) {
     tc::tmem_alloc2(tc::smem_u32(&S->tmem_base), 512);
@@ -200,20 +206,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
 
   if (warp >= 4 && warp < 8) {
     // ====================================================================== gather (128 threads)
-    // q arrives by one tiled TMA per dim block; selected latent rows by TMA gather4 (4 rows x 128 bytes per
-    // instruction, 128-byte swizzle applied by the copy engine).  Each 16 KB ring slot is filled by one of
-    // the four gather warps (one gather4 per lane), round-robin over slots.  Loops holding the named
-    // barrier never break: after a timeout every wait returns at once and the copies are skipped, so all
-    // 128 threads still meet at the same barriers and reach the teardown.
+    // q by one tiled TMA per dim block; this CTA's 48 tokens of every chunk by TMA gather4 (4 rows x 128
+    // bytes per instruction, 128-byte swizzle applied by the copy engine), warp w taking dim blocks w, w+4
+    // (and 8 for warp 0).  Loops holding the named barrier never break: after a timeout every wait returns
+    // at once and the copies are skipped, so all 128 threads still meet at the barriers and the teardown.
     const int t = threadIdx.x - 128, pw = t >> 5;
     const int oob_row = a.bv.num_blocks * 64;           // outside the map: the copy engine fills zeros
-    int slot = 0, fill = 0;
-    uint32_t sphase = 0, v = 0, gch = 0;
+    uint32_t v = 0, g = 0;
     // L2 prefetch cursor, kPrefetchAhead chunks ahead of the chunk being gathered: each CTA prefetches the
-    // full latent rows of its own 64 tokens of the chunk (and the next unit's q when the cursor enters it)
+    // full latent rows of its own 48 tokens (and the next unit's q when the cursor enters it)
     int pf_u = pair, pf_c = 0, pf_row = -1, pf_cb = 0, pf_nch = 0, pf_seq = 0;
     const int32_t *pf_btr = nullptr;
-    auto pf_enter = [&](int uu) -> bool {      // position the cursor at chunk 0 of the first non-empty unit >= uu
+    auto pf_enter = [&](int uu) {
       for (; uu < U; uu += npairs) {
         int r2, cb2, ce2;
         unit_of(a, uu, &r2, &cb2, &ce2);
@@ -223,55 +227,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
           pf_u = uu; pf_c = 0; pf_row = r2; pf_cb = cb2; pf_nch = ce2 - cb2;
           pf_seq = __ldg(a.bv.seq_lens + b2);
           pf_btr = a.bv.block_table + (int64_t)b2 * a.bv.max_blocks_per_seq;
-          if (t < 64) {
-            const __nv_bfloat16 *qr = a.q + ((int64_t)r2 * kAttH + 64 * rank + t) * kAttD;
-            tc::prefetch_l2(qr, kAttD * 2);
-          }
-          return true;
+          if (t < 64) tc::prefetch_l2(a.q + ((int64_t)r2 * kAttH + 64 * rank + t) * kAttD, kAttD * 2);
+          return;
         }
       }
       pf_u = U;
-      return false;
     };
-    auto pf_step = [&]() {                     // prefetch the cursor's chunk, then advance it
+    auto pf_step = [&]() {
       if (pf_u >= U) return;
-      if (t < 64) {
-        const int j = (pf_cb + pf_c) * kAttChunk + 64 * (int)rank + t;
+      if (t < kAttHalf) {
+        const int j = (pf_cb + pf_c) * kAttChunk + kAttHalf * (int)rank + t;
         if (j < a.k) {
           const int s = __ldg(a.idx + (int64_t)pf_row * a.k + j);
           if (s >= 0 && s < pf_seq) {
             const int blk = __ldg(pf_btr + (s >> 6));
-            if ((unsigned)blk < (unsigned)a.bv.num_blocks) tc::prefetch_l2(a.kv + ((int64_t)blk * 64 + (s & 63)) * kAttD, kAttD * 2);
+            if ((unsigned)blk < (unsigned)a.bv.num_blocks)
+              tc::prefetch_l2(a.kv + ((int64_t)blk * 64 + (s & 63)) * kAttD, kAttD * 2);
           }
         }
       }
       if (++pf_c == pf_nch) pf_enter(pf_u + npairs);
-    };
-    // fill one ring slot with 32 gather4 copies: lane -> (dim block d(lane), tokens 4*(lane%16) + [0,4) of
-    // the 64 tokens starting at chunk token key0); blocks with d < 0 are skipped
-    auto fill_slot = [&](int chunk_parity, int key0, int d0, int d1) {
-      const bool mine = (fill & 3) == pw;
-      if (mine) {
-        const int nblk = d1 >= 0 ? 2 : 1;
-        bool ok = true;
-        if (lane == 0) {
-          ok = tc::mbar_wait_cl(tc::smem_u32(&S->slot_empty[slot]), sphase ^ 1u, abort, status);
-          if (ok) tc::mbar_expect_tx(tc::smem_u32(&S->slot_full[slot]), (uint32_t)nblk * 64 * 128);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        const int blk = lane >> 4, g4 = lane & 15;
-        if (ok && blk < nblk) {
-          const int d = blk ? d1 : d0;
-          const int32_t *ph = S->phys[chunk_parity] + key0 + 4 * g4;
-          int r[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) r[e] = ph[e] >= 0 ? ph[e] : oob_row;
-          tc::tma_gather4(tc::smem_u32(sRing + slot * kAttSlotBytes + blk * 8192 + 4 * g4 * 128), &tm_kv, d * 64, r[0],
-                          r[1], r[2], r[3], tc::smem_u32(&S->slot_full[slot]));
-        }
-      }
-      ++fill;
-      if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
     };
     pf_enter(pair);
     for (int d = 0; d < kPrefetchAhead; ++d) pf_step();
@@ -284,7 +259,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
       pos_of_row(a.bv, row, &b);
       const int seq_len = __ldg(a.bv.seq_lens + b);
       const int32_t *btr = a.bv.block_table + (int64_t)b * a.bv.max_blocks_per_seq;
-      // ---- q: this CTA's 64 heads, [9 dim blocks][64 heads][128 B], 128-byte swizzle
       if (t == 0) {
         const bool ok = v == 0 || tc::mbar_wait_cl(tc::smem_u32(&S->q_empty), (v - 1) & 1u, abort, status);
         if (ok) {
@@ -294,39 +268,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
             tc::tma_load_2d(tc::smem_u32(sQ + d * 8192), &tm_q, d * 64, row * kAttH + 64 * (int)rank, bar);
         }
       }
-      for (int i = 0; i <= nch; ++i) {
-        if (i < nch) {
-          // token positions of chunk i -> physical rows (-1: masked); the validity mask goes to the softmax
-          pf_step();
-          const uint32_t mslot = gch & 3u;
-          const bool m_ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->mask_empty[mslot]),
-                                                                  ((gch >> 2) & 1u) ^ 1u, abort, status));
-          tc::named_bar_sync(1, 128);
-          {
-            const int j = (cb + i) * kAttChunk + t;
-            int32_t pr = -1;
-            if (j < a.k) {
-              const int s = __ldg(a.idx + (int64_t)row * a.k + j);
-              if (s >= 0 && s < seq_len) {
-                const int blk = __ldg(btr + (s >> 6));
-                if ((unsigned)blk < (unsigned)a.bv.num_blocks) pr = blk * 64 + (s & 63);
-                else set_status(status, kStatusBadIndex);
-              }
+      for (int i = 0; i < nch; ++i, ++g) {
+        const uint32_t bi = g & 1u, use = g >> 1;
+        pf_step();
+        // token positions of the chunk -> physical rows (-1: masked); validity words go to the softmax
+        const uint32_t mslot = g & 3u;
+        const bool m_ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->mask_empty[mslot]),
+                                                                ((g >> 2) & 1u) ^ 1u, abort, status));
+        tc::named_bar_sync(1, 128);
+        {
+          int32_t pr = -1;
+          const int j = (cb + i) * kAttChunk + t;
+          if (t < kAttChunk && j < a.k) {
+            const int s = __ldg(a.idx + (int64_t)row * a.k + j);
+            if (s >= 0 && s < seq_len) {
+              const int blk = __ldg(btr + (s >> 6));
+              if ((unsigned)blk < (unsigned)a.bv.num_blocks) pr = blk * 64 + (s & 63);
+              else set_status(status, kStatusBadIndex);
             }
-            S->phys[i & 1][t] = pr;
-            const unsigned bits = __ballot_sync(0xffffffffu, pr >= 0);
-            if (lane == 0 && m_ok) reinterpret_cast<uint32_t *>(S->mask[mslot])[t >> 5] = bits;
           }
-          tc::named_bar_sync(1, 128);
-          if (t == 0) tc::mbar_arrive(tc::smem_u32(&S->mask_full[mslot]));
-          ++gch;
-          // QK slots: this CTA's 64 tokens, dim blocks (2s, 2s+1)
-          for (int sl = 0; sl < 5; ++sl) fill_slot(i & 1, 64 * (int)rank, 2 * sl, 2 * sl + 1 < 9 ? 2 * sl + 1 : -1);
+          if (t < kAttChunk) S->phys[bi][t] = pr;
+          const unsigned bits = __ballot_sync(0xffffffffu, pr >= 0);
+          if (lane == 0 && m_ok && pw < 3) S->mask[mslot][pw] = bits;
         }
-        if (i > 0) {
-          // PV slots of chunk i-1: value blocks (4r + 2p, 4r + 2p + 1) of token half kh
-          for (int p = 0; p < 2; ++p)
-            for (int kh = 0; kh < 2; ++kh) fill_slot((i - 1) & 1, 64 * kh, 4 * (int)rank + 2 * p, 4 * (int)rank + 2 * p + 1);
+        tc::named_bar_sync(1, 128);
+        if (t == 0) tc::mbar_arrive(tc::smem_u32(&S->mask_full[mslot]));
+        // this warp's dim blocks of this CTA's 48 tokens, into chunk buffer bi
+        const int nblk = pw == 0 ? 3 : 2;
+        bool ok = true;
+        if (lane == 0) {
+          ok = tc::mbar_wait_cl(tc::smem_u32(&S->buf_empty[bi]), (use & 1u) ^ 1u, abort, status);
+          if (ok) tc::mbar_expect_tx(tc::smem_u32(&S->buf_full[bi]), (uint32_t)nblk * kAttBlkBytes);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok && lane < kAttHalf / 4) {
+          const int32_t *ph = S->phys[bi] + kAttHalf * (int)rank + 4 * lane;
+          int r4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) r4[e] = ph[e] >= 0 ? ph[e] : oob_row;
+          for (int m = 0; m < nblk; ++m) {
+            const int d = pw + 4 * m;
+            tc::tma_gather4(tc::smem_u32(sBuf + bi * kAttBufBytes + d * kAttBlkBytes + 4 * lane * 128), &tm_kv, d * 64,
+                            r4[0], r4[1], r4[2], r4[3], tc::smem_u32(&S->buf_full[bi]));
+          }
         }
       }
       ++v;
@@ -336,8 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     if (lane == 0) {
       const uint32_t peer_pair_full = tc::map_to_rank(tc::smem_u32(&S->pair_full[0]), 0);
       const uint32_t peer_pair_q = tc::map_to_rank(tc::smem_u32(&S->pair_q_full), 0);
-      int slot = 0;
-      uint32_t sphase = 0, v = 0;
+      uint32_t v = 0, g = 0;
       bool ok = true;
       for (int u = pair; u < U && ok; u += npairs) {
         int row, cb, ce;
@@ -347,12 +330,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         if (!tc::mbar_wait(tc::smem_u32(&S->q_full), v & 1u, abort, status)) break;
         tc::fence_proxy_async();
         tc::mbar_arrive_cluster(peer_pair_q);
-        const int fills = 9 * nch;
-        for (int f = 0; f < fills; ++f) {
-          if (!tc::mbar_wait(tc::smem_u32(&S->slot_full[slot]), sphase, abort, status)) { ok = false; break; }
+        for (int i = 0; i < nch; ++i, ++g) {
+          if (!tc::mbar_wait(tc::smem_u32(&S->buf_full[g & 1u]), (g >> 1) & 1u, abort, status)) { ok = false; break; }
           tc::fence_proxy_async();
-          tc::mbar_arrive_cluster(peer_pair_full + slot * 8);
-          if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
+          tc::mbar_arrive_cluster(peer_pair_full + (g & 1u) * 8);
         }
         ++v;
       }
@@ -360,31 +341,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
   } else if (warp == 8) {
     // ====================================================================== MMA issuer (rank 0, lane 0)
     if (rank == 0 && lane == 0) {
-      const uint32_t idesc_qk = tc::make_idesc(1, 1, 128, 128, false, false);
+      const uint32_t idesc_qk = tc::make_idesc(1, 1, 128, kAttChunk, false, false);
       const uint32_t idesc_pv = tc::make_idesc(1, 1, 128, 256, false, true);
       const uint16_t both = 3;
       const uint32_t qbase = tc::smem_u32(sQ), pbase = tc::smem_u32(sP);
-      int slot = 0;
-      uint32_t sphase = 0, v = 0, g = 0;       // g: chunks issued so far (all units)
+      uint32_t v = 0, g = 0;
       bool ok = true;
-      auto pv = [&](int c, uint32_t gc) -> bool {
+      auto pv = [&](uint32_t gc, bool first) -> bool {
         if (!tc::mbar_wait_cl(tc::smem_u32(&S->p_full), gc & 1u, abort, status)) return false;
-        if (c == 0 && v > 0 && !tc::mbar_wait_cl(tc::smem_u32(&S->o_empty), (v - 1) & 1u, abort, status)) return false;
+        if (first && v > 0 && !tc::mbar_wait_cl(tc::smem_u32(&S->o_empty), (v - 1) & 1u, abort, status)) return false;
         tc::fence_after_sync();
+        const uint32_t base = tc::smem_u32(sBuf + (gc & 1u) * kAttBufBytes);
         for (int p = 0; p < 2; ++p)
-          for (int kh = 0; kh < 2; ++kh) {
-            if (!tc::mbar_wait_cl(tc::smem_u32(&S->pair_full[slot]), sphase, abort, status)) return false;
-            tc::fence_after_sync();
-            const uint32_t base = tc::smem_u32(sRing + slot * kAttSlotBytes);
+          for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = tc::desc_sw128(pbase + kh * 8192 + kk * 32, 1024);
-              const uint64_t bd = tc::desc_sw128_lbo(base + kk * 2048, 8192, 1024);
-              tc::mma_bf16_pair(tmem + kTmemO + 128 * p, ad, bd, idesc_pv, (c == 0 && kh == 0 && kk == 0) ? 0u : 1u);
+            for (int ks = 0; ks < kAttHalf / 16; ++ks) {
+              const int kg = (kAttHalf / 16) * kh + ks;          // 16-token step within the chunk
+              const uint64_t ad = tc::desc_sw128(pbase + (kg >> 2) * 8192 + (kg & 3) * 32, 1024);
+              const uint64_t bd =
+                  tc::desc_sw128_lbo(base + (4 * kh + 2 * p) * kAttBlkBytes + ks * 2048, kAttBlkBytes, 1024);
+              tc::mma_bf16_pair(tmem + kTmemO + 128 * p, ad, bd, idesc_pv, (first && kg == 0) ? 0u : 1u);
             }
-            tc::mma_commit_pair(tc::smem_u32(&S->slot_empty[slot]), both);
-            if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
-          }
+        tc::mma_commit_pair(tc::smem_u32(&S->buf_empty[gc & 1u]), both);
         tc::mma_commit_pair(tc::smem_u32(&S->pv_done), both);
         return true;
       };
@@ -396,32 +374,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         if (!tc::mbar_wait_cl(tc::smem_u32(&S->pair_q_full), v & 1u, abort, status)) break;
         tc::fence_after_sync();
         const uint32_t g0 = g;
-        for (int i = 0; i < nch && ok; ++i) {
-          const uint32_t sb = tmem + kTmemS + 64 * (g & 1u);
-          for (int sl = 0; sl < 5; ++sl) {
-            if (!tc::mbar_wait_cl(tc::smem_u32(&S->pair_full[slot]), sphase, abort, status)) { ok = false; break; }
-            tc::fence_after_sync();
-            const uint32_t base = tc::smem_u32(sRing + slot * kAttSlotBytes);
-            for (int blk = 0; blk < 2; ++blk) {
-              const int d = 2 * sl + blk;
-              if (d >= 9) break;
+        for (int i = 0; i < nch; ++i) {
+          if (!tc::mbar_wait_cl(tc::smem_u32(&S->pair_full[g & 1u]), (g >> 1) & 1u, abort, status)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t base = tc::smem_u32(sBuf + (g & 1u) * kAttBufBytes);
+          const uint32_t sb = tmem + kTmemS + kAttHalf * (g & 1u);
+          for (int d = 0; d < 9; ++d) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = tc::desc_sw128(qbase + d * 8192 + kk * 32, 1024);
-                const uint64_t bd = tc::desc_sw128(base + blk * 8192 + kk * 32, 1024);
-                tc::mma_bf16_pair(sb, ad, bd, idesc_qk, (d == 0 && kk == 0) ? 0u : 1u);
-              }
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = tc::desc_sw128(qbase + d * 8192 + kk * 32, 1024);
+              const uint64_t bd = tc::desc_sw128(base + d * kAttBlkBytes + kk * 32, 1024);
+              tc::mma_bf16_pair(sb, ad, bd, idesc_qk, (d == 0 && kk == 0) ? 0u : 1u);
             }
-            tc::mma_commit_pair(tc::smem_u32(&S->slot_empty[slot]), both);
-            if (++slot == kAttSlots) { slot = 0; sphase ^= 1u; }
           }
-          if (!ok) break;
           tc::mma_commit_pair(tc::smem_u32(&S->s_full[g & 1u]), both);
           if (i == nch - 1) tc::mma_commit_pair(tc::smem_u32(&S->q_empty), both);
           ++g;
-          if (i > 0 && !pv(i - 1, g0 + i - 1)) { ok = false; break; }
+          if (i > 0 && !pv(g0 + i - 1, i - 1 == 0)) { ok = false; break; }
         }
-        if (ok && !pv(nch - 1, g0 + nch - 1)) ok = false;
+        if (ok && !pv(g0 + nch - 1, nch == 1)) ok = false;
         ++v;
       }
       tc::mma_commit_pair_local(tc::smem_u32(&S->drain));
@@ -429,7 +400,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
       tc::mbar_wait(tc::smem_u32(&S->drain), 0, &no_abort, status);
     }
   } else {
-    // ====================================================================== softmax + epilogue (128 threads)
+    // ====================================================================== swap + softmax + epilogue
     // Like the gather role, these loops never break (they hold named barrier 2): after a timeout the
     // waits return at once and the remaining chunks run through without touching TMEM or memory.
     const int L = threadIdx.x;                 // TMEM lane
@@ -437,6 +408,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t p_full_r0 = tc::map_to_rank(tc::smem_u32(&S->p_full), 0);
     const uint32_t o_empty_r0 = tc::map_to_rank(tc::smem_u32(&S->o_empty), 0);
+    const uint32_t peer_buf = tc::map_to_rank(tc::smem_u32(sBuf), rank ^ 1u);
+    const uint32_t peer_xchg = tc::map_to_rank(tc::smem_u32(&S->xchg[0]), rank ^ 1u);
+    // the swap moves the value dims this CTA needs from the peer's tokens: rank 0 takes dim blocks 0-3 of
+    // rank 1's tokens into its blocks 4-7; rank 1 takes dim blocks 4-7 of rank 0's tokens into its blocks 0-3
+    const uint32_t src_off = (rank == 0 ? 0u : 4u) * kAttBlkBytes, dst_off = (rank == 0 ? 4u : 0u) * kAttBlkBytes;
+    constexpr int kSwapVec = 4 * kAttBlkBytes / 16 / 128;       // 16-byte vectors per thread
     uint32_t g = 0, v = 0;
     for (int u = pair; u < U; u += npairs) {
       int row, cb, ce;
@@ -456,37 +433,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         }
         continue;
       }
-      int b;
-      pos_of_row(a.bv, row, &b);
-      const int seq_len = __ldg(a.bv.seq_lens + b);
       float m_run = -INFINITY, l_run = 0.f, l_exact = 0.f;
       for (int i = 0; i < nch; ++i, ++g) {
-        // validity of this thread's 64 tokens, published by the gather warps
+        const uint32_t bi = g & 1u;
+        // validity of this thread's 48 tokens, published by the gather warps
         const uint32_t mslot = g & 3u;
         const bool m_ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->mask_full[mslot]),
                                                                 (g >> 2) & 1u, abort, status));
-        uint64_t valid = m_ok ? S->mask[mslot][half] : 0ull;
+        uint64_t valid = 0;
+        if (m_ok) {
+          const uint64_t w0 = S->mask[mslot][0], w1 = S->mask[mslot][1], w2 = S->mask[mslot][2];
+          valid = half == 0 ? (w0 | (w1 << 32)) : ((w1 >> 16) | (w2 << 16));
+          valid &= (1ull << kAttHalf) - 1ull;
+        }
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->mask_empty[mslot]));
-        const bool have_s = tc::mbar_wait_cl(tc::smem_u32(&S->s_full[g & 1u]), (g >> 1) & 1u, abort, status);
+        const bool have_s =
+            __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->s_full[bi]), (g >> 1) & 1u, abort, status));
         tc::fence_after_sync();
-        float sv[64];
+        // ---- swap over distributed shared memory: read the peer's values, hand-shake, write them here
         {
-          float t0[32], t1[32];
-          const uint32_t sa = tmem + lane_base + kTmemS + 64 * (g & 1u);
+          uint4 sw[kSwapVec];
+#pragma unroll
+          for (int m = 0; m < kSwapVec; ++m)
+            sw[m] = have_s ? tc::ld_dsmem16(peer_buf + bi * kAttBufBytes + src_off + (L + 128 * m) * 16)
+                           : make_uint4(0, 0, 0, 0);
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive_cluster(peer_xchg + bi * 8);
+          const bool got = __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->xchg[bi]), (g >> 1) & 1u, abort, status));
+          if (have_s && got) {
+#pragma unroll
+            for (int m = 0; m < kSwapVec; ++m)
+              *reinterpret_cast<uint4 *>(sBuf + bi * kAttBufBytes + dst_off + (L + 128 * m) * 16) = sw[m];
+          }
+        }
+        // ---- S for this thread's head and 48 tokens
+        float sv[kAttHalf];
+        {
+          float t0[32], t1[16];
+          const uint32_t sa = tmem + lane_base + kTmemS + kAttHalf * bi;
           tc::tmem_ld32(sa, t0);
-          tc::tmem_ld32(sa + 32, t1);
+          tc::tmem_ld16(sa + 32, t1);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            sv[c] = t0[c];
-            sv[32 + c] = t1[c];
-          }
+          for (int c = 0; c < 32; ++c) sv[c] = t0[c];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) sv[32 + c] = t1[c];
         }
         if (!have_s) valid = 0;
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < kAttHalf; ++c) {
           sv[c] = ((valid >> c) & 1ull) ? sv[c] * a.scale_log2 : -INFINITY;
           mx = fmaxf(mx, sv[c]);
         }
@@ -494,7 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         S->xm[g & 1u][L] = mloc;
         tc::named_bar_sync(2, 128);
         const float m_new = fmaxf(mloc, S->xm[g & 1u][L ^ 64]);
-        // PV of the previous chunk must be finished before O is touched or P is overwritten
+        // P V of the previous chunk must be finished before O is touched or P is overwritten
         bool pv_ok = true;
         if (i > 0) {
           pv_ok = tc::mbar_wait_cl(tc::smem_u32(&S->pv_done), (g - 1) & 1u, abort, status);
@@ -527,14 +524,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
             }
           }
         }
-        // P = exp2(z - m) in bf16, into the 128-byte-swizzled A operand (row h, tokens of this half).
-        // l_run sums the rounded P (what the MMA multiplies) and normalises O; l_exact sums the
-        // unrounded values and gives lse.
+        // P = exp2(z - m) in bf16 into the 128-byte-swizzled A operand: row h, tokens 48*half + [0, 48).
+        // l_run sums the rounded P (what the MMA multiplies) and normalises O; l_exact gives lse.
         if (pv_ok) {
-          uint8_t *prow = sP + half * 8192 + h * 128;
           float lsum = 0.f, lex = 0.f;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < kAttHalf / 8; ++c) {
             uint32_t w4[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -547,7 +542,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
               lex += p0 + p1;
               w4[e] = *reinterpret_cast<const uint32_t *>(&pb);
             }
-            *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            const int kc = (kAttHalf / 8) * half + c;              // 8-token chunk within the 96 tokens
+            *reinterpret_cast<uint4 *>(sP + (kc >> 3) * 8192 + h * 128 + (((kc & 7) ^ (h & 7)) << 4)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
           l_run += lsum;
           l_exact += lex;
@@ -611,7 +608,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     }
   }
 
-  // ---- teardown: every role is done; MMAs drained; peers done with our barriers and TMEM
+  // ---- teardown: every role is done; MMAs drained; peers done with our barriers, buffers and TMEM
   tc::fence_before_sync();
   __syncthreads();
   tc::cluster_sync();
@@ -696,7 +693,7 @@ static bool make_bf16_rows_map(CUtensorMap *m, const void *base, uint64_t rows, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t attn_smem_bytes() { return 1024 + kAttQBytes + kAttSlots * kAttSlotBytes + kAttPBytes + sizeof(AttSmem); }
+static size_t attn_smem_bytes() { return 1024 + kAttQBytes + 2 * kAttBufBytes + kAttPBytes + sizeof(AttSmem); }
 
 dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, int k, float softmax_scale,
                              const dsa_batch_t *b, void *out, float *lse, void *ws, bool decode, cudaStream_t stream,

@@ -9,23 +9,27 @@
 // tokens in parallel units, decode prefetches the next KV block with asynchronous copies while the
 // current one is computed, partial results are merged by a cross-block reduction.)
 //
-// Work split of a CTA pair (rank r = 0, 1) over chunks of 96 selected tokens:
-//   * each CTA gathers ITS 48 tokens of the chunk (tokens 48r..48r+47), all 576 dims, into a chunk buffer
-//     [9 dim blocks][48 tokens][128 B] (128-byte swizzle), by TMA gather4 through the block table;
-//   * QK^T  : M = 128 heads (rank r holds heads 64r..64r+63 of q), N = 96 tokens (48 from each CTA),
-//             K = 576; each CTA gets S for its 64 heads x all 96 tokens in TMEM;
-//   * swap  : the values each CTA needs for P V are 256 of the 512 value dims of all 96 tokens; its own
-//             tokens already hold them, the peer's tokens are fetched from the peer's chunk buffer over
-//             distributed shared memory (dim blocks 0-3 of rank 1's tokens <-> dim blocks 4-7 of rank 0's
-//             tokens, in place), so every token row crosses the copy engine once per pair;
-//   * softmax: 4 warps per CTA, one (head, 48-token half) per thread, running max shared with the partner
-//             thread, exp2, P (bf16) into smem; O is rescaled in TMEM only when the running max grows by
-//             more than 2^8 (exact: the final division uses the same reference max);
-//   * P V   : M = 128 heads, N = 512 values as two N = 256 MMAs (rank r supplies values 256r..256r+255),
-//             K = 96 tokens; O (64 heads x 512 fp32 per CTA) stays in TMEM, 256 columns.
-// Every MMA is issued by one thread of rank 0 for the pair (cta_group::2).  Chunk buffers are double
-// buffered; rank 1's buffer completions are relayed to rank 0's barriers by one thread.  Token positions
-// that are -1 (or out of range) are zero-filled by the copy engine and masked.
+// Work split of a CTA pair (rank r = 0, 1) over chunks of 64 selected tokens:
+//   * resolve: one warp turns token positions into physical cache rows (block table), publishes the
+//              validity mask of the chunk and prefetches the rows into L2, several chunks ahead;
+//   * gather : each CTA gathers ITS 32 tokens of the chunk (tokens 32r..32r+31), all 576 dims, into one
+//              of three chunk buffers [9 dim blocks][32 tokens][128 B] (128-byte swizzle), by TMA gather4;
+//   * QK^T   : M = 128 heads (rank r holds heads 64r..64r+63 of q), N = 64 tokens (32 from each CTA),
+//              K = 576; each CTA gets S for its 64 heads x all 64 tokens in TMEM;
+//   * cross  : the values each CTA needs for P V are 256 of the 512 value dims of all 64 tokens; its own
+//              tokens already hold them, the peer's 32 tokens' half (16 KB, which the peer's copy engine pulls
+//              through L2 at the same time) is loaded into registers by four warps a chunk ahead and stored
+//              into the dim blocks QK^T no longer needs once it has run (rank 0: blocks 4-7 <- dims 0-255 of
+//              rank 1's tokens; rank 1: blocks 0-3 <- dims 256-511 of rank 0's tokens).  The copy engine
+//              carries each row once per pair; the cross copy uses the load/store path in parallel;
+//   * softmax: 4 warps per CTA, one (head, 32-token half) per thread, running max shared with the partner
+//              thread, exp2, P (bf16) into one of two P buffers; O is rescaled in TMEM only when the
+//              running max grows by more than 2^8 (exact: the final division uses the same reference max);
+//   * P V    : M = 128 heads, N = 512 values as two N = 256 MMAs (rank r supplies values 256r..256r+255),
+//              K = 64 tokens; O (64 heads x 512 fp32 per CTA) stays in TMEM, 256 columns.
+// Every MMA is issued by one thread of rank 0 for the pair (cta_group::2).  Rank 1's buffer completions
+// are relayed to rank 0's barriers by one thread.  Token positions that are -1 (or out of range) are
+// zero-filled by the copy engine and masked.
 //
 // Units: prefill = one row (all its chunks); decode = (row, split) pairs whose partial (o, lse) are
 // merged by attn_combine_kernel.  Rows are taken longest-first (reverse order) round-robin over pairs.
@@ -38,35 +42,39 @@
 namespace dsa {
 
 constexpr int kAttH = 128, kAttD = 576, kAttDv = 512;
-constexpr int kAttChunk = 96;                    // tokens per chunk (48 per CTA)
+constexpr int kAttChunk = 64;                    // tokens per chunk (32 per CTA)
 constexpr int kAttHalf = kAttChunk / 2;
-constexpr int kAttThreads = 320;                 // warps 0-3 softmax, 4-7 gather, 8 MMA, 9 relay
-constexpr uint32_t kAttBlkBytes = kAttHalf * 128;                // one dim block of a CTA's 48 tokens: 6 KB
-constexpr uint32_t kAttBufBytes = 9 * kAttBlkBytes;              // 54 KB
+constexpr int kAttNBuf = 3;                      // chunk buffers
+constexpr int kAttRing = 4;                      // resolved chunks (physical rows + masks) in flight
+constexpr int kAttThreads = 512;                 // warpgroups: softmax, gather, cross, (MMA, relay, resolve, -)
+constexpr int kAttWarpMMA = 12, kAttWarpRelay = 13, kAttWarpResolve = 14;
+constexpr uint32_t kAttRegsSoftmax = 224, kAttRegsOther = 96;    // 128 x 224 + 384 x 96 = 65536
+constexpr uint32_t kAttBlkBytes = kAttHalf * 128;                // one dim block of a CTA's 32 tokens: 4 KB
+constexpr uint32_t kAttBufBytes = 9 * kAttBlkBytes;              // 36 KB
 constexpr uint32_t kAttQBytes = 9 * 8192;
-constexpr uint32_t kAttPBytes = 16384;           // [2 token blocks of 64][64 heads][128 B]
-constexpr uint32_t kTmemO = 0, kTmemS = 256;     // O: 256 columns; S: two buffers of 48 columns
+constexpr uint32_t kAttPBytes = 8192;            // one P buffer: [64 heads][64 tokens] bf16, 128-byte rows
+constexpr uint32_t kTmemO = 0, kTmemS = 256;     // O: 256 columns; S: two buffers of 32 columns
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kPrefetchAhead = 2;                // chunks of L2 prefetch ahead of the gather
 
 struct AttSmem {
-  uint64_t buf_full[2];             // local: TMA bytes of this CTA's half of a chunk (4 producer warps)
-  uint64_t pair_full[2];            // rank 0: 2 relays
-  uint64_t buf_empty[2];            // MMA commit to both CTAs after P V of the chunk
+  uint64_t buf_full[kAttNBuf];      // local: TMA bytes of this CTA's half of a chunk (4 gather warps)
+  uint64_t pair_full[kAttNBuf];     // rank 0: 2 relays
+  uint64_t buf_empty[kAttNBuf];     // MMA commit to both CTAs after P V of the chunk
+  uint64_t v_ready[kAttNBuf];       // rank 0: 8 cross warps (both CTAs) stored the peer's values
   uint64_t q_full, pair_q_full, q_empty;
   uint64_t s_full[2];               // MMA commit to both CTAs
-  uint64_t xchg[2];                 // the peer's 4 softmax warps finished reading this CTA's buffer
-  uint64_t p_full;                  // rank 0: 8 softmax warps (swap written + P written)
-  uint64_t pv_done;                 // MMA commit to both CTAs, once per chunk
+  uint64_t p_full[2];               // rank 0: 8 softmax warps wrote P
+  uint64_t pv_done[2];              // MMA commit to both CTAs, per P buffer
   uint64_t o_empty;                 // rank 0: 8 softmax warps after the epilogue read O
   uint64_t drain;
-  uint64_t mask_full[4], mask_empty[4];   // validity masks of upcoming chunks (gather -> softmax)
+  uint64_t phys_full[kAttRing], phys_empty[kAttRing];   // resolve -> gather
+  uint64_t mask_full[kAttRing], mask_empty[kAttRing];   // resolve -> softmax
   uint32_t tmem_base;
   int abort;
-  uint32_t mask[4][4];              // 3 ballot words per chunk (tokens 0-31, 32-63, 64-95)
+  uint32_t mask[kAttRing][2];       // ballot words of a chunk (tokens 0-31, 32-63)
   float xm[2][128];
-  float xl[2][128];
-  int32_t phys[2][kAttChunk];
+  float xl[128];
+  int32_t phys[kAttRing][kAttChunk];
 };
 
 struct AttArgs {
@@ -102,6 +110,35 @@ __device__ __forceinline__ void unit_of(const AttArgs &a, int u, int *row, int *
 }
 
 __device__ __forceinline__ int num_units(const AttArgs &a) { return a.T * a.splits; }
+
+// Walks the chunks of the units a CTA pair owns (units pair, pair + npairs, ...), skipping empty units.
+struct ChunkCursor {
+  int u, row, j, ce, seq;
+  bool first;                   // j is the first chunk of its unit
+  const int32_t *btr;           // block-table row of the unit's sequence
+
+  __device__ __forceinline__ void seek(const AttArgs &a, int uu, int npairs) {
+    const int U = num_units(a);
+    for (; uu < U; uu += npairs) {
+      int r, cb, ce2;
+      unit_of(a, uu, &r, &cb, &ce2);
+      if (ce2 > cb) {
+        int b;
+        pos_of_row(a.bv, r, &b);
+        u = uu; row = r; j = cb; ce = ce2; first = true;
+        seq = __ldg(a.bv.seq_lens + b);
+        btr = a.bv.block_table + (int64_t)b * a.bv.max_blocks_per_seq;
+        return;
+      }
+    }
+    u = U;
+  }
+  __device__ __forceinline__ void next(const AttArgs &a, int npairs) {
+    if (++j == ce) seek(a, u + npairs, npairs);
+    else first = false;
+  }
+  __device__ __forceinline__ bool done(const AttArgs &a) const { return u >= num_units(a); }
+};
 
 // ------------------------------------------------------------------------------------------------ plan
 // neff[row] = 1 + largest j with a usable idx[row, j] (0 if none); flags positions outside [0, seq_len).
@@ -159,9 +196,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sQ = smem;                                  // [9 dim blocks][64 heads][128 B]
-  uint8_t *sBuf = sQ + kAttQBytes;                     // 2 x [9 dim blocks][48 tokens][128 B]
-  uint8_t *sP = sBuf + 2 * kAttBufBytes;               // [2 token blocks][64 heads][128 B]
-  AttSmem *S = (AttSmem *)(sP + kAttPBytes);
+  uint8_t *sBuf = sQ + kAttQBytes;                     // 3 x [9 dim blocks][32 tokens][128 B]
+  uint8_t *sP = sBuf + kAttNBuf * kAttBufBytes;        // 2 x [64 heads][64 tokens] bf16; epilogue staging
+  AttSmem *S = (AttSmem *)(sP + 2 * kAttPBytes);
 
   const uint32_t rank = tc::cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -169,21 +206,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
   const int U = num_units(a);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAttNBuf; ++i) {
       tc::mbar_init(tc::smem_u32(&S->buf_full[i]), 4);
       tc::mbar_init(tc::smem_u32(&S->pair_full[i]), 2);
       tc::mbar_init(tc::smem_u32(&S->buf_empty[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->v_ready[i]), 8);
+    }
+    for (int i = 0; i < 2; ++i) {
       tc::mbar_init(tc::smem_u32(&S->s_full[i]), 1);
-      tc::mbar_init(tc::smem_u32(&S->xchg[i]), 4);
+      tc::mbar_init(tc::smem_u32(&S->p_full[i]), 8);
+      tc::mbar_init(tc::smem_u32(&S->pv_done[i]), 1);
     }
     tc::mbar_init(tc::smem_u32(&S->q_full), 1);
     tc::mbar_init(tc::smem_u32(&S->pair_q_full), 2);
     tc::mbar_init(tc::smem_u32(&S->q_empty), 1);
-    tc::mbar_init(tc::smem_u32(&S->p_full), 8);
-    tc::mbar_init(tc::smem_u32(&S->pv_done), 1);
     tc::mbar_init(tc::smem_u32(&S->o_empty), 8);
     tc::mbar_init(tc::smem_u32(&S->drain), 1);
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kAttRing; ++i) {
+      tc::mbar_init(tc::smem_u32(&S->phys_full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&S->phys_empty[i]), 8);
       tc::mbar_init(tc::smem_u32(&S->mask_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&S->mask_empty[i]), 4);
     }
@@ -192,7 +233,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     tc::prefetch_tmap(&tm_q);
     tc::prefetch_tmap(&tm_kv);
   }
-  if (warp == 8) {
+  if (warp == kAttWarpMMA) {
     tc::tmem_alloc2(tc::smem_u32(&S->tmem_base), 512);
     tc::tmem_relinquish2();
   }
@@ -200,127 +241,177 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
   __syncthreads();
   tc::cluster_sync();
   tc::fence_after_sync();
+  // Each role starts by moving registers: the softmax warpgroup takes them from the three data-movement
+  // warpgroups (every warp of a warpgroup executes the same setmaxnreg).
+#define ATT_REGS_DEC() asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kAttRegsOther))
+#define ATT_REGS_INC() asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kAttRegsSoftmax))
   const uint32_t tmem = S->tmem_base;
   volatile int *abort = &S->abort;
   uint32_t *status = a.status;
 
-  if (warp >= 4 && warp < 8) {
+  if (warp == kAttWarpResolve) {
+    // ====================================================================== resolve (32 threads)
+    ATT_REGS_DEC();
+    // Chunk c of this pair: token positions -> physical rows (ring slot c % kAttRing, -1 = masked) and two
+    // validity words; on entering a unit this CTA's 64 q rows are prefetched into L2.
+    // The idx loads of chunk c + 1 are in flight while the block-table loads of chunk c resolve.
+    ChunkCursor cur, nxt;
+    cur.seek(a, pair, npairs);
+    auto load_idx = [&](const ChunkCursor &cc, int (&s)[2]) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int j = cc.j * kAttChunk + 32 * e + lane;
+        s[e] = (!cc.done(a) && j < a.k) ? __ldg(a.idx + (int64_t)cc.row * a.k + j) : -1;
+      }
+    };
+    int s_cur[2];
+    load_idx(cur, s_cur);
+    nxt = cur;
+    if (!nxt.done(a)) nxt.next(a, npairs);
+    for (uint32_t c = 0; !cur.done(a); ++c) {
+      int s_nxt[2];
+      load_idx(nxt, s_nxt);
+      if (cur.first) {
+        const __nv_bfloat16 *qr = a.q + ((int64_t)cur.row * kAttH + 64 * (int)rank) * kAttD;
+        tc::prefetch_l2(qr + (int64_t)lane * kAttD, kAttD * 2);
+        tc::prefetch_l2(qr + (int64_t)(lane + 32) * kAttD, kAttD * 2);
+      }
+      int32_t pr[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        pr[e] = -1;
+        const int s = s_cur[e];
+        if (s >= 0 && s < cur.seq) {
+          const int blk = __ldg(cur.btr + (s >> 6));
+          if ((unsigned)blk < (unsigned)a.bv.num_blocks) pr[e] = blk * 64 + (s & 63);
+          else set_status(status, kStatusBadIndex);
+        }
+      }
+      const uint32_t w0 = __ballot_sync(0xffffffffu, pr[0] >= 0), w1 = __ballot_sync(0xffffffffu, pr[1] >= 0);
+      const uint32_t slot = c % kAttRing, ph = ((c / kAttRing) & 1u) ^ 1u;
+      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->phys_empty[slot]), ph, abort, status) &&
+                                                  tc::mbar_wait(tc::smem_u32(&S->mask_empty[slot]), ph, abort, status));
+      if (ok) {
+        S->phys[slot][lane] = pr[0];
+        S->phys[slot][32 + lane] = pr[1];
+        if (lane == 0) {
+          S->mask[slot][0] = w0;
+          S->mask[slot][1] = w1;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(tc::smem_u32(&S->phys_full[slot]));
+        tc::mbar_arrive(tc::smem_u32(&S->mask_full[slot]));
+      }
+      cur = nxt;
+      s_cur[0] = s_nxt[0];
+      s_cur[1] = s_nxt[1];
+      if (!nxt.done(a)) nxt.next(a, npairs);
+    }
+  } else if (warp >= 4 && warp < 8) {
     // ====================================================================== gather (128 threads)
-    // q by one tiled TMA per dim block; this CTA's 48 tokens of every chunk by TMA gather4 (4 rows x 128
-    // bytes per instruction, 128-byte swizzle applied by the copy engine), warp w taking dim blocks w, w+4
-    // (and 8 for warp 0).  Loops holding the named barrier never break: after a timeout every wait returns
-    // at once and the copies are skipped, so all 128 threads still meet at the barriers and the teardown.
+    ATT_REGS_DEC();
+    // Chunk c: this CTA's 32 tokens by TMA gather4 (4 rows x 128 bytes per instruction, 128-byte swizzle
+    // applied by the copy engine), warp w taking dim blocks w, w+4 (and 8 for warp 0); q by one tiled TMA
+    // per dim block when a unit starts.  The loop never breaks: after a timeout every wait returns at once
+    // and the copies are skipped.
     const int t = threadIdx.x - 128, pw = t >> 5;
     const int oob_row = a.bv.num_blocks * 64;           // outside the map: the copy engine fills zeros
-    uint32_t v = 0, g = 0;
-    // L2 prefetch cursor, kPrefetchAhead chunks ahead of the chunk being gathered: each CTA prefetches the
-    // full latent rows of its own 48 tokens (and the next unit's q when the cursor enters it)
-    int pf_u = pair, pf_c = 0, pf_row = -1, pf_cb = 0, pf_nch = 0, pf_seq = 0;
-    const int32_t *pf_btr = nullptr;
-    auto pf_enter = [&](int uu) {
-      for (; uu < U; uu += npairs) {
-        int r2, cb2, ce2;
-        unit_of(a, uu, &r2, &cb2, &ce2);
-        if (ce2 > cb2) {
-          int b2;
-          pos_of_row(a.bv, r2, &b2);
-          pf_u = uu; pf_c = 0; pf_row = r2; pf_cb = cb2; pf_nch = ce2 - cb2;
-          pf_seq = __ldg(a.bv.seq_lens + b2);
-          pf_btr = a.bv.block_table + (int64_t)b2 * a.bv.max_blocks_per_seq;
-          if (t < 64) tc::prefetch_l2(a.q + ((int64_t)r2 * kAttH + 64 * rank + t) * kAttD, kAttD * 2);
-          return;
+    ChunkCursor pc;
+    pc.seek(a, pair, npairs);
+    uint32_t v = 0;
+    for (uint32_t c = 0; !pc.done(a); ++c) {
+      const uint32_t b = c % kAttNBuf, use = c / kAttNBuf, slot = c % kAttRing;
+      const int nblk = pw == 0 ? 3 : 2;
+      bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->phys_full[slot]), (c / kAttRing) & 1u, abort, status));
+      if (lane == 0 && ok) {
+        ok = tc::mbar_wait_cl(tc::smem_u32(&S->buf_empty[b]), (use & 1u) ^ 1u, abort, status);
+        if (ok) tc::mbar_expect_tx(tc::smem_u32(&S->buf_full[b]), (uint32_t)nblk * kAttBlkBytes);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok && lane < kAttHalf / 4) {
+        const int32_t *ph = S->phys[slot] + kAttHalf * (int)rank + 4 * lane;
+        int r4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) r4[e] = ph[e] >= 0 ? ph[e] : oob_row;
+        for (int m = 0; m < nblk; ++m) {
+          const int d = pw + 4 * m;
+          tc::tma_gather4(tc::smem_u32(sBuf + b * kAttBufBytes + d * kAttBlkBytes + 4 * lane * 128), &tm_kv, d * 64, r4[0],
+                          r4[1], r4[2], r4[3], tc::smem_u32(&S->buf_full[b]));
         }
       }
-      pf_u = U;
-    };
-    auto pf_step = [&]() {
-      if (pf_u >= U) return;
-      if (t < kAttHalf) {
-        const int j = (pf_cb + pf_c) * kAttChunk + kAttHalf * (int)rank + t;
-        if (j < a.k) {
-          const int s = __ldg(a.idx + (int64_t)pf_row * a.k + j);
-          if (s >= 0 && s < pf_seq) {
-            const int blk = __ldg(pf_btr + (s >> 6));
-            if ((unsigned)blk < (unsigned)a.bv.num_blocks)
-              tc::prefetch_l2(a.kv + ((int64_t)blk * 64 + (s & 63)) * kAttD, kAttD * 2);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->phys_empty[slot]));
+      if (pc.first) {
+        if (t == 0) {
+          const bool okq = v == 0 || tc::mbar_wait_cl(tc::smem_u32(&S->q_empty), (v - 1) & 1u, abort, status);
+          if (okq) {
+            const uint32_t bar = tc::smem_u32(&S->q_full);
+            tc::mbar_expect_tx(bar, kAttQBytes);
+            for (int d = 0; d < 9; ++d)
+              tc::tma_load_2d(tc::smem_u32(sQ + d * 8192), &tm_q, d * 64, pc.row * kAttH + 64 * (int)rank, bar);
           }
         }
+        ++v;
       }
-      if (++pf_c == pf_nch) pf_enter(pf_u + npairs);
-    };
-    pf_enter(pair);
-    for (int d = 0; d < kPrefetchAhead; ++d) pf_step();
+      pc.next(a, npairs);
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ====================================================================== cross (128 threads)
+    ATT_REGS_DEC();
+    // Chunk c: the peer's 32 tokens' half of the values (rank 0 takes dims 0-255, rank 1 dims 256-511),
+    // 16 bytes per load, a warp reading one 512-byte row segment per step, into registers; once QK^T of the
+    // chunk has run they are stored with the 128-byte swizzle into the dim blocks it no longer needs
+    // (rank 0: 4-7, rank 1: 0-3).  Masked tokens store zeros.
+    const int t = threadIdx.x - 256;
+    const uint32_t dst_blk0 = rank == 0 ? 4u : 0u;
+    const int dim0 = rank == 0 ? 0 : 256;
+    constexpr int kCrossVec = 4 * kAttBlkBytes / 16 / 128;      // 16-byte loads per thread
+    const uint32_t v_ready_r0 = tc::map_to_rank(tc::smem_u32(&S->v_ready[0]), 0);
+    uint32_t c = 0;
     for (int u = pair; u < U; u += npairs) {
       int row, cb, ce;
       unit_of(a, u, &row, &cb, &ce);
-      const int nch = ce - cb;
-      if (nch <= 0) continue;
-      int b;
-      pos_of_row(a.bv, row, &b);
-      const int seq_len = __ldg(a.bv.seq_lens + b);
-      const int32_t *btr = a.bv.block_table + (int64_t)b * a.bv.max_blocks_per_seq;
-      if (t == 0) {
-        const bool ok = v == 0 || tc::mbar_wait_cl(tc::smem_u32(&S->q_empty), (v - 1) & 1u, abort, status);
-        if (ok) {
-          const uint32_t bar = tc::smem_u32(&S->q_full);
-          tc::mbar_expect_tx(bar, kAttQBytes);
-          for (int d = 0; d < 9; ++d)
-            tc::tma_load_2d(tc::smem_u32(sQ + d * 8192), &tm_q, d * 64, row * kAttH + 64 * (int)rank, bar);
-        }
-      }
-      for (int i = 0; i < nch; ++i, ++g) {
-        const uint32_t bi = g & 1u, use = g >> 1;
-        pf_step();
-        // token positions of the chunk -> physical rows (-1: masked); validity words go to the softmax
-        const uint32_t mslot = g & 3u;
-        const bool m_ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->mask_empty[mslot]),
-                                                                ((g >> 2) & 1u) ^ 1u, abort, status));
-        tc::named_bar_sync(1, 128);
-        {
-          int32_t pr = -1;
-          const int j = (cb + i) * kAttChunk + t;
-          if (t < kAttChunk && j < a.k) {
-            const int s = __ldg(a.idx + (int64_t)row * a.k + j);
-            if (s >= 0 && s < seq_len) {
-              const int blk = __ldg(btr + (s >> 6));
-              if ((unsigned)blk < (unsigned)a.bv.num_blocks) pr = blk * 64 + (s & 63);
-              else set_status(status, kStatusBadIndex);
-            }
-          }
-          if (t < kAttChunk) S->phys[bi][t] = pr;
-          const unsigned bits = __ballot_sync(0xffffffffu, pr >= 0);
-          if (lane == 0 && m_ok && pw < 3) S->mask[mslot][pw] = bits;
-        }
-        tc::named_bar_sync(1, 128);
-        if (t == 0) tc::mbar_arrive(tc::smem_u32(&S->mask_full[mslot]));
-        // this warp's dim blocks of this CTA's 48 tokens, into chunk buffer bi
-        const int nblk = pw == 0 ? 3 : 2;
-        bool ok = true;
-        if (lane == 0) {
-          ok = tc::mbar_wait_cl(tc::smem_u32(&S->buf_empty[bi]), (use & 1u) ^ 1u, abort, status);
-          if (ok) tc::mbar_expect_tx(tc::smem_u32(&S->buf_full[bi]), (uint32_t)nblk * kAttBlkBytes);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok && lane < kAttHalf / 4) {
-          const int32_t *ph = S->phys[bi] + kAttHalf * (int)rank + 4 * lane;
-          int r4[4];
+      for (int i = 0; i < ce - cb; ++i, ++c) {
+        const uint32_t b = c % kAttNBuf, slot = c % kAttRing;
+        const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->phys_full[slot]), (c / kAttRing) & 1u, abort, status));
+        const int32_t *ph = S->phys[slot] + kAttHalf * (int)(rank ^ 1u);
+        uint4 val[kCrossVec];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) r4[e] = ph[e] >= 0 ? ph[e] : oob_row;
-          for (int m = 0; m < nblk; ++m) {
-            const int d = pw + 4 * m;
-            tc::tma_gather4(tc::smem_u32(sBuf + bi * kAttBufBytes + d * kAttBlkBytes + 4 * lane * 128), &tm_kv, d * 64,
-                            r4[0], r4[1], r4[2], r4[3], tc::smem_u32(&S->buf_full[bi]));
+        for (int m = 0; m < kCrossVec; ++m) {
+          const int idx = t + 128 * m, r = idx >> 5, cq = idx & 31;
+          const int pr = ph[r];
+          val[m] = (ok && pr >= 0) ? __ldg(reinterpret_cast<const uint4 *>(a.kv + (int64_t)pr * kAttD + dim0 + cq * 8))
+                                   : make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->phys_empty[slot]));
+        // QK^T of the chunk has read this CTA's buffer
+        const bool have = __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->s_full[c & 1u]), (c >> 1) & 1u, abort, status));
+        if (have) {
+          uint8_t *base = sBuf + b * kAttBufBytes + dst_blk0 * kAttBlkBytes;
+#pragma unroll
+          for (int m = 0; m < kCrossVec; ++m) {
+            const int idx = t + 128 * m, r = idx >> 5, cq = idx & 31;
+            *reinterpret_cast<uint4 *>(base + (cq >> 3) * kAttBlkBytes + r * 128 + (((cq & 7) ^ (r & 7)) << 4)) = val[m];
           }
         }
+        tc::fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) tc::mbar_arrive(tc::smem_u32(&S->v_ready[b]));
+          else tc::mbar_arrive_cluster(v_ready_r0 + b * 8);
+        }
       }
-      ++v;
     }
-  } else if (warp == 9) {
+  } else if (warp == kAttWarpRelay) {
     // ====================================================================== relay (lane 0)
+    ATT_REGS_DEC();
     if (lane == 0) {
       const uint32_t peer_pair_full = tc::map_to_rank(tc::smem_u32(&S->pair_full[0]), 0);
       const uint32_t peer_pair_q = tc::map_to_rank(tc::smem_u32(&S->pair_q_full), 0);
-      uint32_t v = 0, g = 0;
+      uint32_t v = 0, c = 0;
       bool ok = true;
       for (int u = pair; u < U && ok; u += npairs) {
         int row, cb, ce;
@@ -328,42 +419,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         const int nch = ce - cb;
         if (nch <= 0) continue;
         if (!tc::mbar_wait(tc::smem_u32(&S->q_full), v & 1u, abort, status)) break;
-        tc::fence_proxy_async();
         tc::mbar_arrive_cluster(peer_pair_q);
-        for (int i = 0; i < nch; ++i, ++g) {
-          if (!tc::mbar_wait(tc::smem_u32(&S->buf_full[g & 1u]), (g >> 1) & 1u, abort, status)) { ok = false; break; }
-          tc::fence_proxy_async();
-          tc::mbar_arrive_cluster(peer_pair_full + (g & 1u) * 8);
+        for (int i = 0; i < nch; ++i, ++c) {
+          const uint32_t b = c % kAttNBuf;
+          if (!tc::mbar_wait(tc::smem_u32(&S->buf_full[b]), (c / kAttNBuf) & 1u, abort, status)) { ok = false; break; }
+          tc::mbar_arrive_cluster(peer_pair_full + b * 8);
         }
         ++v;
       }
     }
-  } else if (warp == 8) {
-    // ====================================================================== MMA issuer (rank 0, lane 0)
-    if (rank == 0 && lane == 0) {
+  } else if (warp == kAttWarpMMA) {
+    // ====================================================================== MMA issuer (rank 0, whole warp)
+    ATT_REGS_DEC();
+    // The warp runs the loop uniformly and one elected lane issues each MMA and commit.  Descriptors are a
+    // base descriptor plus the byte offset / 16 (the address field cannot carry: shared memory < 256 KB).
+    if (rank == 0) {
       const uint32_t idesc_qk = tc::make_idesc(1, 1, 128, kAttChunk, false, false);
       const uint32_t idesc_pv = tc::make_idesc(1, 1, 128, 256, false, true);
       const uint16_t both = 3;
-      const uint32_t qbase = tc::smem_u32(sQ), pbase = tc::smem_u32(sP);
-      uint32_t v = 0, g = 0;
+      const uint64_t q_desc = tc::desc_sw128(tc::smem_u32(sQ), 1024);
+      const uint64_t p_desc = tc::desc_sw128(tc::smem_u32(sP), 1024);
+      const uint64_t kv_desc = tc::desc_sw128(tc::smem_u32(sBuf), 1024);
+      const uint64_t v_desc = tc::desc_sw128_lbo(tc::smem_u32(sBuf), kAttBlkBytes, 1024);
+      uint32_t v = 0, c = 0;
       bool ok = true;
-      auto pv = [&](uint32_t gc, bool first) -> bool {
-        if (!tc::mbar_wait_cl(tc::smem_u32(&S->p_full), gc & 1u, abort, status)) return false;
-        if (first && v > 0 && !tc::mbar_wait_cl(tc::smem_u32(&S->o_empty), (v - 1) & 1u, abort, status)) return false;
+      auto pv = [&](uint32_t cc, bool first) -> bool {
+        const uint32_t b = cc % kAttNBuf, pb = cc & 1u;
+        if (!tc::mbar_wait_cl_w(tc::smem_u32(&S->p_full[pb]), (cc >> 1) & 1u, abort, status)) return false;
+        if (!tc::mbar_wait_cl_w(tc::smem_u32(&S->v_ready[b]), (cc / kAttNBuf) & 1u, abort, status)) return false;
+        if (first && v > 0 && !tc::mbar_wait_cl_w(tc::smem_u32(&S->o_empty), (v - 1) & 1u, abort, status)) return false;
         tc::fence_after_sync();
-        const uint32_t base = tc::smem_u32(sBuf + (gc & 1u) * kAttBufBytes);
+        const uint64_t pa = p_desc + ((pb * kAttPBytes) >> 4), vb = v_desc + ((b * kAttBufBytes) >> 4);
+#pragma unroll
         for (int p = 0; p < 2; ++p)
+#pragma unroll
           for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
             for (int ks = 0; ks < kAttHalf / 16; ++ks) {
               const int kg = (kAttHalf / 16) * kh + ks;          // 16-token step within the chunk
-              const uint64_t ad = tc::desc_sw128(pbase + (kg >> 2) * 8192 + (kg & 3) * 32, 1024);
-              const uint64_t bd =
-                  tc::desc_sw128_lbo(base + (4 * kh + 2 * p) * kAttBlkBytes + ks * 2048, kAttBlkBytes, 1024);
-              tc::mma_bf16_pair(tmem + kTmemO + 128 * p, ad, bd, idesc_pv, (first && kg == 0) ? 0u : 1u);
+              tc::mma_bf16_pair_w(tmem + kTmemO + 128 * p, pa + ((kg * 32) >> 4),
+                                  vb + (((4 * kh + 2 * p) * kAttBlkBytes + ks * 2048) >> 4), idesc_pv,
+                                  (first && kg == 0) ? 0u : 1u);
             }
-        tc::mma_commit_pair(tc::smem_u32(&S->buf_empty[gc & 1u]), both);
-        tc::mma_commit_pair(tc::smem_u32(&S->pv_done), both);
+        tc::mma_commit_pair_w(tc::smem_u32(&S->buf_empty[b]), both);
+        tc::mma_commit_pair_w(tc::smem_u32(&S->pv_done[pb]), both);
         return true;
       };
       for (int u = pair; u < U && ok; u += npairs) {
@@ -371,50 +470,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         unit_of(a, u, &row, &cb, &ce);
         const int nch = ce - cb;
         if (nch <= 0) continue;
-        if (!tc::mbar_wait_cl(tc::smem_u32(&S->pair_q_full), v & 1u, abort, status)) break;
+        if (!tc::mbar_wait_cl_w(tc::smem_u32(&S->pair_q_full), v & 1u, abort, status)) break;
         tc::fence_after_sync();
-        const uint32_t g0 = g;
+        const uint32_t c0 = c;
         for (int i = 0; i < nch; ++i) {
-          if (!tc::mbar_wait_cl(tc::smem_u32(&S->pair_full[g & 1u]), (g >> 1) & 1u, abort, status)) { ok = false; break; }
+          const uint32_t b = c % kAttNBuf;
+          if (!tc::mbar_wait_cl_w(tc::smem_u32(&S->pair_full[b]), (c / kAttNBuf) & 1u, abort, status)) { ok = false; break; }
           tc::fence_after_sync();
-          const uint32_t base = tc::smem_u32(sBuf + (g & 1u) * kAttBufBytes);
-          const uint32_t sb = tmem + kTmemS + kAttHalf * (g & 1u);
+          const uint64_t kb = kv_desc + ((b * kAttBufBytes) >> 4);
+          const uint32_t sb = tmem + kTmemS + kAttHalf * (c & 1u);
+#pragma unroll 1
           for (int d = 0; d < 9; ++d) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = tc::desc_sw128(qbase + d * 8192 + kk * 32, 1024);
-              const uint64_t bd = tc::desc_sw128(base + d * kAttBlkBytes + kk * 32, 1024);
-              tc::mma_bf16_pair(sb, ad, bd, idesc_qk, (d == 0 && kk == 0) ? 0u : 1u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              tc::mma_bf16_pair_w(sb, q_desc + ((d * 8192 + kk * 32) >> 4), kb + ((d * kAttBlkBytes + kk * 32) >> 4),
+                                  idesc_qk, (d == 0 && kk == 0) ? 0u : 1u);
           }
-          tc::mma_commit_pair(tc::smem_u32(&S->s_full[g & 1u]), both);
-          if (i == nch - 1) tc::mma_commit_pair(tc::smem_u32(&S->q_empty), both);
-          ++g;
-          if (i > 0 && !pv(g0 + i - 1, i - 1 == 0)) { ok = false; break; }
+          tc::mma_commit_pair_w(tc::smem_u32(&S->s_full[c & 1u]), both);
+          if (i == nch - 1) tc::mma_commit_pair_w(tc::smem_u32(&S->q_empty), both);
+          ++c;
+          if (i > 0 && !pv(c0 + i - 1, i - 1 == 0)) { ok = false; break; }
         }
-        if (ok && !pv(g0 + nch - 1, nch == 1)) ok = false;
+        if (ok && !pv(c0 + nch - 1, nch == 1)) ok = false;
         ++v;
       }
-      tc::mma_commit_pair_local(tc::smem_u32(&S->drain));
+      tc::mma_commit_pair_local_w(tc::smem_u32(&S->drain));
       volatile int no_abort = 0;
-      tc::mbar_wait(tc::smem_u32(&S->drain), 0, &no_abort, status);
+      __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->drain), 0, &no_abort, status));
     }
+  } else if (warp >= 4) {
+    ATT_REGS_DEC();                            // the spare warp of the last warpgroup
   } else {
-    // ====================================================================== swap + softmax + epilogue
-    // Like the gather role, these loops never break (they hold named barrier 2): after a timeout the
-    // waits return at once and the remaining chunks run through without touching TMEM or memory.
+    // ====================================================================== softmax + epilogue (warps 0-3)
+    ATT_REGS_INC();
+    // The loops never break (they hold named barrier 2): after a timeout the waits return at once and the
+    // remaining chunks run through without touching TMEM or memory.
     const int L = threadIdx.x;                 // TMEM lane
     const int h = L & 63, half = L >> 6;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t p_full_r0 = tc::map_to_rank(tc::smem_u32(&S->p_full), 0);
+    const uint32_t p_full_r0 = tc::map_to_rank(tc::smem_u32(&S->p_full[0]), 0);
     const uint32_t o_empty_r0 = tc::map_to_rank(tc::smem_u32(&S->o_empty), 0);
-    const uint32_t peer_buf = tc::map_to_rank(tc::smem_u32(sBuf), rank ^ 1u);
-    const uint32_t peer_xchg = tc::map_to_rank(tc::smem_u32(&S->xchg[0]), rank ^ 1u);
-    // the swap moves the value dims this CTA needs from the peer's tokens: rank 0 takes dim blocks 0-3 of
-    // rank 1's tokens into its blocks 4-7; rank 1 takes dim blocks 4-7 of rank 0's tokens into its blocks 0-3
-    const uint32_t src_off = (rank == 0 ? 0u : 4u) * kAttBlkBytes, dst_off = (rank == 0 ? 4u : 0u) * kAttBlkBytes;
-    constexpr int kSwapVec = 4 * kAttBlkBytes / 16 / 128;       // 16-byte vectors per thread
-    uint32_t g = 0, v = 0;
+    uint32_t c = 0;
     for (int u = pair; u < U; u += npairs) {
       int row, cb, ce;
       unit_of(a, u, &row, &cb, &ce);
@@ -424,87 +520,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         // nothing selected: o = 0, lse = -inf
         if (a.splits == 1) {
           __nv_bfloat16 *o = a.out + ((int64_t)row * kAttH + head) * kAttDv + 256 * half;
-          for (int c = 0; c < 256; c += 8) *reinterpret_cast<uint4 *>(o + c) = make_uint4(0, 0, 0, 0);
+          for (int e = 0; e < 256; e += 8) *reinterpret_cast<uint4 *>(o + e) = make_uint4(0, 0, 0, 0);
           if (a.lse && half == 0) a.lse[(int64_t)row * kAttH + head] = -INFINITY;
         } else {
           float *o = a.part_o + ((int64_t)u * kAttH + head) * kAttDv + 256 * half;
-          for (int c = 0; c < 256; c += 4) *reinterpret_cast<float4 *>(o + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int e = 0; e < 256; e += 4) *reinterpret_cast<float4 *>(o + e) = make_float4(0.f, 0.f, 0.f, 0.f);
           if (half == 0) a.part_lse[(int64_t)u * kAttH + head] = -INFINITY;
         }
         continue;
       }
-      float m_run = -INFINITY, l_run = 0.f, l_exact = 0.f;
-      for (int i = 0; i < nch; ++i, ++g) {
-        const uint32_t bi = g & 1u;
-        // validity of this thread's 48 tokens, published by the gather warps
-        const uint32_t mslot = g & 3u;
-        const bool m_ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->mask_full[mslot]),
-                                                                (g >> 2) & 1u, abort, status));
-        uint64_t valid = 0;
-        if (m_ok) {
-          const uint64_t w0 = S->mask[mslot][0], w1 = S->mask[mslot][1], w2 = S->mask[mslot][2];
-          valid = half == 0 ? (w0 | (w1 << 32)) : ((w1 >> 16) | (w2 << 16));
-          valid &= (1ull << kAttHalf) - 1ull;
-        }
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int i = 0; i < nch; ++i, ++c) {
+        // validity of this thread's 32 tokens
+        const uint32_t slot = c % kAttRing;
+        const bool m_ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->mask_full[slot]),
+                                                                (c / kAttRing) & 1u, abort, status));
+        uint32_t valid = m_ok ? S->mask[slot][half] : 0u;
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->mask_empty[mslot]));
+        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->mask_empty[slot]));
         const bool have_s =
-            __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->s_full[bi]), (g >> 1) & 1u, abort, status));
+            __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->s_full[c & 1u]), (c >> 1) & 1u, abort, status));
         tc::fence_after_sync();
-        // ---- swap over distributed shared memory: read the peer's values, hand-shake, write them here
-        {
-          uint4 sw[kSwapVec];
-#pragma unroll
-          for (int m = 0; m < kSwapVec; ++m)
-            sw[m] = have_s ? tc::ld_dsmem16(peer_buf + bi * kAttBufBytes + src_off + (L + 128 * m) * 16)
-                           : make_uint4(0, 0, 0, 0);
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive_cluster(peer_xchg + bi * 8);
-          const bool got = __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->xchg[bi]), (g >> 1) & 1u, abort, status));
-          if (have_s && got) {
-#pragma unroll
-            for (int m = 0; m < kSwapVec; ++m)
-              *reinterpret_cast<uint4 *>(sBuf + bi * kAttBufBytes + dst_off + (L + 128 * m) * 16) = sw[m];
-          }
-        }
-        // ---- S for this thread's head and 48 tokens
         float sv[kAttHalf];
-        {
-          float t0[32], t1[16];
-          const uint32_t sa = tmem + lane_base + kTmemS + kAttHalf * bi;
-          tc::tmem_ld32(sa, t0);
-          tc::tmem_ld16(sa + 32, t1);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) sv[c] = t0[c];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) sv[32 + c] = t1[c];
-        }
-        if (!have_s) valid = 0;
+        tc::tmem_ld32(tmem + lane_base + kTmemS + kAttHalf * (c & 1u), sv);
+        tc::tmem_wait_ld();
+        if (!have_s) valid = 0u;
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kAttHalf; ++c) {
-          sv[c] = ((valid >> c) & 1ull) ? sv[c] * a.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, sv[c]);
+        for (int e = 0; e < kAttHalf; ++e) {
+          sv[e] = ((valid >> e) & 1u) ? sv[e] * a.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sv[e]);
         }
         const float mloc = fmaxf(m_run, mx);
-        S->xm[g & 1u][L] = mloc;
+        S->xm[c & 1u][L] = mloc;
         tc::named_bar_sync(2, 128);
-        const float m_new = fmaxf(mloc, S->xm[g & 1u][L ^ 64]);
-        // P V of the previous chunk must be finished before O is touched or P is overwritten
+        const float m_new = fmaxf(mloc, S->xm[c & 1u][L ^ 64]);
         bool pv_ok = true;
-        if (i > 0) {
-          pv_ok = tc::mbar_wait_cl(tc::smem_u32(&S->pv_done), (g - 1) & 1u, abort, status);
-          tc::fence_after_sync();
-        }
-        pv_ok = __all_sync(0xffffffffu, pv_ok);
         if (i == 0) {
           m_run = m_new;
         } else {
           // TMEM loads/stores are warp-collective: the warp rescales if any of its rows needs it,
-          // rows that do not keep their reference max (alpha = 1)
+          // rows that do not keep their reference max (alpha = 1).  P V of the previous chunk must
+          // have finished before O is touched.
           const bool want = m_new > m_run + kRescaleLog2;
           if (__any_sync(0xffffffffu, want)) {
+            const uint32_t cp = c - 1;
+            pv_ok = __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->pv_done[cp & 1u]), (cp >> 1) & 1u, abort, status));
+            tc::fence_after_sync();
             const float alpha = want ? tc::ex2(m_run - m_new) : 1.f;
             if (pv_ok) {
               for (int cc = 0; cc < 8; ++cc) {
@@ -519,92 +581,104 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
             }
             if (want) {
               l_run *= alpha;
-              l_exact *= alpha;
               m_run = m_new;
             }
           }
         }
-        // P = exp2(z - m) in bf16 into the 128-byte-swizzled A operand: row h, tokens 48*half + [0, 48).
-        // l_run sums the rounded P (what the MMA multiplies) and normalises O; l_exact gives lse.
+        // this chunk's P buffer was last read by P V of chunk c - 2
+        if (c >= 2)
+          pv_ok = __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->pv_done[c & 1u]), ((c >> 1) & 1u) ^ 1u, abort,
+                                                           status)) && pv_ok;
+        // P = exp2(z - m) in bf16 into the 128-byte-swizzled A operand: row h, tokens 32*half + [0, 32);
+        // masked tokens hold -inf and give 0.  l_run sums the unrounded P.
         if (pv_ok) {
-          float lsum = 0.f, lex = 0.f;
+          const float m_use = m_run == -INFINITY ? 0.f : m_run;
+          uint8_t *pbuf = sP + (c & 1u) * kAttPBytes + h * 128;
+          float lsum = 0.f;
 #pragma unroll
-          for (int c = 0; c < kAttHalf / 8; ++c) {
+          for (int q8 = 0; q8 < kAttHalf / 8; ++q8) {
             uint32_t w4[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int t0 = 8 * c + 2 * e;
-              const float p0 = ((valid >> t0) & 1ull) ? tc::ex2(sv[t0] - m_run) : 0.f;
-              const float p1 = ((valid >> (t0 + 1)) & 1ull) ? tc::ex2(sv[t0 + 1] - m_run) : 0.f;
+              const int t0 = 8 * q8 + 2 * e;
+              const float p0 = tc::ex2(sv[t0] - m_use), p1 = tc::ex2(sv[t0 + 1] - m_use);
+              lsum += p0 + p1;
               const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-              const float2 pr = __bfloat1622float2(pb);
-              lsum += pr.x + pr.y;
-              lex += p0 + p1;
               w4[e] = *reinterpret_cast<const uint32_t *>(&pb);
             }
-            const int kc = (kAttHalf / 8) * half + c;              // 8-token chunk within the 96 tokens
-            *reinterpret_cast<uint4 *>(sP + (kc >> 3) * 8192 + h * 128 + (((kc & 7) ^ (h & 7)) << 4)) =
-                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            const int kc = (kAttHalf / 8) * half + q8;             // 8-token group within the 64 tokens
+            *reinterpret_cast<uint4 *>(pbuf + (((kc & 7) ^ (h & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
           l_run += lsum;
-          l_exact += lex;
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive_cluster(p_full_r0);
+        if (lane == 0) {
+          if (rank == 0) tc::mbar_arrive(tc::smem_u32(&S->p_full[c & 1u]));
+          else tc::mbar_arrive_cluster(p_full_r0 + (c & 1u) * 8);
+        }
       }
-      // ---- epilogue: wait for the last P V, normalise, store
+      // ---- epilogue: wait for the last P V, normalise, store through a per-warp staging tile
+      const uint32_t cl = c - 1;
       const bool o_ok =
-          __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->pv_done), (g - 1) & 1u, abort, status));
+          __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->pv_done[cl & 1u]), (cl >> 1) & 1u, abort, status));
       tc::fence_after_sync();
-      S->xl[0][L] = l_run;
-      S->xl[1][L] = l_exact;
+      S->xl[L] = l_run;
       tc::named_bar_sync(2, 128);
-      const float l_tot = l_run + S->xl[0][L ^ 64];
-      const float l_ex = l_exact + S->xl[1][L ^ 64];
+      const float l_tot = l_run + S->xl[L ^ 64];
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      const float lse_v = l_ex > 0.f ? (m_run + __log2f(l_ex)) * 0.69314718055994531f : -INFINITY;
+      const float lse_v = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       if (o_ok) {
-        if (a.splits == 1) {
-          __nv_bfloat16 *o = a.out + ((int64_t)row * kAttH + head) * kAttDv + 256 * half;
-          for (int cc = 0; cc < 8; ++cc) {
-            float ov[32];
-            tc::tmem_ld32(tmem + lane_base + kTmemO + 32 * cc, ov);
-            tc::tmem_wait_ld();
+        // both P buffers are free once the last P V finished: each warp stages a 32 x 32 fp32 tile
+        // (row = lane, 16-byte group j at j ^ (row & 7)) and writes whole 128-byte row segments
+        float *stg = reinterpret_cast<float *>(sP) + warp * 1024;
+        const int head0 = 64 * (int)rank + 32 * (warp & 1), col0 = 256 * (warp >> 1);
+        for (int cc = 0; cc < 8; ++cc) {
+          float ov[32];
+          tc::tmem_ld32(tmem + lane_base + kTmemO + 32 * cc, ov);
+          tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) {
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4 *>(stg + lane * 32 + 4 * (j ^ (lane & 7))) =
+                make_float4(ov[4 * j] * inv, ov[4 * j + 1] * inv, ov[4 * j + 2] * inv, ov[4 * j + 3] * inv);
+          __syncwarp();
+          if (a.splits == 1) {
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int r = 8 * it + (lane >> 2), j0 = 2 * (lane & 3);
+              const float4 f0 = *reinterpret_cast<const float4 *>(stg + r * 32 + 4 * (j0 ^ (r & 7)));
+              const float4 f1 = *reinterpret_cast<const float4 *>(stg + r * 32 + 4 * ((j0 + 1) ^ (r & 7)));
+              __nv_bfloat162 b0 = __floats2bfloat162_rn(f0.x, f0.y), b1 = __floats2bfloat162_rn(f0.z, f0.w);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(f1.x, f1.y), b3 = __floats2bfloat162_rn(f1.z, f1.w);
               uint4 w;
-              __nv_bfloat162 b0 = __floats2bfloat162_rn(ov[e] * inv, ov[e + 1] * inv);
-              __nv_bfloat162 b1 = __floats2bfloat162_rn(ov[e + 2] * inv, ov[e + 3] * inv);
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(ov[e + 4] * inv, ov[e + 5] * inv);
-              __nv_bfloat162 b3 = __floats2bfloat162_rn(ov[e + 6] * inv, ov[e + 7] * inv);
               w.x = *reinterpret_cast<uint32_t *>(&b0);
               w.y = *reinterpret_cast<uint32_t *>(&b1);
               w.z = *reinterpret_cast<uint32_t *>(&b2);
               w.w = *reinterpret_cast<uint32_t *>(&b3);
-              *reinterpret_cast<uint4 *>(o + 32 * cc + e) = w;
+              *reinterpret_cast<uint4 *>(a.out + ((int64_t)row * kAttH + head0 + r) * kAttDv + col0 + 32 * cc + 4 * j0) = w;
+            }
+          } else {
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int r = 4 * it + (lane >> 3), j = lane & 7;
+              *reinterpret_cast<float4 *>(a.part_o + ((int64_t)u * kAttH + head0 + r) * kAttDv + col0 + 32 * cc + 4 * j) =
+                  *reinterpret_cast<const float4 *>(stg + r * 32 + 4 * (j ^ (r & 7)));
             }
           }
-          if (a.lse && half == 0) a.lse[(int64_t)row * kAttH + head] = lse_v;
-        } else {
-          float *o = a.part_o + ((int64_t)u * kAttH + head) * kAttDv + 256 * half;
-          for (int cc = 0; cc < 8; ++cc) {
-            float ov[32];
-            tc::tmem_ld32(tmem + lane_base + kTmemO + 32 * cc, ov);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4 *>(o + 32 * cc + e) =
-                  make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv, ov[e + 3] * inv);
+          __syncwarp();
+        }
+        if (half == 0) {
+          if (a.splits == 1) {
+            if (a.lse) a.lse[(int64_t)row * kAttH + head] = lse_v;
+          } else {
+            a.part_lse[(int64_t)u * kAttH + head] = lse_v;
           }
-          if (half == 0) a.part_lse[(int64_t)u * kAttH + head] = lse_v;
         }
       }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive_cluster(o_empty_r0);
-      ++v;
     }
   }
 
@@ -612,10 +686,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::cluster_sync();
-  if (warp == 8) {
+  if (warp == kAttWarpMMA) {
     tc::fence_after_sync();
     tc::tmem_dealloc2(tmem, 512);
   }
+#undef ATT_REGS_DEC
+#undef ATT_REGS_INC
 }
 
 // ------------------------------------------------------------------------------------------------ combine
@@ -693,7 +769,9 @@ static bool make_bf16_rows_map(CUtensorMap *m, const void *base, uint64_t rows, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t attn_smem_bytes() { return 1024 + kAttQBytes + 2 * kAttBufBytes + kAttPBytes + sizeof(AttSmem); }
+static size_t attn_smem_bytes() {
+  return 1024 + kAttQBytes + kAttNBuf * kAttBufBytes + 2 * kAttPBytes + sizeof(AttSmem);
+}
 
 dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, int k, float softmax_scale,
                              const dsa_batch_t *b, void *out, float *lse, void *ws, bool decode, cudaStream_t stream,

@@ -314,8 +314,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             tc::mbar_wait(tc::smem_u32(&S->bfull[s2]), (b_last_par >> s2) & 1u, &no_abort, status);
           }
       }
-    } else if (warp == 1 && lane == 0) {
-      // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer (whole warp, one elected lane issues)
       int gi, t;
       unit_locate(pv.tile_prefix, G, u0, &gi, &t);
       int stage = 0, acc = 0, nb_groups = 0, bslot = 0, cur = -1;
@@ -323,34 +323,34 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       for (int u = u0; u < u1; ++u) {
         if (gi != cur) {
           bslot = nb_groups & 1;
-          if (!tc::mbar_wait(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort, status)) break;
+          if (!tc::mbar_wait_w(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort, status)) break;
           ++nb_groups;
           cur = gi;
         }
-        if (!tc::mbar_wait(tc::smem_u32(&S->tempty[acc]), acc_phase ^ 1u, abort, status)) break;
+        if (!tc::mbar_wait_w(tc::smem_u32(&S->tempty[acc]), acc_phase ^ 1u, abort, status)) break;
         tc::fence_after_sync();
-        if (!tc::mbar_wait(tc::smem_u32(&S->full[stage]), phase, abort, status)) break;
+        if (!tc::mbar_wait_w(tc::smem_u32(&S->full[stage]), phase, abort, status)) break;
         const int nr = pv.g_nrows[gi];
         const uint32_t idesc = tc::make_idesc(0, 0, 128, 64 * nr, false, false);
         const uint32_t a0 = tc::smem_u32(sA + stage * kIdxTileBytes);
         const uint32_t b0 = tc::smem_u32(sB + bslot * kIdxBSlotBytes);
 #pragma unroll
         for (int k = 0; k < kIdxDi / 32; ++k) {
-          tc::mma_f8f6f4(tmem + acc * 256, tc::desc_sw128(a0 + 32 * k, 1024), tc::desc_sw128(b0 + 32 * k, 1024), idesc,
+          tc::mma_f8f6f4_w(tmem + acc * 256, tc::desc_sw128(a0 + 32 * k, 1024), tc::desc_sw128(b0 + 32 * k, 1024), idesc,
                          k > 0 ? 1u : 0u);
         }
-        tc::mma_commit(tc::smem_u32(&S->empty[stage]));
-        tc::mma_commit(tc::smem_u32(&S->tfull[acc]));
+        tc::mma_commit_w(tc::smem_u32(&S->empty[stage]));
+        tc::mma_commit_w(tc::smem_u32(&S->tfull[acc]));
         const bool last_of_group = (t + 1 == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) || (u + 1 == u1);
-        if (last_of_group) tc::mma_commit(tc::smem_u32(&S->bempty[bslot]));
+        if (last_of_group) tc::mma_commit_w(tc::smem_u32(&S->bempty[bslot]));
         if (++stage == kIdxStages) { stage = 0; phase ^= 1u; }
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         if (++t == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) { ++gi; t = 0; }
       }
       // every MMA issued by this thread has completed before TMEM is released
-      tc::mma_commit(tc::smem_u32(&S->drain));
+      tc::mma_commit_w(tc::smem_u32(&S->drain));
       volatile int no_abort = 0;
-      tc::mbar_wait(tc::smem_u32(&S->drain), 0, &no_abort, status);
+      tc::mbar_wait_w(tc::smem_u32(&S->drain), 0, &no_abort, status);
     } else if (warp >= 2 && warp < 6) {
       // ------------------------------------------------------------------ epilogue
       const int quad = warp & 3;                 // TMEM lane quadrant this warp may access

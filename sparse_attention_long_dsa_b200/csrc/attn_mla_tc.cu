@@ -27,9 +27,9 @@
 //              running max grows by more than 2^8 (exact: the final division uses the same reference max);
 //   * P V    : M = 128 heads, N = 512 values as two N = 256 MMAs (rank r supplies values 256r..256r+255),
 //              K = 64 tokens; O (64 heads x 512 fp32 per CTA) stays in TMEM, 256 columns.
-// Every MMA is issued by one thread of rank 0 for the pair (cta_group::2).  Rank 1's buffer completions
-// are relayed to rank 0's barriers by one thread.  Token positions that are -1 (or out of range) are
-// zero-filled by the copy engine and masked.
+// Every MMA is issued by rank 0's MMA warp for the pair (cta_group::2).  Both CTAs' copies of a chunk (and
+// of q) complete on rank 0's barriers (.cta_group::2 TMA), so rank 0 sees one barrier per operand.  Token
+// positions that are -1 (or out of range) are zero-filled by the copy engine and masked.
 //
 // Units: prefill = one row (all its chunks); decode = (row, split) pairs whose partial (o, lse) are
 // merged by attn_combine_kernel.  Rows are taken longest-first (reverse order) round-robin over pairs.
@@ -46,9 +46,10 @@ constexpr int kAttChunk = 64;                    // tokens per chunk (32 per CTA
 constexpr int kAttHalf = kAttChunk / 2;
 constexpr int kAttNBuf = 3;                      // chunk buffers
 constexpr int kAttRing = 4;                      // resolved chunks (physical rows + masks) in flight
-constexpr int kAttThreads = 512;                 // warpgroups: softmax, gather, cross, (MMA, relay, resolve, -)
-constexpr int kAttWarpMMA = 12, kAttWarpRelay = 13, kAttWarpResolve = 14;
-constexpr uint32_t kAttRegsSoftmax = 224, kAttRegsOther = 96;    // 128 x 224 + 384 x 96 = 65536
+constexpr int kAttThreads = 512;                 // warpgroups: softmax, gather, cross, (MMA, -, resolve, -)
+constexpr int kAttWarpMMA = 12, kAttWarpResolve = 14;
+// registers per thread after the split: 128 x (224 + 96 + 96 + 96) = 65536
+constexpr uint32_t kAttRegsSoftmax = 224, kAttRegsGather = 96, kAttRegsCross = 96, kAttRegsMisc = 96;
 constexpr uint32_t kAttBlkBytes = kAttHalf * 128;                // one dim block of a CTA's 32 tokens: 4 KB
 constexpr uint32_t kAttBufBytes = 9 * kAttBlkBytes;              // 36 KB
 constexpr uint32_t kAttQBytes = 9 * 8192;
@@ -57,11 +58,10 @@ constexpr uint32_t kTmemO = 0, kTmemS = 256;     // O: 256 columns; S: two buffe
 constexpr float kRescaleLog2 = 8.0f;
 
 struct AttSmem {
-  uint64_t buf_full[kAttNBuf];      // local: TMA bytes of this CTA's half of a chunk (4 gather warps)
-  uint64_t pair_full[kAttNBuf];     // rank 0: 2 relays
+  uint64_t buf_full[kAttNBuf];      // rank 0: TMA bytes of both CTAs' halves of a chunk (4 gather warps expect)
   uint64_t buf_empty[kAttNBuf];     // MMA commit to both CTAs after P V of the chunk
   uint64_t v_ready[kAttNBuf];       // rank 0: 8 cross warps (both CTAs) stored the peer's values
-  uint64_t q_full, pair_q_full, q_empty;
+  uint64_t q_full, q_empty;         // q_full: rank 0, both CTAs' q bytes
   uint64_t s_full[2];               // MMA commit to both CTAs
   uint64_t p_full[2];               // rank 0: 8 softmax warps wrote P
   uint64_t pv_done[2];              // MMA commit to both CTAs, per P buffer
@@ -208,7 +208,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kAttNBuf; ++i) {
       tc::mbar_init(tc::smem_u32(&S->buf_full[i]), 4);
-      tc::mbar_init(tc::smem_u32(&S->pair_full[i]), 2);
       tc::mbar_init(tc::smem_u32(&S->buf_empty[i]), 1);
       tc::mbar_init(tc::smem_u32(&S->v_ready[i]), 8);
     }
@@ -218,7 +217,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
       tc::mbar_init(tc::smem_u32(&S->pv_done[i]), 1);
     }
     tc::mbar_init(tc::smem_u32(&S->q_full), 1);
-    tc::mbar_init(tc::smem_u32(&S->pair_q_full), 2);
     tc::mbar_init(tc::smem_u32(&S->q_empty), 1);
     tc::mbar_init(tc::smem_u32(&S->o_empty), 8);
     tc::mbar_init(tc::smem_u32(&S->drain), 1);
@@ -243,7 +241,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
   tc::fence_after_sync();
   // Each role starts by moving registers: the softmax warpgroup takes them from the three data-movement
   // warpgroups (every warp of a warpgroup executes the same setmaxnreg).
-#define ATT_REGS_DEC() asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kAttRegsOther))
+#define ATT_REGS_DEC(n) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(n))
 #define ATT_REGS_INC() asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kAttRegsSoftmax))
   const uint32_t tmem = S->tmem_base;
   volatile int *abort = &S->abort;
@@ -251,7 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
 
   if (warp == kAttWarpResolve) {
     // ====================================================================== resolve (32 threads)
-    ATT_REGS_DEC();
+    ATT_REGS_DEC(kAttRegsMisc);
     // Chunk c of this pair: token positions -> physical rows (ring slot c % kAttRing, -1 = masked) and two
     // validity words; on entering a unit this CTA's 64 q rows are prefetched into L2.
     // The idx loads of chunk c + 1 are in flight while the block-table loads of chunk c resolve.
@@ -311,13 +309,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     }
   } else if (warp >= 4 && warp < 8) {
     // ====================================================================== gather (128 threads)
-    ATT_REGS_DEC();
+    ATT_REGS_DEC(kAttRegsGather);
     // Chunk c: this CTA's 32 tokens by TMA gather4 (4 rows x 128 bytes per instruction, 128-byte swizzle
     // applied by the copy engine), warp w taking dim blocks w, w+4 (and 8 for warp 0); q by one tiled TMA
     // per dim block when a unit starts.  The loop never breaks: after a timeout every wait returns at once
     // and the copies are skipped.
     const int t = threadIdx.x - 128, pw = t >> 5;
     const int oob_row = a.bv.num_blocks * 64;           // outside the map: the copy engine fills zeros
+    const uint32_t buf_full_r0 = tc::map_to_rank(tc::smem_u32(&S->buf_full[0]), 0);
+    const uint32_t q_full_r0 = tc::map_to_rank(tc::smem_u32(&S->q_full), 0);
     ChunkCursor pc;
     pc.seek(a, pair, npairs);
     uint32_t v = 0;
@@ -327,7 +327,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
       bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->phys_full[slot]), (c / kAttRing) & 1u, abort, status));
       if (lane == 0 && ok) {
         ok = tc::mbar_wait_cl(tc::smem_u32(&S->buf_empty[b]), (use & 1u) ^ 1u, abort, status);
-        if (ok) tc::mbar_expect_tx(tc::smem_u32(&S->buf_full[b]), (uint32_t)nblk * kAttBlkBytes);
+        // rank 0 expects the bytes of this warp's dim blocks from both CTAs
+        if (ok && rank == 0) tc::mbar_expect_tx(tc::smem_u32(&S->buf_full[b]), 2u * (uint32_t)nblk * kAttBlkBytes);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (ok && lane < kAttHalf / 4) {
@@ -337,8 +338,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         for (int e = 0; e < 4; ++e) r4[e] = ph[e] >= 0 ? ph[e] : oob_row;
         for (int m = 0; m < nblk; ++m) {
           const int d = pw + 4 * m;
-          tc::tma_gather4(tc::smem_u32(sBuf + b * kAttBufBytes + d * kAttBlkBytes + 4 * lane * 128), &tm_kv, d * 64, r4[0],
-                          r4[1], r4[2], r4[3], tc::smem_u32(&S->buf_full[b]));
+          tc::tma_gather4_pair(tc::smem_u32(sBuf + b * kAttBufBytes + d * kAttBlkBytes + 4 * lane * 128), &tm_kv, d * 64,
+                               r4[0], r4[1], r4[2], r4[3], buf_full_r0 + b * 8);
         }
       }
       __syncwarp();
@@ -347,10 +348,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         if (t == 0) {
           const bool okq = v == 0 || tc::mbar_wait_cl(tc::smem_u32(&S->q_empty), (v - 1) & 1u, abort, status);
           if (okq) {
-            const uint32_t bar = tc::smem_u32(&S->q_full);
-            tc::mbar_expect_tx(bar, kAttQBytes);
+            if (rank == 0) tc::mbar_expect_tx(tc::smem_u32(&S->q_full), 2u * kAttQBytes);
             for (int d = 0; d < 9; ++d)
-              tc::tma_load_2d(tc::smem_u32(sQ + d * 8192), &tm_q, d * 64, pc.row * kAttH + 64 * (int)rank, bar);
+              tc::tma_load_2d_pair(tc::smem_u32(sQ + d * 8192), &tm_q, d * 64, pc.row * kAttH + 64 * (int)rank, q_full_r0);
           }
         }
         ++v;
@@ -359,7 +359,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     }
   } else if (warp >= 8 && warp < 12) {
     // ====================================================================== cross (128 threads)
-    ATT_REGS_DEC();
+    ATT_REGS_DEC(kAttRegsCross);
     // Chunk c: the peer's 32 tokens' half of the values (rank 0 takes dims 0-255, rank 1 dims 256-511),
     // 16 bytes per load, a warp reading one 512-byte row segment per step, into registers; once QK^T of the
     // chunk has run they are stored with the 128-byte swizzle into the dim blocks it no longer needs
@@ -401,36 +401,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         __syncwarp();
         if (lane == 0) {
           if (rank == 0) tc::mbar_arrive(tc::smem_u32(&S->v_ready[b]));
-          else tc::mbar_arrive_cluster(v_ready_r0 + b * 8);
+          else tc::mbar_arrive_remote(v_ready_r0 + b * 8);
         }
-      }
-    }
-  } else if (warp == kAttWarpRelay) {
-    // ====================================================================== relay (lane 0)
-    ATT_REGS_DEC();
-    if (lane == 0) {
-      const uint32_t peer_pair_full = tc::map_to_rank(tc::smem_u32(&S->pair_full[0]), 0);
-      const uint32_t peer_pair_q = tc::map_to_rank(tc::smem_u32(&S->pair_q_full), 0);
-      uint32_t v = 0, c = 0;
-      bool ok = true;
-      for (int u = pair; u < U && ok; u += npairs) {
-        int row, cb, ce;
-        unit_of(a, u, &row, &cb, &ce);
-        const int nch = ce - cb;
-        if (nch <= 0) continue;
-        if (!tc::mbar_wait(tc::smem_u32(&S->q_full), v & 1u, abort, status)) break;
-        tc::mbar_arrive_cluster(peer_pair_q);
-        for (int i = 0; i < nch; ++i, ++c) {
-          const uint32_t b = c % kAttNBuf;
-          if (!tc::mbar_wait(tc::smem_u32(&S->buf_full[b]), (c / kAttNBuf) & 1u, abort, status)) { ok = false; break; }
-          tc::mbar_arrive_cluster(peer_pair_full + b * 8);
-        }
-        ++v;
       }
     }
   } else if (warp == kAttWarpMMA) {
     // ====================================================================== MMA issuer (rank 0, whole warp)
-    ATT_REGS_DEC();
+    ATT_REGS_DEC(kAttRegsMisc);
     // The warp runs the loop uniformly and one elected lane issues each MMA and commit.  Descriptors are a
     // base descriptor plus the byte offset / 16 (the address field cannot carry: shared memory < 256 KB).
     if (rank == 0) {
@@ -450,17 +427,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         if (first && v > 0 && !tc::mbar_wait_cl_w(tc::smem_u32(&S->o_empty), (v - 1) & 1u, abort, status)) return false;
         tc::fence_after_sync();
         const uint64_t pa = p_desc + ((pb * kAttPBytes) >> 4), vb = v_desc + ((b * kAttBufBytes) >> 4);
+        // per half p of the values: K steps of 16 tokens = kh (token half, 4 dim blocks apart) x ks (16 rows)
+        static_assert(kAttHalf == 32, "two 16-token steps per token half");
+        constexpr int kS = (16 * 128) >> 4, kH = (4 * kAttBlkBytes) >> 4;
 #pragma unroll
         for (int p = 0; p < 2; ++p)
-#pragma unroll
-          for (int kh = 0; kh < 2; ++kh)
-#pragma unroll
-            for (int ks = 0; ks < kAttHalf / 16; ++ks) {
-              const int kg = (kAttHalf / 16) * kh + ks;          // 16-token step within the chunk
-              tc::mma_bf16_pair_w(tmem + kTmemO + 128 * p, pa + ((kg * 32) >> 4),
-                                  vb + (((4 * kh + 2 * p) * kAttBlkBytes + ks * 2048) >> 4), idesc_pv,
-                                  (first && kg == 0) ? 0u : 1u);
-            }
+          tc::mma_bf16_pair_x4_w<kS, kH, kH + kS>(tmem + kTmemO + 128 * p, pa, vb + ((2 * p * kAttBlkBytes) >> 4), idesc_pv,
+                                                  first ? 0u : 1u);
         tc::mma_commit_pair_w(tc::smem_u32(&S->buf_empty[b]), both);
         tc::mma_commit_pair_w(tc::smem_u32(&S->pv_done[pb]), both);
         return true;
@@ -470,22 +443,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         unit_of(a, u, &row, &cb, &ce);
         const int nch = ce - cb;
         if (nch <= 0) continue;
-        if (!tc::mbar_wait_cl_w(tc::smem_u32(&S->pair_q_full), v & 1u, abort, status)) break;
+        if (!tc::mbar_wait_cl_w(tc::smem_u32(&S->q_full), v & 1u, abort, status)) break;
         tc::fence_after_sync();
         const uint32_t c0 = c;
         for (int i = 0; i < nch; ++i) {
           const uint32_t b = c % kAttNBuf;
-          if (!tc::mbar_wait_cl_w(tc::smem_u32(&S->pair_full[b]), (c / kAttNBuf) & 1u, abort, status)) { ok = false; break; }
+          if (!tc::mbar_wait_cl_w(tc::smem_u32(&S->buf_full[b]), (c / kAttNBuf) & 1u, abort, status)) { ok = false; break; }
           tc::fence_after_sync();
           const uint64_t kb = kv_desc + ((b * kAttBufBytes) >> 4);
           const uint32_t sb = tmem + kTmemS + kAttHalf * (c & 1u);
 #pragma unroll 1
-          for (int d = 0; d < 9; ++d) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              tc::mma_bf16_pair_w(sb, q_desc + ((d * 8192 + kk * 32) >> 4), kb + ((d * kAttBlkBytes + kk * 32) >> 4),
-                                  idesc_qk, (d == 0 && kk == 0) ? 0u : 1u);
-          }
+          for (int d = 0; d < 9; ++d)
+            tc::mma_bf16_pair_x4_w<2, 4, 6>(sb, q_desc + ((d * 8192) >> 4), kb + ((d * kAttBlkBytes) >> 4), idesc_qk,
+                                            d == 0 ? 0u : 1u);
           tc::mma_commit_pair_w(tc::smem_u32(&S->s_full[c & 1u]), both);
           if (i == nch - 1) tc::mma_commit_pair_w(tc::smem_u32(&S->q_empty), both);
           ++c;
@@ -499,7 +469,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
       __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->drain), 0, &no_abort, status));
     }
   } else if (warp >= 4) {
-    ATT_REGS_DEC();                            // the spare warp of the last warpgroup
+    ATT_REGS_DEC(kAttRegsMisc);                // the spare warps of the last warpgroup
   } else {
     // ====================================================================== softmax + epilogue (warps 0-3)
     ATT_REGS_INC();
@@ -616,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
         __syncwarp();
         if (lane == 0) {
           if (rank == 0) tc::mbar_arrive(tc::smem_u32(&S->p_full[c & 1u]));
-          else tc::mbar_arrive_cluster(p_full_r0 + (c & 1u) * 8);
+          else tc::mbar_arrive_remote(p_full_r0 + (c & 1u) * 8);
         }
       }
       // ---- epilogue: wait for the last P V, normalise, store through a per-warp staging tile
@@ -678,7 +648,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive_cluster(o_empty_r0);
+      if (lane == 0) {
+        if (rank == 0) tc::mbar_arrive(tc::smem_u32(&S->o_empty));
+        else tc::mbar_arrive_remote(o_empty_r0);
+      }
     }
   }
 

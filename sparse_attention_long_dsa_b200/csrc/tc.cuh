@@ -266,6 +266,14 @@ __device__ __forceinline__ bool mbar_wait_cl(uint32_t bar, uint32_t parity, vola
   }
 }
 
+// 16-byte asynchronous store into the shared memory of another CTA of the cluster; the bytes are counted on
+// `remote_bar` (a barrier in the destination CTA) when they have landed.
+__device__ __forceinline__ void st_async16(uint32_t remote_addr, const uint4 &v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+               ::"r"(remote_addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar)
+               : "memory");
+}
+
 // ------------------------------------------------------------------------------------------ cp.async
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -348,6 +356,57 @@ __device__ __forceinline__ void mma_bf16_pair_x4_w(uint32_t d_tmem, uint64_t a_d
       "@e tcgen05.mma.cta_group::2.kind::f16 [%0], a2, b2, %3, t;\n\t"
       "@e tcgen05.mma.cta_group::2.kind::f16 [%0], a3, b3, %3, t;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(B1), "n"(B2), "n"(B3)
+      : "memory");
+}
+// The 36 MMAs of a QK^T chunk (9 dim blocks x 4 K steps) in one block issued by one elected lane: A (q)
+// advances 8192 bytes per dim block, B (the chunk buffer) kBBlk bytes, both 32 bytes per K step; the
+// first MMA starts a fresh accumulator, the rest accumulate.  Descriptor offsets are immediates (bytes/16).
+template <int kBBlk>
+__device__ __forceinline__ void mma_qk36_pair_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
+  static_assert(kBBlk == 4096, "immediates below assume 4 KB dim blocks");
+  asm volatile(
+      "{\n\t.reg .pred e, t, f;\n\t.reg .b64 ra, rb;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "setp.ne.b32 f, 0, 0;\n\t"
+      "add.u64 ra, %1, 0;\n\tadd.u64 rb, %2, 0;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, f;\n\t"
+      "add.u64 ra, %1, 2;\n\tadd.u64 rb, %2, 2;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 4;\n\tadd.u64 rb, %2, 4;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 6;\n\tadd.u64 rb, %2, 6;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 512;\n\tadd.u64 rb, %2, 256;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 514;\n\tadd.u64 rb, %2, 258;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 516;\n\tadd.u64 rb, %2, 260;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 518;\n\tadd.u64 rb, %2, 262;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 1024;\n\tadd.u64 rb, %2, 512;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 1026;\n\tadd.u64 rb, %2, 514;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 1028;\n\tadd.u64 rb, %2, 516;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 1030;\n\tadd.u64 rb, %2, 518;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 1536;\n\tadd.u64 rb, %2, 768;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 1538;\n\tadd.u64 rb, %2, 770;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 1540;\n\tadd.u64 rb, %2, 772;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 1542;\n\tadd.u64 rb, %2, 774;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 2048;\n\tadd.u64 rb, %2, 1024;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 2050;\n\tadd.u64 rb, %2, 1026;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 2052;\n\tadd.u64 rb, %2, 1028;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 2054;\n\tadd.u64 rb, %2, 1030;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 2560;\n\tadd.u64 rb, %2, 1280;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 2562;\n\tadd.u64 rb, %2, 1282;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 2564;\n\tadd.u64 rb, %2, 1284;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 2566;\n\tadd.u64 rb, %2, 1286;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 3072;\n\tadd.u64 rb, %2, 1536;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 3074;\n\tadd.u64 rb, %2, 1538;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 3076;\n\tadd.u64 rb, %2, 1540;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 3078;\n\tadd.u64 rb, %2, 1542;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 3584;\n\tadd.u64 rb, %2, 1792;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 3586;\n\tadd.u64 rb, %2, 1794;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 3588;\n\tadd.u64 rb, %2, 1796;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 3590;\n\tadd.u64 rb, %2, 1798;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 4096;\n\tadd.u64 rb, %2, 2048;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 4098;\n\tadd.u64 rb, %2, 2050;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 4100;\n\tadd.u64 rb, %2, 2052;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "add.u64 ra, %1, 4102;\n\tadd.u64 rb, %2, 2054;\n\t@e tcgen05.mma.cta_group::2.kind::f16 [%0], ra, rb, %3, t;\n\t"
+      "}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc)
       : "memory");
 }
 __device__ __forceinline__ void mma_commit_pair_w(uint32_t bar, uint16_t cta_mask) {

@@ -144,52 +144,67 @@ struct ChunkCursor {
 
 // ------------------------------------------------------------------------------------------------ plan
 // neff[row] = 1 + largest j with a usable idx[row, j] (0 if none); flags positions outside [0, seq_len).
-// One warp per row; every lane reads 16-byte vectors, all of them issued before any is used.
-__global__ void attn_plan_kernel(const int32_t *__restrict__ idx, int k, BatchView bv, int T, int32_t *neff,
-                                 uint32_t *status) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= T) return;
+// One 256-thread CTA per row; every thread reads 16-byte vectors, all of them issued before any is used.
+constexpr int kAttPlanThreads = 256;
+__global__ void __launch_bounds__(kAttPlanThreads) attn_plan_kernel(const int32_t *__restrict__ idx, int k, BatchView bv,
+                                                                   int T, int32_t *neff, uint32_t *status) {
+  __shared__ int s_last[kAttPlanThreads / 32];
+  __shared__ int s_bad[kAttPlanThreads / 32];
+  pdl_wait();
+  pdl_trigger();
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int b;
-  pos_of_row(bv, warp, &b);
+  pos_of_row(bv, row, &b);
   const int seq_len = __ldg(bv.seq_lens + b);
   int last = -1;
   bool bad = false;
-  const int32_t *ir = idx + (int64_t)warp * k;
+  const int32_t *ir = idx + (int64_t)row * k;
   const bool vec = (k & 3) == 0 && (((uintptr_t)ir) & 15) == 0;
   if (vec) {
     const int k4 = k >> 2;
-    for (int base = 0; base < k4; base += 32 * 8) {
-      int4 v[8];
+    for (int base = 0; base < k4; base += kAttPlanThreads * 4) {
+      int4 v[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int j4 = base + e * 32 + lane;
+      for (int e = 0; e < 4; ++e) {
+        const int j4 = base + e * kAttPlanThreads + tid;
         v[e] = j4 < k4 ? __ldg(reinterpret_cast<const int4 *>(ir) + j4) : make_int4(-1, -1, -1, -1);
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int j = 4 * (base + e * 32 + lane);
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * (base + e * kAttPlanThreads + tid);
         const int vals[4] = {v[e].x, v[e].y, v[e].z, v[e].w};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (vals[c] >= 0 && vals[c] < seq_len) last = max(last, j + c);
-          else if (vals[c] >= seq_len) bad = true;
+        for (int q = 0; q < 4; ++q) {
+          if (vals[q] >= 0 && vals[q] < seq_len) last = max(last, j + q);
+          else if (vals[q] >= seq_len) bad = true;
         }
       }
     }
   } else {
-    for (int j = lane; j < k; j += 32) {
-      const int s = __ldg(ir + j);
-      if (s >= 0 && s < seq_len) last = j;
-      else if (s >= seq_len) bad = true;
+    for (int j = tid; j < k; j += kAttPlanThreads) {
+      const int sj = __ldg(ir + j);
+      if (sj >= 0 && sj < seq_len) last = j;
+      else if (sj >= seq_len) bad = true;
     }
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
   bad = __any_sync(0xffffffffu, bad);
   if (lane == 0) {
-    neff[warp] = last + 1;
-    if (bad) set_status(status, kStatusBadIndex);
+    s_last[warp] = last;
+    s_bad[warp] = bad;
   }
+  __syncthreads();
+  if (tid == 0) {
+    int m = -1, any = 0;
+    for (int w = 0; w < kAttPlanThreads / 32; ++w) {
+      m = max(m, s_last[w]);
+      any |= s_bad[w];
+    }
+    neff[row] = m + 1;
+    if (any) set_status(status, kStatusBadIndex);
+  }
+  (void)T;
 }
 
 // ------------------------------------------------------------------------------------------------ main
@@ -250,6 +265,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
   const uint32_t tmem = S->tmem_base;
   volatile int *abort = &S->abort;
   uint32_t *status = a.status;
+  // inputs (q, idx, neff, the cache) come from earlier work on the stream
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == kAttWarpResolve) {
     // ====================================================================== resolve (32 threads)
@@ -671,6 +689,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restrict__ part_o,
                                                            const float *__restrict__ part_lse, int splits,
                                                            __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x, h = blockIdx.y;
   float mx = -INFINITY;
   for (int s = 0; s < splits; ++s) mx = fmaxf(mx, __ldg(part_lse + ((int64_t)row * splits + s) * kAttH + h));
@@ -776,8 +796,8 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
     set_error("attention: cuTensorMapEncodeTiled failed");
     return DSA_ERR_CUDA;
   }
-  attn_plan_kernel<<<(a.T + 3) / 4, 128, 0, stream>>>(idx, k, a.bv, a.T, neff, a.status);
-  DSA_LAUNCH_CHECK("attn_plan_kernel");
+  DSA_LAUNCH_PDL("attn_plan_kernel", attn_plan_kernel, dim3(a.T), dim3(kAttPlanThreads), 0, stream, idx, k, a.bv, a.T,
+                 neff, a.status);
   const size_t smem = attn_smem_bytes();
   cudaFuncSetAttribute(attn_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   // persistent grid: as many CTA pairs as can be resident at once
@@ -804,12 +824,10 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
   }
   const int units = a.T * a.splits;
   const int pairs = std::min(max_pairs, units);
-  attn_mla_kernel<<<2 * pairs, kAttThreads, smem, stream>>>(tm_q, tm_kv, a);
-  DSA_LAUNCH_CHECK("attn_mla_kernel");
+  DSA_LAUNCH_PDL("attn_mla_kernel", attn_mla_kernel, dim3(2 * pairs), dim3(kAttThreads), smem, stream, tm_q, tm_kv, a);
   if (a.splits > 1) {
-    attn_combine_kernel<<<dim3(a.T, kAttH), 128, 0, stream>>>(a.part_o, a.part_lse, a.splits, (__nv_bfloat16 *)out,
-                                                               lse);
-    DSA_LAUNCH_CHECK("attn_combine_kernel");
+    DSA_LAUNCH_PDL("attn_combine_kernel", attn_combine_kernel, dim3(a.T, kAttH), dim3(128), 0, stream,
+                   (const float *)a.part_o, (const float *)a.part_lse, a.splits, (__nv_bfloat16 *)out, lse);
   }
   return DSA_OK;
 }

@@ -62,6 +62,13 @@ __device__ __forceinline__ int64_t phys_row(const BatchView &bv, int b, int s) {
   return (int64_t)blk * bv.page_size + (s % bv.page_size);
 }
 
+// Programmatic dependent launch: every kernel of the path is launched so that it may start while the
+// previous kernel of the stream finishes.  pdl_wait() blocks until the previous grid has completed and its
+// memory is visible, and must precede every global-memory access of the kernel (reads of inputs that the
+// previous kernel may produce, writes that it may still read); pdl_trigger() lets the next kernel launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // fp32 -> unsigned key whose integer order is the float order (-0 folded onto +0)
 __device__ __forceinline__ uint32_t ordered_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -115,6 +122,37 @@ namespace dsa {
 void set_error(const char *fmt, ...);
 void count_launch();
 }
+
+#include <utility>
+namespace dsa {
+// launch with programmatic stream serialization (see pdl_wait / pdl_trigger)
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+}  // namespace dsa
+
+// launch a kernel with launch_pdl and fail the calling entry point on a launch error
+#define DSA_LAUNCH_PDL(what, kernel, grid, block, smem, stream, ...)                    \
+  do {                                                                                   \
+    cudaError_t le_ = ::dsa::launch_pdl(kernel, grid, block, smem, stream, __VA_ARGS__); \
+    if (le_ != cudaSuccess) {                                                            \
+      ::dsa::set_error("%s: %s", what, cudaGetErrorString(le_));                         \
+      return DSA_ERR_CUDA;                                                               \
+    }                                                                                    \
+    DSA_LAUNCH_CHECK(what);                                                              \
+  } while (0)
 
 #define DSA_LAUNCH_CHECK(what)                                                 \
   do {                                                                         \

@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(1024) indexer_plan_kernel(BatchView bv, IdxPla
   __shared__ uint32_t tmp[64];
   __shared__ uint32_t s_carry;
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (tid == 0) s_carry = 0;
   __syncthreads();
   // groups per sequence -> seq_goff (exclusive prefix)
@@ -165,9 +167,6 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   IdxSmem *S = (IdxSmem *)(sKS + kIdxStages * kIdxTile);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = pv.hdr[0], U = pv.hdr[1];
-  const int u0 = (int)(((int64_t)blockIdx.x * U) / gridDim.x);
-  const int u1 = (int)(((int64_t)(blockIdx.x + 1) * U) / gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kIdxStages; ++i) {
@@ -195,6 +194,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   tc::fence_after_sync();
   const uint32_t tmem = S->tmem_base;
   volatile int *abort = &S->abort;
+  // the plan (and the inputs) come from earlier work on the stream
+  pdl_wait();
+  pdl_trigger();
+  const int G = pv.hdr[0], U = pv.hdr[1];
+  const int u0 = (int)(((int64_t)blockIdx.x * U) / gridDim.x);
+  const int u1 = (int)(((int64_t)(blockIdx.x + 1) * U) / gridDim.x);
 
   if (u0 < u1) {
     if (warp == 0 || warp >= 6) {
@@ -468,13 +473,11 @@ dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t 
     set_error("indexer: cuTensorMapEncodeTiled failed");
     return DSA_ERR_CUDA;
   }
-  indexer_plan_kernel<<<1, 1024, 0, stream>>>(bv, pv);
-  DSA_LAUNCH_CHECK("indexer_plan_kernel");
+  DSA_LAUNCH_PDL("indexer_plan_kernel", indexer_plan_kernel, dim3(1), dim3(1024), 0, stream, bv, pv);
   const size_t smem = indexer_tc_smem();
   cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  indexer_tc_kernel<<<num_sms, kIdxThreads, smem, stream>>>(tm_k, tm_q, kscale, w, bv, pv, scores, ld,
-                                                             (uint32_t *)ws);
-  DSA_LAUNCH_CHECK("indexer_tc_kernel");
+  DSA_LAUNCH_PDL("indexer_tc_kernel", indexer_tc_kernel, dim3(num_sms), dim3(kIdxThreads), smem, stream, tm_k, tm_q,
+                 kscale, w, bv, pv, scores, ld, (uint32_t *)ws);
   return DSA_OK;
 }
 

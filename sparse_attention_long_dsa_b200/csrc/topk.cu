@@ -105,6 +105,8 @@ __device__ void find_threshold_bin(const uint32_t *hist, int nbins, uint32_t k_r
 __global__ void __launch_bounds__(kTopkThreadsA)
 topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, int k,
                       int32_t *__restrict__ idx, TopkWs lw, int register_long) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint32_t sm[];
   uint32_t *keys = sm;
   uint32_t *hist = sm + kTopkSmemCap;
@@ -219,6 +221,8 @@ __device__ int stage_segment(const float *__restrict__ scores, int64_t ld, int r
 
 __global__ void __launch_bounds__(kTopkThreadsB)
 topk_long_hist_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, TopkWs w, int pass) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ __align__(16) uint32_t keys[kTopkSeg];
   __shared__ uint32_t hist[kRadixBins];
   __shared__ uint32_t tmp[64];
@@ -269,6 +273,8 @@ topk_long_hist_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
 
 __global__ void __launch_bounds__(kTopkThreadsB)
 topk_long_count_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, TopkWs w) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ __align__(16) uint32_t keys[kTopkSeg];
   __shared__ uint32_t tmp[64];
   const int items = (int)(*w.count) * w.max_segs;
@@ -293,6 +299,8 @@ topk_long_count_kernel(const float *__restrict__ scores, int64_t ld, BatchView b
 __global__ void __launch_bounds__(kTopkThreadsB)
 topk_long_write_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, TopkWs w, int k,
                        int32_t *__restrict__ idx) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ __align__(16) uint32_t keys[kTopkSeg];
   __shared__ uint32_t tmp[64];
   __shared__ uint32_t s_gt_before, s_eq_before;
@@ -357,18 +365,18 @@ dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, 
   }
   const size_t smem = (size_t)(kTopkSmemCap + kRadixBins + 64) * 4;
   cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  topk_rows_smem_kernel<<<b->total_q, kTopkThreadsA, smem, stream>>>(scores, ld, bv, k, idx, lw, has_long ? 1 : 0);
-  DSA_LAUNCH_CHECK("topk_rows_smem_kernel");
+  DSA_LAUNCH_PDL("topk_rows_smem_kernel", topk_rows_smem_kernel, dim3(b->total_q), dim3(kTopkThreadsA), smem, stream,
+                 scores, ld, bv, k, idx, lw, has_long ? 1 : 0);
   if (has_long) {
     const int grid = max(num_sms * 4, topk_max_segs(b->max_seq_len));   // one segment per CTA per row
     for (int pass = 0; pass < 3; ++pass) {
-      topk_long_hist_kernel<<<grid, kTopkThreadsB, 0, stream>>>(scores, ld, bv, lw, pass);
-      DSA_LAUNCH_CHECK("topk_long_hist_kernel");
+      DSA_LAUNCH_PDL("topk_long_hist_kernel", topk_long_hist_kernel, dim3(grid), dim3(kTopkThreadsB), 0, stream, scores,
+                     ld, bv, lw, pass);
     }
-    topk_long_count_kernel<<<grid, kTopkThreadsB, 0, stream>>>(scores, ld, bv, lw);
-    DSA_LAUNCH_CHECK("topk_long_count_kernel");
-    topk_long_write_kernel<<<grid, kTopkThreadsB, 0, stream>>>(scores, ld, bv, lw, k, idx);
-    DSA_LAUNCH_CHECK("topk_long_write_kernel");
+    DSA_LAUNCH_PDL("topk_long_count_kernel", topk_long_count_kernel, dim3(grid), dim3(kTopkThreadsB), 0, stream, scores,
+                   ld, bv, lw);
+    DSA_LAUNCH_PDL("topk_long_write_kernel", topk_long_write_kernel, dim3(grid), dim3(kTopkThreadsB), 0, stream, scores,
+                   ld, bv, lw, k, idx);
   }
   return DSA_OK;
 }

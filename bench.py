@@ -250,6 +250,26 @@ def workload_config(wl, args):
     return d
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum per launch) of the dominant kernel from one
+# ncu capture (profiles/), valid only while the kernel's sources are the ones that were captured.
+MEASURED_TRAFFIC = {
+    ("attention", "decode_batch"): {"bytes": 84244736 + 3541248,
+                                    "sources": ("attn_mla_tc.cu", "tc.cuh", "common.cuh"), "sha256_16": "2d3feb2eec1e9655"},
+}
+
+
+def measured_traffic(stage, workload):
+    import hashlib
+    rec = MEASURED_TRAFFIC.get((stage, workload))
+    if rec is None:
+        return None
+    m = hashlib.sha256()
+    for f in rec["sources"]:
+        with open(os.path.join(ROOT, "sparse_attention_long_dsa_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    return rec["bytes"] if m.hexdigest()[:16] == rec["sha256_16"] else None
+
+
 def roofline_entry(stage, ms, work, peaks, src, args, decode):
     """Decode stages are HBM-bound (bytes / HBM copy bandwidth); prefill attention and indexer are
     tensor-bound (flops / dense peak: bf16 for attention, 2x bf16 for the FP8 indexer)."""
@@ -261,13 +281,15 @@ def roofline_entry(stage, ms, work, peaks, src, args, decode):
         peak = peaks["hbm_gbs"]
         return {"kernel": stage, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "peak_source": f"{tag} hbm_gbs", "algorithmic_bytes_per_launch": w["bytes"],
-                "avg_launch_ms": ms, "traffic": None, "tflops": w["flops"] / secs / 1e12}
+                "avg_launch_ms": ms, "traffic": measured_traffic(stage, args.workload),
+                "tflops": w["flops"] / secs / 1e12}
     ach = w["flops"] / secs / 1e12
     fp8 = stage == "indexer"
     peak = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
     return {"kernel": stage, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
             "peak_source": f"{tag} bf16_tflops_sustained" + (" x2 (fp8 = 2x bf16 dense ratio)" if fp8 else ""),
-            "algorithmic_flops_per_launch": w["flops"], "avg_launch_ms": ms, "traffic": None,
+            "algorithmic_flops_per_launch": w["flops"], "avg_launch_ms": ms,
+            "traffic": measured_traffic(stage, args.workload),
             "gbs": w["bytes"] / secs / 1e9}
 
 

@@ -16,12 +16,12 @@
 //              of three chunk buffers [9 dim blocks][32 tokens][128 B] (128-byte swizzle), by TMA gather4;
 //   * QK^T   : M = 128 heads (rank r holds heads 64r..64r+63 of q), N = 64 tokens (32 from each CTA),
 //              K = 576; each CTA gets S for its 64 heads x all 64 tokens in TMEM;
-//   * swap   : the values each CTA needs for P V are 256 of the 512 value dims of all 64 tokens; its own
-//              tokens already hold them, the peer's tokens' half (16 KB) sits in the peer's buffer.  Once QK^T
-//              has run, four swap warps per CTA read the half the PEER needs (rank 0: its blocks 4-7 = dims
-//              256-511 of its tokens; rank 1: its blocks 0-3 = dims 0-255) into registers, hand-shake, and
-//              push them with st.async into the same blocks of the peer, completing on the peer's barrier:
-//              an in-place exchange through distributed shared memory, every row read from HBM once per pair;
+//   * cross  : the values each CTA needs for P V are 256 of the 512 value dims of all 64 tokens; its own
+//              tokens already hold them, the peer's 32 tokens' half (16 KB, which the peer's copy engine pulls
+//              through L2 at the same time) is loaded into registers by four warps a chunk ahead and stored
+//              into the dim blocks QK^T no longer needs once it has run (rank 0: blocks 4-7 <- dims 0-255 of
+//              rank 1's tokens; rank 1: blocks 0-3 <- dims 256-511 of rank 0's tokens).  HBM carries each row
+//              once per pair (the peer's half is an L2 hit); each CTA writes only its own shared memory;
 //   * softmax: 4 warps per CTA, one (head, 32-token half) per thread, running max shared with the partner
 //              thread, exp2, P (bf16) into one of two P buffers; O is rescaled in TMEM only when the
 //              running max grows by more than 2^8 (exact: the final division uses the same reference max);
@@ -60,9 +60,7 @@ constexpr float kRescaleLog2 = 8.0f;
 struct AttSmem {
   uint64_t buf_full[kAttNBuf];      // rank 0: TMA bytes of both CTAs' halves of a chunk (4 gather warps expect)
   uint64_t buf_empty[kAttNBuf];     // MMA commit to both CTAs after P V of the chunk
-  uint64_t v_ready[kAttNBuf];       // rank 0: 8 swap warps (both CTAs) have the peer's values in place
-  uint64_t region_free;             // the peer's 4 swap warps hold their send half in registers
-  uint64_t v_arrived;               // the peer's 16 KB landed (st.async bytes; one local expect_tx)
+  uint64_t v_ready[kAttNBuf];       // rank 0: 8 cross warps (both CTAs) stored the peer's values
   uint64_t q_full, q_empty;         // q_full: rank 0, both CTAs' q bytes
   uint64_t s_full[2];               // MMA commit to both CTAs
   uint64_t p_full[2];               // rank 0: 8 softmax warps wrote P
@@ -236,12 +234,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     tc::mbar_init(tc::smem_u32(&S->q_full), 1);
     tc::mbar_init(tc::smem_u32(&S->q_empty), 1);
     tc::mbar_init(tc::smem_u32(&S->o_empty), 8);
-    tc::mbar_init(tc::smem_u32(&S->region_free), 4);
-    tc::mbar_init(tc::smem_u32(&S->v_arrived), 1);
     tc::mbar_init(tc::smem_u32(&S->drain), 1);
     for (int i = 0; i < kAttRing; ++i) {
       tc::mbar_init(tc::smem_u32(&S->phys_full[i]), 1);
-      tc::mbar_init(tc::smem_u32(&S->phys_empty[i]), 4);
+      tc::mbar_init(tc::smem_u32(&S->phys_empty[i]), 8);
       tc::mbar_init(tc::smem_u32(&S->mask_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&S->mask_empty[i]), 4);
     }
@@ -380,43 +376,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
       pc.next(a, npairs);
     }
   } else if (warp >= 8 && warp < 12) {
-    // ====================================================================== swap (128 threads)
-    // Chunk c, after QK^T: this CTA's send half (rank 0: blocks 4-7, rank 1: blocks 0-3 of its buffer) into
-    // registers; tell the peer this region may be overwritten; once the peer has done the same, push the
-    // registers into the peer's matching region (the other half of its blocks 0-7) by st.async, and wait for
-    // the peer's 16 KB to land in this CTA's region.  Loops never break: after a timeout the waits return
-    // at once and the copies are skipped.
+    // ====================================================================== cross (128 threads)
     ATT_REGS_DEC(kAttRegsCross);
+    // Chunk c: the peer's 32 tokens' half of the values (rank 0 takes dims 0-255, rank 1 dims 256-511),
+    // 16 bytes per load, a warp reading one 512-byte row segment per step, into registers; once QK^T of the
+    // chunk has run they are stored with the 128-byte swizzle into the dim blocks it no longer needs
+    // (rank 0: 4-7, rank 1: 0-3).  Masked tokens store zeros.
     const int t = threadIdx.x - 256;
-    const uint32_t own_off = (rank == 0 ? 4u : 0u) * kAttBlkBytes, peer_off = (rank == 0 ? 0u : 4u) * kAttBlkBytes;
-    constexpr int kSwapVec = 4 * kAttBlkBytes / 16 / 128;       // 16-byte pieces per thread
-    const uint32_t peer_buf = tc::map_to_rank(tc::smem_u32(sBuf), rank ^ 1u);
-    const uint32_t peer_region_free = tc::map_to_rank(tc::smem_u32(&S->region_free), rank ^ 1u);
-    const uint32_t peer_v_arrived = tc::map_to_rank(tc::smem_u32(&S->v_arrived), rank ^ 1u);
+    const uint32_t dst_blk0 = rank == 0 ? 4u : 0u;
+    const int dim0 = rank == 0 ? 0 : 256;
+    constexpr int kCrossVec = 4 * kAttBlkBytes / 16 / 128;      // 16-byte loads per thread
     const uint32_t v_ready_r0 = tc::map_to_rank(tc::smem_u32(&S->v_ready[0]), 0);
     uint32_t c = 0;
     for (int u = pair; u < U; u += npairs) {
       int row, cb, ce;
       unit_of(a, u, &row, &cb, &ce);
       for (int i = 0; i < ce - cb; ++i, ++c) {
-        const uint32_t b = c % kAttNBuf;
-        // QK^T of the chunk has read both buffers
-        const bool have = __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->s_full[c & 1u]), (c >> 1) & 1u, abort, status));
-        const uint8_t *src = sBuf + b * kAttBufBytes + own_off;
-        uint4 val[kSwapVec];
+        const uint32_t b = c % kAttNBuf, slot = c % kAttRing;
+        const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->phys_full[slot]), (c / kAttRing) & 1u, abort, status));
+        const int32_t *ph = S->phys[slot] + kAttHalf * (int)(rank ^ 1u);
+        uint4 val[kCrossVec];
 #pragma unroll
-        for (int m = 0; m < kSwapVec; ++m) val[m] = *reinterpret_cast<const uint4 *>(src + (t + 128 * m) * 16);
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive_remote(peer_region_free);
-        if (t == 0) tc::mbar_expect_tx(tc::smem_u32(&S->v_arrived), 4 * kAttBlkBytes);
-        const bool ok = __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->region_free), c & 1u, abort, status));
-        if (have && ok) {
-          const uint32_t dst = peer_buf + b * kAttBufBytes + peer_off;
-#pragma unroll
-          for (int m = 0; m < kSwapVec; ++m) tc::st_async16(dst + (t + 128 * m) * 16, val[m], peer_v_arrived);
+        for (int m = 0; m < kCrossVec; ++m) {
+          const int idx = t + 128 * m, r = idx >> 5, cq = idx & 31;
+          const int pr = ph[r];
+          val[m] = (ok && pr >= 0) ? __ldg(reinterpret_cast<const uint4 *>(a.kv + (int64_t)pr * kAttD + dim0 + cq * 8))
+                                   : make_uint4(0, 0, 0, 0);
         }
-        const bool got = __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->v_arrived), c & 1u, abort, status));
-        (void)got;
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->phys_empty[slot]));
+        // QK^T of the chunk has read this CTA's buffer
+        const bool have = __all_sync(0xffffffffu, tc::mbar_wait_cl(tc::smem_u32(&S->s_full[c & 1u]), (c >> 1) & 1u, abort, status));
+        if (have) {
+          uint8_t *base = sBuf + b * kAttBufBytes + dst_blk0 * kAttBlkBytes;
+#pragma unroll
+          for (int m = 0; m < kCrossVec; ++m) {
+            const int idx = t + 128 * m, r = idx >> 5, cq = idx & 31;
+            *reinterpret_cast<uint4 *>(base + (cq >> 3) * kAttBlkBytes + r * 128 + (((cq & 7) ^ (r & 7)) << 4)) = val[m];
+          }
+        }
         tc::fence_proxy_async();
         __syncwarp();
         if (lane == 0) {

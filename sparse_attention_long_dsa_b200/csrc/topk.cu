@@ -11,13 +11,17 @@
 // Day-0 Adaptation of Million-Token Context Models on Domestic AI Chips", Four Key Layers 1).
 //
 // Two regimes:
-//   A) n <= kTopkSmemCap candidates: one CTA per row, the row's keys staged once in shared memory,
-//      all digit passes and the ordered write from shared memory.  One launch.
+//   A) n <= C * kTopkSmemCap candidates: a cluster of C CTAs per row (C = 1, 2, 4 or 8, more when there
+//      are few rows, so that the rows fill the GPU), each CTA staging one contiguous slice of the row in
+//      shared memory.  Every digit pass builds slice histograms, which each CTA sums over the cluster
+//      through distributed shared memory to the same row histogram; the ordered write offsets each
+//      slice by the counts of the slices before it.  One launch.
 //   B) longer rows (a million-token decode): the row is split into segments of kTopkSeg keys over
 //      a persistent grid; each digit pass is one launch whose CTAs add segment histograms into a
 //      per-row global histogram, and the last CTA of a row to finish (atomic counter, no waiting)
 //      picks the digit.  Then a count launch and an ordered-write launch.  No CTA ever waits for
 //      another.
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -102,27 +106,56 @@ __device__ void find_threshold_bin(const uint32_t *hist, int nbins, uint32_t k_r
 // ------------------------------------------------------------------------------------------------
 // Regime A
 // ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cl_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cl_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cl_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// u32 at the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t cl_ld(const void *p, uint32_t rank) {
+  uint32_t a = (uint32_t)__cvta_generic_to_shared(p), ra, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+// shared memory of a regime-A CTA: two slice histograms (alternating passes), the row histogram, scan
+// scratch, the slice's counts, then the slice's keys
+constexpr int kTopkSmemFixedU32 = 3 * kRadixBins + 64 + 4;
+
 __global__ void __launch_bounds__(kTopkThreadsA)
 topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, int k,
                       int32_t *__restrict__ idx, TopkWs lw, int register_long) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) uint32_t sm[];
-  uint32_t *keys = sm;
-  uint32_t *hist = sm + kTopkSmemCap;
-  uint32_t *tmp = hist + kRadixBins;
+  uint32_t *hist_s[2] = {sm, sm + kRadixBins};          // this slice, even / odd passes
+  uint32_t *ghist = sm + 2 * kRadixBins;                 // the row (sum over the cluster)
+  uint32_t *tmp = sm + 3 * kRadixBins;
+  uint32_t *cnt = tmp + 64;                              // [0] keys > T, [1] keys == T in this slice
+  uint32_t *keys = sm + kTopkSmemFixedU32;
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
 
-  const int row = blockIdx.x;
+  const uint32_t C = cl_size(), r = cl_rank();
+  const int row = blockIdx.x / (int)C;
   const int tid = threadIdx.x, bs = blockDim.x;
   int b;
   const int n = pos_of_row(bv, row, &b) + 1;
   int32_t *out = idx + (int64_t)row * k;
 
-  if (n > kTopkSmemCap) {
+  // (every branch below depends on n only, so all CTAs of a cluster take it together)
+  if (n > (int)C * kTopkSmemCap) {
     // long row: hand it to regime B, initialise its state and histogram
-    if (register_long) {
+    if (register_long && r == 0) {
       if (tid == 0) {
         uint32_t slot = atomicAdd(lw.count, 1u);
         lw.list[slot] = row;
@@ -133,19 +166,23 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
     return;
   }
   if (n <= k) {
-    for (int j = tid; j < k; j += bs) out[j] = j < n ? j : -1;
+    if (r == 0)
+      for (int j = tid; j < k; j += bs) out[j] = j < n ? j : -1;
     return;
   }
 
-  const float *src = scores + (int64_t)row * ld;
-  const int n4 = n >> 2;
+  // this CTA's slice [lo, lo + m): a multiple of 4 keys long, so 16-byte loads stay aligned
+  const int slice = ((n + (int)C - 1) / (int)C + 3) & ~3;
+  const int lo = min(n, (int)r * slice), m = min(n, lo + slice) - lo;
+  const float *src = scores + (int64_t)row * ld + lo;
+  const int m4 = m >> 2;
   const float4 *src4 = reinterpret_cast<const float4 *>(src);
-  for (int i = tid; i < n4; i += bs) {
+  for (int i = tid; i < m4; i += bs) {
     float4 v = __ldg(src4 + i);
     uint4 u = make_uint4(ordered_key(v.x), ordered_key(v.y), ordered_key(v.z), ordered_key(v.w));
     reinterpret_cast<uint4 *>(keys)[i] = u;
   }
-  for (int i = 4 * n4 + tid; i < n; i += bs) keys[i] = ordered_key(__ldg(src + i));
+  for (int i = 4 * m4 + tid; i < m; i += bs) keys[i] = ordered_key(__ldg(src + i));
   __syncthreads();
 
   uint32_t prefix = 0u, pmask = 0u, k_rem = (uint32_t)k;
@@ -153,14 +190,28 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const int nb = pass == 2 ? 1024 : 2048;
+    uint32_t *hist = hist_s[pass & 1];
     for (int i = tid; i < nb; i += bs) hist[i] = 0u;
     __syncthreads();
-    for (int i = tid; i < n; i += bs) {
+    for (int i = tid; i < m; i += bs) {
       uint32_t u = keys[i];
       if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & (nb - 1)], 1u);
     }
     __syncthreads();
-    find_threshold_bin(hist, nb, k_rem, tmp, &s_bin, &s_above);
+    if (C > 1) {
+      // every slice histogram of the row is complete (the other parity's buffers were last read before
+      // this barrier, so they may be cleared in the next pass)
+      cl_sync();
+      for (int i = tid; i < nb; i += bs) {
+        uint32_t sum = 0u;
+        for (uint32_t c = 0; c < C; ++c) sum += cl_ld(hist + i, c);
+        ghist[i] = sum;
+      }
+    } else {
+      for (int i = tid; i < nb; i += bs) ghist[i] = hist[i];
+    }
+    __syncthreads();
+    find_threshold_bin(ghist, nb, k_rem, tmp, &s_bin, &s_above);
     prefix |= (uint32_t)s_bin << shift;
     pmask |= (uint32_t)(nb - 1) << shift;
     k_rem -= s_above;
@@ -168,25 +219,47 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
   }
   const uint32_t T = prefix;
 
-  // ordered compaction: each thread owns a contiguous range of positions
-  const int per = (n + bs - 1) / bs;
-  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  // ordered compaction: each thread owns a contiguous range of the slice; the slice's output offset is
+  // the selection of the slices before it (every key > T, keys == T in position order up to k_rem)
+  const int per = (m + bs - 1) / bs;
+  const int tlo = min(m, tid * per), thi = min(m, tlo + per);
   uint32_t gt = 0, eq = 0;
-  for (int i = lo; i < hi; ++i) {
+  for (int i = tlo; i < thi; ++i) {
     uint32_t u = keys[i];
     gt += u > T;
     eq += u == T;
   }
-  uint32_t eq_before = block_exclusive_scan(eq, tmp, nullptr);
-  uint32_t take_eq = k_rem > eq_before ? min(eq, k_rem - eq_before) : 0u;
-  uint32_t off = block_exclusive_scan(gt + take_eq, tmp, nullptr);
+  uint32_t gt_tot, eq_tot;
+  uint32_t eq_before = block_exclusive_scan(eq, tmp, &eq_tot);
+  const uint32_t gt_before = block_exclusive_scan(gt, tmp, &gt_tot);
+  uint32_t out_base = 0u, eq_base = 0u;
+  if (C > 1) {
+    if (tid == 0) {
+      cnt[0] = gt_tot;
+      cnt[1] = eq_tot;
+    }
+    cl_sync();
+    for (uint32_t c = 0; c < r; ++c) {
+      const uint32_t g = cl_ld(cnt, c), e = cl_ld(cnt + 1, c);
+      const uint32_t take = k_rem > eq_base ? min(e, k_rem - eq_base) : 0u;
+      out_base += g + take;
+      eq_base += e;
+    }
+  }
+  eq_before += eq_base;
+  const uint32_t take_eq = k_rem > eq_before ? min(eq, k_rem - eq_before) : 0u;
+  // equal keys taken before this thread, in this slice
+  const uint32_t eq_taken_slice = min(eq_before, k_rem) - min(eq_base, k_rem);
+  uint32_t off = out_base + gt_before + eq_taken_slice;
   uint32_t e = 0;
-  for (int i = lo; i < hi; ++i) {
+  for (int i = tlo; i < thi; ++i) {
     uint32_t u = keys[i];
     bool sel = u > T;
     if (u == T) { sel = e < take_eq; ++e; }
-    if (sel && off < (uint32_t)k) out[off++] = i;
+    if (sel && off < (uint32_t)k) out[off++] = lo + i;
   }
+  // no CTA leaves while another may still read its shared memory
+  if (C > 1) cl_sync();
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -363,10 +436,36 @@ dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, 
       return DSA_ERR_CUDA;
     }
   }
-  const size_t smem = (size_t)(kTopkSmemCap + kRadixBins + 64) * 4;
+  // cluster size: enough CTAs per row to fill the GPU when there are few rows
+  int C = 1;
+  while (C < 8 && (int64_t)b->total_q * C * 2 <= num_sms) C *= 2;
+  const int slice_max = std::min(kTopkSmemCap, ((b->max_seq_len + C - 1) / C + 3) & ~3);
+  const size_t smem = (size_t)(kTopkSmemFixedU32 + std::max(slice_max, 4)) * 4;
   cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  DSA_LAUNCH_PDL("topk_rows_smem_kernel", topk_rows_smem_kernel, dim3(b->total_q), dim3(kTopkThreadsA), smem, stream,
-                 scores, ld, bv, k, idx, lw, has_long ? 1 : 0);
+  cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(b->total_q * C));
+    cfg.blockDim = dim3(kTopkThreadsA);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)C;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    const int reg_long = has_long ? 1 : 0;
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, topk_rows_smem_kernel, scores, ld, bv, k, idx, lw, reg_long);
+    if (le != cudaSuccess) {
+      set_error("topk_rows_smem_kernel: %s", cudaGetErrorString(le));
+      return DSA_ERR_CUDA;
+    }
+    DSA_LAUNCH_CHECK("topk_rows_smem_kernel");
+  }
   if (has_long) {
     const int grid = max(num_sms * 4, topk_max_segs(b->max_seq_len));   // one segment per CTA per row
     for (int pass = 0; pass < 3; ++pass) {

@@ -62,6 +62,28 @@ def test_mla_small_prefill_every_row(grid):
     compare_rows(wl, db, list(range(wl.total_q)))
 
 
+def test_repeated_launches_are_bitwise_identical():
+    """The whole path is deterministic: the same batch run again (the first launch included) gives the
+    same bits.  Catches ordering races between the CTAs of a pair, which show up as run-to-run
+    differences in a few value blocks long before they break a tolerance."""
+    seq_lens = [70, 300, 2100, 2600]
+    q_lens = [70, 37, 300, 5]
+    wl = W.make_workload("small_prefill", kind="mla", seed=101, seq_lens=seq_lens, q_lens=q_lens, topk=2048,
+                         grid=True)
+    db = DeviceBatch(wl)
+    runs = []
+    for _ in range(5):
+        db.run()
+        torch.cuda.synchronize()
+        db.check_status()
+        runs.append((db.idx.clone(), db.out.clone(), db.lse.clone()))
+    for i, (ix, o, l) in enumerate(runs[1:], 1):
+        assert torch.equal(ix, runs[0][0]), f"launch {i}: top-k differs from the first launch"
+        bad = torch.nonzero((o != runs[0][1]).flatten(1).any(dim=1)).flatten().tolist()
+        assert not bad, f"launch {i}: attention output differs from the first launch in rows {bad[:8]}"
+        assert torch.equal(l, runs[0][2]), f"launch {i}: lse differs from the first launch"
+
+
 @pytest.mark.parametrize("grid", [True, False])
 def test_mla_small_decode_every_row(grid):
     wl = W.make_workload("small_decode", kind="mla", seed=102, seq_lens=EDGE_LENS, q_lens=[1] * len(EDGE_LENS),

@@ -112,6 +112,7 @@ __device__ __forceinline__ void unit_of(const AttArgs &a, int u, int *row, int *
 __device__ __forceinline__ int num_units(const AttArgs &a) { return a.T * a.splits; }
 
 // Walks the chunks of the units a CTA pair owns (units pair, pair + npairs, ...), skipping empty units.
+// Used by whole warps (the sequence lookup is warp-cooperative).
 struct ChunkCursor {
   int u, row, j, ce, seq;
   bool first;                   // j is the first chunk of its unit
@@ -124,7 +125,7 @@ struct ChunkCursor {
       unit_of(a, uu, &r, &cb, &ce2);
       if (ce2 > cb) {
         int b;
-        pos_of_row(a.bv, r, &b);
+        pos_of_row_warp(a.bv, r, &b);
         u = uu; row = r; j = cb; ce = ce2; first = true;
         seq = __ldg(a.bv.seq_lens + b);
         btr = a.bv.block_table + (int64_t)b * a.bv.max_blocks_per_seq;
@@ -339,6 +340,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
     ChunkCursor pc;
     pc.seek(a, pair, npairs);
     uint32_t v = 0;
+    auto load_q = [&](int qrow) {
+      if (rank == 0) tc::mbar_expect_tx(tc::smem_u32(&S->q_full), 2u * kAttQBytes);
+      for (int d = 0; d < 9; ++d)
+        tc::tma_load_2d_pair(tc::smem_u32(sQ + d * 8192), &tm_q, d * 64, qrow * kAttH + 64 * (int)rank, q_full_r0);
+    };
+    // the first unit's q needs no wait: fetch it before the first chunk's rows
+    if (!pc.done(a) && t == 0) load_q(pc.row);
     for (uint32_t c = 0; !pc.done(a); ++c) {
       const uint32_t b = c % kAttNBuf, use = c / kAttNBuf, slot = c % kAttRing;
       const int nblk = pw == 0 ? 3 : 2;
@@ -363,14 +371,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->phys_empty[slot]));
       if (pc.first) {
-        if (t == 0) {
-          const bool okq = v == 0 || tc::mbar_wait_cl(tc::smem_u32(&S->q_empty), (v - 1) & 1u, abort, status);
-          if (okq) {
-            if (rank == 0) tc::mbar_expect_tx(tc::smem_u32(&S->q_full), 2u * kAttQBytes);
-            for (int d = 0; d < 9; ++d)
-              tc::tma_load_2d_pair(tc::smem_u32(sQ + d * 8192), &tm_q, d * 64, pc.row * kAttH + 64 * (int)rank, q_full_r0);
-          }
-        }
+        // later units: q is overwritten once the previous unit's last QK^T has run
+        if (t == 0 && v > 0 && tc::mbar_wait_cl(tc::smem_u32(&S->q_empty), (v - 1) & 1u, abort, status)) load_q(pc.row);
         ++v;
       }
       pc.next(a, npairs);

@@ -55,6 +55,35 @@ __device__ __forceinline__ int pos_of_row(const BatchView &bv, int row, int *seq
   return __ldg(bv.seq_lens + b) - (c1 - c0) + (row - c0);
 }
 
+// seq_of_row for a whole warp (every lane calls it with the same row and gets the same result): each
+// round the 32 lanes test 32 evenly spaced entries of cu_q at once, so a batch of up to 33 sequences
+// needs one round of loads instead of a chain of dependent ones.  cu_q is non-decreasing, so the lanes
+// whose entry is <= row form a prefix of the warp.
+__device__ __forceinline__ int seq_of_row_warp(const int32_t *cu_q, int num_seqs, int row) {
+  const int lane = threadIdx.x & 31;
+  int lo = 0, hi = num_seqs - 1;       // the answer lies in [lo, hi]
+  while (lo < hi) {
+    const int step = (hi - lo + 31) / 32;
+    const int i = lo + 1 + lane * step;
+    const bool le = i <= hi && __ldg(cu_q + i) <= row;
+    const unsigned m = __ballot_sync(0xffffffffu, le);
+    if (m == 0u) {
+      hi = lo;
+    } else {
+      const int last = 31 - __clz(m);
+      lo = lo + 1 + last * step;
+      hi = min(hi, lo + step - 1);
+    }
+  }
+  return lo;
+}
+__device__ __forceinline__ int pos_of_row_warp(const BatchView &bv, int row, int *seq_out) {
+  int b = seq_of_row_warp(bv.cu_q, bv.num_seqs, row);
+  int c0 = __ldg(bv.cu_q + b), c1 = __ldg(bv.cu_q + b + 1);
+  *seq_out = b;
+  return __ldg(bv.seq_lens + b) - (c1 - c0) + (row - c0);
+}
+
 // physical row (block * page + slot) of logical token s of sequence b; -1 if the block id is bad
 __device__ __forceinline__ int64_t phys_row(const BatchView &bv, int b, int s) {
   int blk = __ldg(bv.block_table + (int64_t)b * bv.max_blocks_per_seq + s / bv.page_size);

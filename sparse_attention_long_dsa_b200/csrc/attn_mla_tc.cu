@@ -10,8 +10,9 @@
 // current one is computed, partial results are merged by a cross-block reduction.)
 //
 // Work split of a CTA pair (rank r = 0, 1) over chunks of 64 selected tokens:
-//   * resolve: one warp turns token positions into physical cache rows (block table), publishes the
-//              validity mask of the chunk and prefetches the rows into L2, several chunks ahead;
+//   * resolve: one warp turns token positions into physical cache rows (block table) and publishes the
+//              validity mask of the chunk, up to four chunks ahead (KV rows are not prefetched into L2:
+//              prefetches share the copy engine with the gathers and slowed them);
 //   * gather : each CTA gathers ITS 32 tokens of the chunk (tokens 32r..32r+31), all 576 dims, into one
 //              of three chunk buffers [9 dim blocks][32 tokens][128 B] (128-byte swizzle), by TMA gather4;
 //   * QK^T   : M = 128 heads (rank r holds heads 64r..64r+63 of q), N = 64 tokens (32 from each CTA),

@@ -139,6 +139,24 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------------- ours
+# ---------------------------------------------------------------------------------------------- multi-rank
+def slowest_rank_ms(ms, world, device):
+    """The job's time for a timed region is its slowest rank's: MAX all-reduce of this rank's CUDA-event
+    milliseconds (a no-op on one rank).  `device` is where the collective's tensor lives (the rank's GPU
+    under NCCL, the CPU under gloo)."""
+    if world > 1:
+        import torch
+        t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def job_tokens_per_s(tokens_per_rank_step, world, ms_per_step):
+    """Whole-job throughput under weak scaling: every rank processes its own batch of the same shape."""
+    return world * tokens_per_rank_step / (ms_per_step / 1e3)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     from sparse_attention_long_dsa_b200 import binding as B
@@ -205,12 +223,9 @@ def run_ours(args, rank, world, local_rank):
         for j, s in enumerate(stages):
             stage_ms[s].append(e[j].elapsed_time(e[j + 1]))
     stage_avg = {s: float(np.mean(v)) for s, v in stage_ms.items()}
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = slowest_rank_ms(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * work["tokens"] / (ms_per_step / 1e3)
+    value = job_tokens_per_s(work["tokens"], world, ms_per_step)
 
     # e2e: per-step inputs from pinned host memory, results read back, same public calls
     e2e = run_e2e(args, wl, replicas[0], stream, dev, world)
@@ -325,12 +340,8 @@ def run_e2e(args, wl, db, stream, dev, world):
             step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-    ms = a.elapsed_time(b)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * wl.total_q * args.steps / (ms / 1e3)
+    ms = slowest_rank_ms(a.elapsed_time(b), world, dev)
+    value = job_tokens_per_s(wl.total_q, world, ms / args.steps)
     return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": ms / args.steps}
 

@@ -28,6 +28,9 @@
  * Asynchrony: every compute call only enqueues work on `stream` (a cudaStream_t
  *   passed as void*; NULL is the legacy default stream) and returns without
  *   synchronising the host.  Outputs are valid once the stream reaches them.
+ *   Kernels are launched with programmatic dependent launch: one may be scheduled
+ *   while the preceding work on the stream finishes, but it touches no global
+ *   memory until that work has completed, so stream order holds as usual.
  * Errors: argument errors are detected on the host before anything is enqueued
  *   and return DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED / DSA_ERR_WORKSPACE with
  *   nothing written.  A failed launch returns DSA_ERR_CUDA.  Kernels never spin

@@ -11,9 +11,9 @@
 // Day-0 Adaptation of Million-Token Context Models on Domestic AI Chips", Four Key Layers 1).
 //
 // Two regimes:
-//   A) n <= C * kTopkSmemCap candidates: a cluster of C CTAs per row (C = 1, 2, 4 or 8, more when there
-//      are few rows, so that the rows fill the GPU), each CTA staging one contiguous slice of the row in
-//      shared memory.  Every digit pass builds slice histograms, which each CTA sums over the cluster
+//   A) n <= C * kTopkSmemCap candidates: a cluster of C CTAs per row (C = 1, 2, 4 or 8: more when there
+//      are few rows, so that the rows fill the GPU, and as many as the longest row needs, at most 2 for
+//      a large batch), each CTA staging one contiguous slice of the row in shared memory.  Every digit pass builds slice histograms, which each CTA sums over the cluster
 //      through distributed shared memory to the same row histogram; the ordered write offsets each
 //      slice by the counts of the slices before it.  One launch.
 //   B) longer rows (a million-token decode): the row is split into segments of kTopkSeg keys over
@@ -427,7 +427,16 @@ topk_long_write_kernel(const float *__restrict__ scores, int64_t ld, BatchView b
 dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx, void *ws,
                          cudaStream_t stream, int num_sms) {
   BatchView bv = view_of(b);
-  const bool has_long = b->max_seq_len > kTopkSmemCap;
+  // cluster size: enough CTAs per row to fill the GPU when there are few rows, then enough for the longest
+  // row to fit in the cluster's shared memory.  Regime B suits a handful of very long rows; a large batch
+  // of rows just past one CTA's capacity (a prefill chunk deep in a long prompt) is far cheaper here.
+  // With many rows the length-driven growth stops at 2 CTAs, since every CTA then takes the shared memory
+  // of the longest slice and fewer rows run at once; the rare longer rows of such a batch go to regime B.
+  int C = 1;
+  while (C < 8 && (int64_t)b->total_q * C * 2 <= num_sms) C *= 2;
+  const int c_len_max = (int64_t)b->total_q * 2 > num_sms ? 2 : 8;
+  while (C < c_len_max && (int64_t)b->max_seq_len > (int64_t)C * kTopkSmemCap) C *= 2;
+  const bool has_long = (int64_t)b->max_seq_len > (int64_t)C * kTopkSmemCap;
   TopkWs lw{};
   if (has_long) {
     lw = topk_ws_view(ws, b->total_q, b->max_seq_len);
@@ -436,9 +445,6 @@ dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, 
       return DSA_ERR_CUDA;
     }
   }
-  // cluster size: enough CTAs per row to fill the GPU when there are few rows
-  int C = 1;
-  while (C < 8 && (int64_t)b->total_q * C * 2 <= num_sms) C *= 2;
   const int slice_max = std::min(kTopkSmemCap, ((b->max_seq_len + C - 1) / C + 3) & ~3);
   const size_t smem = (size_t)(kTopkSmemFixedU32 + std::max(slice_max, 4)) * 4;
   cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

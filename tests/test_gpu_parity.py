@@ -171,6 +171,18 @@ def test_topk_alone_ties_and_lengths(k):
     _topk_alone(rows, k)
 
 
+@pytest.mark.parametrize("max_len", [131072, 300000])
+def test_topk_alone_many_rows_past_one_cta(max_len):
+    # more rows than half the SMs, all longer than one CTA's shared-memory slice: the rows are taken by
+    # 2-CTA clusters up to 98304 candidates and by the multi-launch long-row path beyond, in one call
+    rng = np.random.default_rng(max_len)
+    rows = []
+    for i, n in enumerate(rng.integers(49153, max_len + 1, 150)):
+        n = int(max_len) if i == 0 else int(n)
+        rows.append(rng.integers(-40, 40, n).astype(np.float32) if i % 2 else rng.standard_normal(n).astype(np.float32))
+    _topk_alone(rows, 2048)
+
+
 def test_topk_alone_long_row():
     rng = np.random.default_rng(9)
     rows = [rng.standard_normal(1 << 20).astype(np.float32),

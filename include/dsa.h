@@ -42,6 +42,10 @@
  *   cu_q[b] .. cu_q[b+1]-1, which are its LAST n_b = cu_q[b+1]-cu_q[b] tokens:
  *   row cu_q[b]+i sits at absolute position pos = seq_lens[b] - n_b + i and may
  *   attend to positions 0..pos (its own entry is already in the cache).
+ *   A sequence may own no rows (n_b == 0) anywhere in the batch.  An empty batch
+ *   (total_q == 0) is a no-op: every compute call checks the descriptor and returns
+ *   DSA_OK without enqueueing anything or needing a device; its data pointers may
+ *   then be NULL.
  * Paged cache: token s of sequence b lives in physical block
  *   block_table[b * max_blocks_per_seq + s / page_size], slot s % page_size.
  *   Only entries for s < seq_lens[b] are read.

@@ -179,6 +179,7 @@ dsa_status_t dsa_indexer_scores(const void *q_idx, dsa_dtype_t q_dt, const float
                                 void *stream) {
   dsa_status_t st = check_batch(b);
   if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
   CHECK_ARG(q_idx && w && k_idx_pool && scores, "q_idx, w, k_idx_pool and scores are required");
   CHECK_ARG(q_dt == k_dt, "query and key dtypes differ");
   CHECK_ARG(ld_scores >= b->max_seq_len && ld_scores % 4 == 0,
@@ -194,7 +195,6 @@ dsa_status_t dsa_indexer_scores(const void *q_idx, dsa_dtype_t q_dt, const float
   if ((st = check_ws(ws, ws_bytes, indexer_workspace_bytes(b->num_seqs, b->total_q))) != DSA_OK) return st;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
-  if (b->total_q == 0) return DSA_OK;
   if (mla)
     return indexer_tc_launch((const uint8_t *)q_idx, w, (const uint8_t *)k_idx_pool, k_scale_pool, b, scores,
                              ld_scores, ws, (cudaStream_t)stream, dev.num_sms);
@@ -206,6 +206,7 @@ dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_batch_t 
                       void *ws, size_t ws_bytes, void *stream) {
   dsa_status_t st = check_batch(b);
   if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
   CHECK_ARG(scores && idx, "scores and idx are required");
   CHECK_SUP(k >= 1 && k <= 16384, "k must be in [1, 16384] (got %d)", k);
   CHECK_ARG(ld_scores >= b->max_seq_len && ld_scores % 4 == 0,
@@ -214,7 +215,6 @@ dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_batch_t 
   if ((st = check_ws(ws, ws_bytes, topk_workspace_bytes(b->total_q, b->max_seq_len))) != DSA_OK) return st;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
-  if (b->total_q == 0) return DSA_OK;
   return topk_launch(scores, ld_scores, b, k, idx, ws, (cudaStream_t)stream, dev.num_sms);
 }
 
@@ -222,6 +222,7 @@ dsa_status_t dsa_topk_noalloc(const float *scores, int64_t ld_scores, const dsa_
                               int32_t *idx, void *stream) {
   dsa_status_t st = check_batch(b);
   if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
   CHECK_ARG(scores && idx, "scores and idx are required");
   CHECK_SUP(k >= 1 && k <= 16384, "k must be in [1, 16384] (got %d)", k);
   CHECK_ARG(ld_scores >= b->max_seq_len && ld_scores % 4 == 0,
@@ -229,7 +230,6 @@ dsa_status_t dsa_topk_noalloc(const float *scores, int64_t ld_scores, const dsa_
   CHECK_ARG(((uintptr_t)scores & 15) == 0, "scores must be 16-byte aligned");
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
-  if (b->total_q == 0) return DSA_OK;
   return topk_noalloc_launch(scores, ld_scores, b, k, idx, (cudaStream_t)stream, dev.num_sms);
 }
 
@@ -239,6 +239,7 @@ static dsa_status_t attn_common(bool decode, const void *q, dsa_dtype_t dt, cons
                                 void *stream) {
   dsa_status_t st = check_batch(b);
   if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
   CHECK_ARG(q && kv_pool && idx && out, "q, kv_pool, idx and out are required");
   CHECK_ARG(k >= 1, "k must be >= 1");
   CHECK_ARG(softmax_scale == softmax_scale && softmax_scale > 0.f && softmax_scale < 1e30f,
@@ -255,7 +256,6 @@ static dsa_status_t attn_common(bool decode, const void *q, dsa_dtype_t dt, cons
   if ((st = check_ws(ws, ws_bytes, attn_ws_bytes(b, k, H, Dv, decode))) != DSA_OK) return st;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
-  if (b->total_q == 0) return DSA_OK;
   if (mla)
     return attn_mla_launch(q, kv_pool, idx, k, softmax_scale, b, out, lse, ws, decode, (cudaStream_t)stream,
                            dev.num_sms);

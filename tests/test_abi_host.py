@@ -94,3 +94,19 @@ def test_nonfinite_scale_rejected():
     with pytest.raises(B.DSAError) as e:
         B.dsa_sparse_attn_decode(P, B.DSA_BF16, P, None, 128, 576, 512, float("nan"), P, 16, b, P, P, P, 1 << 20, 0)
     assert e.value.status == B.DSA_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_noop_without_a_device():
+    """total_q == 0: every compute entry validates the descriptor and returns DSA_OK, enqueueing nothing
+    (no device is touched, so this holds on a host without a GPU) and accepting NULL data pointers."""
+    b = _batch(total_q=0, max_q_per_seq=0)
+    n0 = B.dsa_launch_count()
+    B.dsa_indexer_scores(None, B.DSA_FP8_E4M3, None, None, B.DSA_FP8_E4M3, None, 64, 128, b, None, 128, None, 0, 0)
+    B.dsa_topk(None, 128, b, 2048, None, None, 0, 0)
+    B.dsa_topk_noalloc(None, 128, b, 2048, None, 0)
+    B.dsa_sparse_attn_prefill(None, B.DSA_BF16, None, None, 128, 576, 512, 0.07, None, 2048, b, None, None, None, 0, 0)
+    B.dsa_sparse_attn_decode(None, B.DSA_BF16, None, None, 128, 576, 512, 0.07, None, 2048, b, None, None, None, 0, 0)
+    assert B.dsa_launch_count() == n0
+    with pytest.raises(B.DSAError) as e:      # the descriptor itself is still checked
+        B.dsa_topk(None, 128, _batch(total_q=0, max_q_per_seq=0, page_size=32), 2048, None, None, 0, 0)
+    assert e.value.status == B.DSA_ERR_UNSUPPORTED

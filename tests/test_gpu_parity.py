@@ -236,3 +236,24 @@ def test_errors_leave_outputs_untouched():
     assert e.value.status == B.DSA_ERR_INVALID_ARG          # two query rows in one sequence
     torch.cuda.synchronize()
     assert bool((db.idx == -5).all())
+
+
+# --------------------------------------------------------------------------------------- ragged batches
+@pytest.mark.parametrize("grid", [True, False])
+def test_sequences_without_query_rows(grid):
+    """Sequences that own no query rows, first, between others and last, beside a whole 64-token prompt,
+    a one-token sequence and rows past the 2048-token top-k: every row against the oracle."""
+    wl = W.make_workload("ragged_empty", kind="mla", seed=107, seq_lens=[100, 64, 2100, 1, 700, 130, 3000, 90],
+                         q_lens=[0, 64, 0, 1, 3, 0, 2, 0], topk=2048, grid=grid)
+    db = _run(wl)
+    compare_rows(wl, db, list(range(wl.total_q)))
+
+
+def test_empty_batch_launches_nothing():
+    wl = W.make_workload("empty", kind="mla", seed=108, seq_lens=[50, 300], q_lens=[0, 0], topk=2048)
+    db = DeviceBatch(wl)
+    n0 = B.dsa_launch_count()
+    db.run()
+    torch.cuda.synchronize()
+    assert B.dsa_launch_count() == n0
+    assert db.out.numel() == 0 and db.idx.numel() == 0

@@ -35,6 +35,7 @@
 // Units: prefill = one row (all its chunks); decode = (row, split) pairs whose partial (o, lse) are
 // merged by attn_combine_kernel.  Rows are taken longest-first (reverse order) round-robin over pairs.
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstdlib>
 
@@ -801,8 +802,12 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
                  neff, a.status);
   const size_t smem = attn_smem_bytes();
   cudaFuncSetAttribute(attn_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  // persistent grid: as many CTA pairs as can be resident at once
-  static int max_pairs = 0;
+  // persistent grid: as many CTA pairs as can be resident at once (found once per device; threads that race
+  // on the first call compute the same number)
+  static std::atomic<int> resident_pairs[kMaxDevices];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = -1;
+  int max_pairs = dev >= 0 ? resident_pairs[dev].load(std::memory_order_relaxed) : 0;
   if (max_pairs == 0) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr;
@@ -821,6 +826,7 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
       n = num_sms / 2;
     }
     max_pairs = std::min(n, num_sms / 2);
+    if (dev >= 0) resident_pairs[dev].store(max_pairs, std::memory_order_relaxed);
     if (getenv("DSA_VERBOSE")) fprintf(stderr, "[libdsa] attention: %d resident CTA pairs\n", max_pairs);
   }
   const int units = a.T * a.splits;

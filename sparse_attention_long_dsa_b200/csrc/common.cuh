@@ -15,6 +15,7 @@ namespace dsa {
 // error bits set by kernels (bounded waits that ran out, out-of-range ids).
 // ---------------------------------------------------------------------------------------------
 constexpr size_t kWsHeader = 256;
+constexpr int kMaxDevices = 64;        // per-device host caches are indexed by the CUDA device ordinal
 constexpr uint32_t kStatusTimeout = 1u;
 constexpr uint32_t kStatusBadIndex = 2u;
 

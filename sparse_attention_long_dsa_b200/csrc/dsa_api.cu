@@ -43,7 +43,6 @@ void set_error(const char *fmt, ...) {
   va_end(ap);
 }
 
-constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   int num_sms = 0;
   int cc_major = 0, cc_minor = 0;

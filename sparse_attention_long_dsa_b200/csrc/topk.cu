@@ -503,13 +503,13 @@ constexpr size_t kNoAllocBytes =
 
 static __device__ __align__(256) unsigned char g_topk_scratch[kNoAllocBytes];
 
-static void *g_topk_scratch_addr[64];
+static void *g_topk_scratch_addr[kMaxDevices];
 static std::mutex g_topk_scratch_mu;
 
 // device address of the scratch array on the current device (looked up on first use per device)
 static dsa_status_t topk_scratch_address(void **out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     set_error("dsa_topk_noalloc: no current CUDA device");
     return DSA_ERR_CUDA;
   }

@@ -36,6 +36,14 @@ What each step follows (page titles and sections of the source pages):
   o = sum p V / sum p, lse = m + ln(sum p).
 * Split combine -- "Engineering Practices ...", Four Key Layers 3 (partial
   results over candidate KV blocks followed by a cross-block reduction).
+* Cache append -- "Engineering Practices ...", Four Key Layers 3 (the decode
+  step writes the new token into the KV cache, merged with its attention
+  launch) and 2 (the block table places a token in its block); the indexer
+  key is stored as FP8 E4M3 with one scale per token ("Day-0 Adaptation for
+  LLMs ...", III.1: low-precision index scoring).  The pages do not spell the
+  quantiser out; this library takes scale = max|k| / 448 (1 for an all-zero
+  key) and code = the E4M3 value nearest to k / scale, ties to the even code,
+  clamped to +-448, both divisions in fp32.
 
 Every function is pinned by tests/test_oracle_pins.py against values fixed
 by hand or by independent arithmetic (exact rationals, torch library
@@ -92,6 +100,23 @@ def _real(arr: np.ndarray, fmt: str) -> np.ndarray:
     raise ValueError(fmt)
 
 
+E4M3_MAX = 448.0
+_E4M3_NONNEG = E4M3[:0x7F]          # codes 0x00..0x7E: the finite non-negative values, increasing
+
+
+def e4m3_encode_rne(v) -> np.ndarray:
+    """E4M3 code of each real v: the finite value nearest to v, on a tie the code whose last
+    mantissa bit is 0, magnitudes beyond 448 clamped to 448; the sign bit is v's (so a
+    negative v that rounds to zero gives -0).  Brute force over all 127 magnitudes."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    d = np.abs(a[..., None] - _E4M3_NONNEG)                 # [..., 127] distance to every magnitude
+    nearest = d == d.min(axis=-1, keepdims=True)            # one code, or two adjacent ones on a tie
+    even = nearest & (np.arange(_E4M3_NONNEG.size) % 2 == 0)
+    code = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(nearest, axis=-1))
+    return np.where(np.signbit(v), code | 0x80, code).astype(np.uint8)
+
+
 # ----------------------------------------------------------------------------
 # paged layout
 # ----------------------------------------------------------------------------
@@ -115,6 +140,42 @@ def _formats(case):
     if case.kind == "f32":
         return dict(q="f32", kv="f32", qI="f32", kI="f32")
     return dict(q="bf16", kv="bf16", qI="e4m3", kI="e4m3")
+
+
+# ----------------------------------------------------------------------------
+# step 0: appending new tokens to the paged cache
+# ----------------------------------------------------------------------------
+
+def quantize_index_key(k):
+    """(codes, scale) of one indexer key: scale = max|k| / 448 in fp32 (1 when that is 0),
+    codes = e4m3(k / scale) with the quotient taken in fp32."""
+    k32 = np.asarray(k, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(k32))) if k32.size else np.float32(0.0)
+    scale = np.float32(amax / np.float32(E4M3_MAX))
+    if scale == 0:
+        scale = np.float32(1.0)
+    return e4m3_encode_rne((k32 / scale).astype(np.float64)), scale
+
+
+def cache_append(case, kv_new, kI_new, kI_fmt: str):
+    """The pools after the batch's query rows are written as new tokens.  Row cu_q[b] + i is the
+    token at position seq_lens[b] - q_len[b] + i of sequence b (the same rows the other steps
+    treat as queries); its latent row is copied bit for bit into kv_pool, its indexer key is
+    quantised into kI_pool (codes) and kS_pool (scale), all at the token's (block, slot).
+    Returns new arrays (kv_pool, kI_pool, kS_pool); the inputs are not modified."""
+    kv_pool = np.array(case.kv_pool, copy=True)
+    kI_pool = np.array(case.kI_pool, copy=True)
+    kS_pool = np.array(case.kS_pool, copy=True)
+    T = int(case.cu_q[-1])
+    for row in range(T):
+        b, pos = row_location(case.seq_lens, case.cu_q, row)
+        blk, slot = token_slots(case.block_table[b], np.array([pos]), case.page_size)
+        blk, slot = int(blk[0]), int(slot[0])
+        kv_pool[blk, slot] = np.asarray(kv_new[row])
+        codes, scale = quantize_index_key(_real(kI_new[row], kI_fmt))
+        kI_pool[blk, slot] = codes
+        kS_pool[blk, slot] = scale
+    return kv_pool, kI_pool, kS_pool
 
 
 # ----------------------------------------------------------------------------

@@ -327,3 +327,88 @@ def test_planted_long_context_selection():
     assert np.array_equal(idx, wl.planted)
     others = np.delete(sc, wl.planted)
     assert sc[wl.planted].min() > 2.0 * max(others.max(), 0.0)
+
+
+# ----------------------------------------------------------------------------- cache append (FP8 key quantiser)
+
+def _e4m3_midpoints():
+    """Every value halfway between two adjacent finite E4M3 magnitudes (exact in fp32), with the
+    fp32 neighbours on either side of each."""
+    mags = oracle.E4M3[:0x7F].astype(np.float32)
+    mid = ((mags[:-1].astype(np.float64) + mags[1:]) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (mags[:-1].astype(np.float64) + mags[1:]) / 2)
+    return np.concatenate([mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(np.inf))])
+
+
+def test_e4m3_encoder_matches_torch_cast():
+    """Round to nearest, ties to even, signed zero: torch's fp32 -> float8_e4m3fn cast on |v| <= 448
+    (ties between every adjacent pair of codes, the subnormal range, random values, +-0)."""
+    rng = np.random.default_rng(5)
+    pos = np.concatenate([_e4m3_midpoints(), oracle.E4M3[:0x7F].astype(np.float32),
+                          rng.uniform(0, 448, 20000).astype(np.float32),
+                          (rng.uniform(0, 2 ** -6, 5000)).astype(np.float32),
+                          np.array([0.0, 1e-30, 2 ** -10, 3 * 2 ** -11, 448.0], np.float32)])
+    v = np.concatenate([pos, -pos])
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode_rne(v.astype(np.float64)), ref)
+
+
+def test_e4m3_encoder_saturates():
+    codes = oracle.e4m3_encode_rne(np.array([448.0, 460.0, 464.0, 500.0, 1e9, -470.0, -1e30]))
+    assert codes.tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE]
+
+
+def test_quantize_index_key_hand():
+    g = _golden("cache_append_hand.json")
+    for row in g["rows"]:
+        codes, scale = oracle.quantize_index_key(np.array(row["k"], np.float32))
+        assert codes.tolist() == row["codes"], row["note"]
+        exact = Fraction(row["scale"])
+        # the fp32 value nearest to the exact scale: no fp32 neighbour is closer
+        assert scale.dtype == np.float32
+        for nb in (np.nextafter(scale, np.float32(0)), np.nextafter(scale, np.float32(np.inf))):
+            assert abs(Fraction(float(scale)) - exact) <= abs(Fraction(float(nb)) - exact)
+
+
+def test_quantize_index_key_error_bound_and_range():
+    """Dequantised keys are within half a grid step of the key (a step is 2^-3 of the binade for
+    normal codes, 2^-9 for subnormal ones, both times the scale), and the largest |k| maps to 448."""
+    rng = np.random.default_rng(6)
+    for i in range(300):
+        k = (rng.standard_normal(128) * 10.0 ** rng.uniform(-3, 3)).astype(np.float32)
+        if i % 7 == 0:
+            k[rng.integers(0, 128, 40)] = 0.0
+        codes, scale = oracle.quantize_index_key(k)
+        deq = oracle.E4M3[codes] * float(scale)
+        q = np.abs(k.astype(np.float64)) / float(scale)
+        step = np.where(q >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(q, 2.0 ** -6))) - 3), 2.0 ** -9)
+        assert np.all(np.abs(deq - k) <= 0.5 * step * float(scale) * (1 + 1e-6) + 1e-300)
+        assert np.all((codes & 0x7F) <= 0x7E)
+        assert (codes[np.argmax(np.abs(k))] & 0x7F) == 0x7E
+
+
+def test_cache_append_places_tokens_by_hand():
+    """Two sequences, shuffled blocks: row 0, 1 are positions 68, 69 of sequence 0 (its block 1 =
+    physical 0, slots 4 and 5); row 2 is position 4 of sequence 1 (its block 0 = physical 1, slot 4).
+    Nothing else changes."""
+    rng = np.random.default_rng(7)
+    NB, P = 4, 64
+    case = SimpleNamespace(page_size=P, seq_lens=np.array([70, 5], np.int32), cu_q=np.array([0, 2, 3], np.int32),
+                           block_table=np.array([[3, 0], [1, 2]], np.int32),
+                           kv_pool=rng.integers(0, 1 << 16, (NB, P, 576)).astype(np.uint16),
+                           kI_pool=rng.integers(0, 256, (NB, P, 128)).astype(np.uint8),
+                           kS_pool=rng.uniform(0.1, 1, (NB, P)).astype(np.float32))
+    kv_new = rng.integers(0, 1 << 16, (3, 576)).astype(np.uint16)
+    kI_new = np.stack([np.full(128, 448.0), np.zeros(128), np.full(128, -2.0)]).astype(np.float32)
+    kv, kI, kS = oracle.cache_append(case, kv_new, kI_new, "f32")
+    where = {0: (0, 4), 1: (0, 5), 2: (1, 4)}
+    touched = np.zeros((NB, P), bool)
+    for r, (blk, slot) in where.items():
+        touched[blk, slot] = True
+        assert np.array_equal(kv[blk, slot], kv_new[r])
+    assert kI[0, 4].tolist() == [0x7E] * 128 and kS[0, 4] == np.float32(1.0)
+    assert kI[0, 5].tolist() == [0] * 128 and kS[0, 5] == np.float32(1.0)
+    assert kI[1, 4].tolist() == [0xFE] * 128 and kS[1, 4] == np.float32(2.0 / 448.0)
+    assert np.array_equal(kv[~touched], case.kv_pool[~touched])
+    assert np.array_equal(kI[~touched], case.kI_pool[~touched])
+    assert np.array_equal(kS[~touched], case.kS_pool[~touched])

@@ -12,6 +12,7 @@
  *   dsa_topk                 the k best s per query row (ties -> lower s), ascending
  *   dsa_sparse_attn_prefill  softmax attention of every head over the selected rows
  *   dsa_sparse_attn_decode   the same, specialised for one query row per sequence
+ *   dsa_cache_append         writes the batch's new tokens into the paged pools (FP8 keys)
  *
  * ("Day-0 Adaptation for LLMs: Implementing Sparse Attention and Low-Precision
  * Weights", III.1 Index Selection Path and the decode sketch: score -> topk ->
@@ -89,7 +90,8 @@ typedef enum {
   DSA_OP_INDEXER = 0,
   DSA_OP_TOPK = 1,
   DSA_OP_ATTN_PREFILL = 2,
-  DSA_OP_ATTN_DECODE = 3
+  DSA_OP_ATTN_DECODE = 3,
+  DSA_OP_CACHE_APPEND = 4
 } dsa_op_t;
 
 /* Batch descriptor shared by every call.  The three host integers at the end are
@@ -182,6 +184,28 @@ DSA_API dsa_status_t dsa_sparse_attn_decode(const void *q, dsa_dtype_t dt, const
                                     int32_t H, int32_t Dqk, int32_t Dv, float softmax_scale,
                                     const int32_t *idx, int32_t k, const dsa_batch_t *b,
                                     void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* Cache append ("Engineering Practices ...", Four Key Layers 3: the decode step writes the
+ * new token into the KV cache; Four Key Layers 2: the block table places it; "Day-0
+ * Adaptation for LLMs ...", III.1: FP8 indexer keys).  Every query row of the batch is a new
+ * token, at the position the other calls give it (row cu_q[b] + i is token
+ * seq_lens[b] - n_b + i of sequence b, so seq_lens already counts the new tokens).  For each:
+ *   kv_pool[token]      = kv_new[row]                         (576 bf16, copied bit for bit)
+ *   k_scale_pool[token] = max_d |k_new[row, d]| / 448          (fp32; 1 if that is 0)
+ *   k_idx_pool[token,d] = E4M3(k_new[row, d] / scale)          (fp32 quotient, round to nearest
+ *                                                                even, saturating at +-448)
+ *   kv_new      [total_q, Dqk] of kv_dt;   k_new [total_q, Di] of k_dt (f32 or bf16, finite)
+ *   kv_pool     [num_blocks, page_size, Dqk];  k_idx_pool [num_blocks, page_size, Di] e4m3;
+ *   k_scale_pool [num_blocks, page_size] f32
+ * Supported: kv_dt bf16 with Dqk = 576, Di = 128 (the MLA path's pools).  kv_new, k_new,
+ * kv_pool and k_idx_pool 16-byte aligned.  The workspace only carries the status word
+ * (dsa_workspace_size(DSA_OP_CACHE_APPEND) = 256 bytes): a block id outside [0, num_blocks)
+ * or a position outside the block table leaves that token unwritten and is reported by
+ * dsa_read_device_status as DSA_ERR_DEVICE_CHECK.  Two rows that map to the same token race. */
+DSA_API dsa_status_t dsa_cache_append(const void *kv_new, dsa_dtype_t kv_dt, const void *k_new, dsa_dtype_t k_dt,
+                                      int32_t Dqk, int32_t Di, const dsa_batch_t *b, void *kv_pool,
+                                      void *k_idx_pool, float *k_scale_pool, void *ws, size_t ws_bytes,
+                                      void *stream);
 
 /* Synchronises `stream`, then reads and clears the status word at the start of a
  * workspace used by the calls above: DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK. */

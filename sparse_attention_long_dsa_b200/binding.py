@@ -17,11 +17,11 @@ LIB_PATH = os.path.join(PKG, "libdsa.so")
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_DEVICE_CHECK, \
     DSA_ERR_TIMEOUT = range(7)
 DSA_F32, DSA_BF16, DSA_FP8_E4M3 = 0, 1, 2
-DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_ATTN_PREFILL, DSA_OP_ATTN_DECODE = 0, 1, 2, 3
+DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_ATTN_PREFILL, DSA_OP_ATTN_DECODE, DSA_OP_CACHE_APPEND = 0, 1, 2, 3, 4
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn_prefill",
            "dsa_sparse_attn_decode", "dsa_read_device_status", "dsa_status_string", "dsa_last_error",
-           "dsa_version", "dsa_launch_count", "dsa_topk_noalloc")
+           "dsa_version", "dsa_launch_count", "dsa_topk_noalloc", "dsa_cache_append")
 
 
 class dsa_batch_t(ctypes.Structure):
@@ -66,6 +66,7 @@ def load(path: str = LIB_PATH):
         "dsa_topk_noalloc": [P, I64, B, I32, P, P],
         "dsa_sparse_attn_prefill": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
         "dsa_sparse_attn_decode": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
+        "dsa_cache_append": [P, I32, P, I32, I32, I32, B, P, P, P, P, SZ, P],
         "dsa_read_device_status": [P, P],
     }
     for name, args in sig.items():
@@ -152,6 +153,13 @@ def dsa_sparse_attn_decode(q, dt: int, kv_pool, v_pool, H: int, Dqk: int, Dv: in
     _check(load().dsa_sparse_attn_decode(_ptr(q), dt, _ptr(kv_pool), _ptr(v_pool), H, Dqk, Dv, softmax_scale,
                                          _ptr(idx), k, ctypes.byref(batch), _ptr(out), _ptr(lse), _ptr(ws),
                                          ws_bytes, _stream(stream)), "dsa_sparse_attn_decode")
+
+
+def dsa_cache_append(kv_new, kv_dt: int, k_new, k_dt: int, Dqk: int, Di: int, batch: dsa_batch_t, kv_pool, k_idx_pool,
+                     k_scale_pool, ws, ws_bytes: int, stream=None):
+    _check(load().dsa_cache_append(_ptr(kv_new), kv_dt, _ptr(k_new), k_dt, Dqk, Di, ctypes.byref(batch), _ptr(kv_pool),
+                                   _ptr(k_idx_pool), _ptr(k_scale_pool), _ptr(ws), ws_bytes, _stream(stream)),
+           "dsa_cache_append")
 
 
 def dsa_read_device_status(ws, stream=None):

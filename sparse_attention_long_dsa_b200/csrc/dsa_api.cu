@@ -27,6 +27,8 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
                              const dsa_batch_t *b, void *out, float *lse, void *ws, bool decode, cudaStream_t stream,
                              int num_sms);
 size_t attn_workspace_bytes(int T, int k, bool decode);
+dsa_status_t cache_append_launch(const void *kv_new, const void *k_new, bool k_bf16, const dsa_batch_t *b,
+                                 void *kv_pool, void *kI_pool, float *kS_pool, void *ws, cudaStream_t stream);
 dsa_status_t attn_simt_launch(const void *q, dsa_dtype_t dt, const void *kv, const void *v, int H, int Dqk, int Dv,
                               float scale, const int32_t *idx, int k, const dsa_batch_t *b, void *out, float *lse,
                               cudaStream_t stream);
@@ -167,6 +169,7 @@ dsa_status_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t *b, int32_t k, in
     case DSA_OP_TOPK: *bytes = topk_workspace_bytes(b->total_q, b->max_seq_len); return DSA_OK;
     case DSA_OP_ATTN_PREFILL: *bytes = attn_ws_bytes(b, k, H, Dv, false); return DSA_OK;
     case DSA_OP_ATTN_DECODE: *bytes = attn_ws_bytes(b, k, H, Dv, true); return DSA_OK;
+    case DSA_OP_CACHE_APPEND: *bytes = kWsHeader; return DSA_OK;
   }
   set_error("unknown op %d", (int)op);
   return DSA_ERR_INVALID_ARG;
@@ -276,6 +279,26 @@ dsa_status_t dsa_sparse_attn_decode(const void *q, dsa_dtype_t dt, const void *k
                                     void *stream) {
   return attn_common(true, q, dt, kv_pool, v_pool, H, Dqk, Dv, softmax_scale, idx, k, b, out, lse, ws, ws_bytes,
                      stream);
+}
+
+dsa_status_t dsa_cache_append(const void *kv_new, dsa_dtype_t kv_dt, const void *k_new, dsa_dtype_t k_dt, int32_t Dqk,
+                              int32_t Di, const dsa_batch_t *b, void *kv_pool, void *k_idx_pool, float *k_scale_pool,
+                              void *ws, size_t ws_bytes, void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
+  CHECK_ARG(kv_new && k_new && kv_pool && k_idx_pool && k_scale_pool,
+            "kv_new, k_new, kv_pool, k_idx_pool and k_scale_pool are required");
+  CHECK_SUP(kv_dt == DSA_BF16 && Dqk == 576 && Di == 128 && (k_dt == DSA_F32 || k_dt == DSA_BF16),
+            "cache append supports bf16 latent rows of 576 and f32 or bf16 indexer keys of 128");
+  CHECK_ARG((((uintptr_t)kv_new | (uintptr_t)k_new | (uintptr_t)kv_pool | (uintptr_t)k_idx_pool) & 15) == 0 &&
+                ((uintptr_t)k_scale_pool & 3) == 0,
+            "kv_new, k_new, kv_pool and k_idx_pool must be 16-byte aligned, k_scale_pool 4-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, kWsHeader)) != DSA_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return cache_append_launch(kv_new, k_new, k_dt == DSA_BF16, b, kv_pool, k_idx_pool, k_scale_pool, ws,
+                             (cudaStream_t)stream);
 }
 
 dsa_status_t dsa_read_device_status(void *ws, void *stream) {

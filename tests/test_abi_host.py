@@ -106,7 +106,31 @@ def test_empty_batch_is_a_noop_without_a_device():
     B.dsa_topk_noalloc(None, 128, b, 2048, None, 0)
     B.dsa_sparse_attn_prefill(None, B.DSA_BF16, None, None, 128, 576, 512, 0.07, None, 2048, b, None, None, None, 0, 0)
     B.dsa_sparse_attn_decode(None, B.DSA_BF16, None, None, 128, 576, 512, 0.07, None, 2048, b, None, None, None, 0, 0)
+    B.dsa_cache_append(None, B.DSA_BF16, None, B.DSA_F32, 576, 128, b, None, None, None, None, 0, 0)
     assert B.dsa_launch_count() == n0
     with pytest.raises(B.DSAError) as e:      # the descriptor itself is still checked
         B.dsa_topk(None, 128, _batch(total_q=0, max_q_per_seq=0, page_size=32), 2048, None, None, 0, 0)
     assert e.value.status == B.DSA_ERR_UNSUPPORTED
+
+
+def test_cache_append_rejects_before_launch():
+    b = _batch()
+    P = 1 << 24
+    assert B.dsa_workspace_size(B.DSA_OP_CACHE_APPEND, b) == 256
+    cases = [
+        (dict(Di=64), B.DSA_ERR_UNSUPPORTED),                         # only the MLA pools' key width
+        (dict(Dqk=512), B.DSA_ERR_UNSUPPORTED),
+        (dict(k_dt=B.DSA_FP8_E4M3), B.DSA_ERR_UNSUPPORTED),           # keys arrive unquantised
+        (dict(kv_dt=B.DSA_F32), B.DSA_ERR_UNSUPPORTED),
+        (dict(k_scale_pool=None), B.DSA_ERR_INVALID_ARG),
+        (dict(k_new=P + 8), B.DSA_ERR_INVALID_ARG),                   # misaligned
+        (dict(ws_bytes=128), B.DSA_ERR_WORKSPACE),
+    ]
+    for bad, status in cases:
+        a = dict(kv_new=P, kv_dt=B.DSA_BF16, k_new=P, k_dt=B.DSA_F32, Dqk=576, Di=128, kv_pool=P, k_idx_pool=P,
+                 k_scale_pool=P, ws=P, ws_bytes=256)
+        a.update(bad)
+        with pytest.raises(B.DSAError) as e:
+            B.dsa_cache_append(a["kv_new"], a["kv_dt"], a["k_new"], a["k_dt"], a["Dqk"], a["Di"], b, a["kv_pool"],
+                               a["k_idx_pool"], a["k_scale_pool"], a["ws"], a["ws_bytes"], 0)
+        assert e.value.status == status, bad

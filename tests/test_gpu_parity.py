@@ -257,3 +257,85 @@ def test_empty_batch_launches_nothing():
     torch.cuda.synchronize()
     assert B.dsa_launch_count() == n0
     assert db.out.numel() == 0 and db.idx.numel() == 0
+
+
+# --------------------------------------------------------------------------------------- cache append
+def _e4m3_ties_row():
+    """448 (so the scale is 1) and every value halfway between two adjacent E4M3 magnitudes (126 of
+    them, all exact in bf16), padded with 1.0 to 128 entries."""
+    mags = oracle.E4M3[:0x7F]
+    mid = (mags[:-1] + mags[1:]) / 2
+    return np.concatenate([[448.0], mid, [1.0]]).astype(np.float32)
+
+
+def _append_inputs(T, rng, k_bf16):
+    """(kv_new as int16 bf16 bits, keys as passed to the call, their format) for T new tokens."""
+    kv_new = W.bf16_encode(rng.standard_normal((T, 576)).astype(np.float32)).view(np.int16)
+    k = (rng.standard_normal((T, 128)) * 10.0 ** rng.uniform(-3, 3, (T, 1))).astype(np.float32)
+    k[0] = 0.0                                                      # all-zero key: scale 1
+    k[1] = 0.0
+    k[1, 17] = -3.0                                                 # one non-zero entry
+    k[2] = _e4m3_ties_row()                                         # scale 1: the ties themselves round
+    k[3] = -k[2]
+    if k_bf16:
+        kb = W.bf16_encode(k)
+        assert np.array_equal(oracle.bf16_decode(kb[2]), k[2])     # the ties survive the bf16 encoding
+        return kv_new, kb.view(np.int16), "bf16"
+    return kv_new, k, "f32"
+
+
+def _dev_copy(a, dev):
+    a = np.ascontiguousarray(a)
+    return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a.copy()).to(dev)
+
+
+@pytest.mark.parametrize("k_bf16", [False, True])
+def test_cache_append_matches_oracle(k_bf16):
+    """New tokens written into shuffled pages: a whole 70-token prompt, a 3-token chunk, single decode
+    tokens; latent rows and scales bit-exact, FP8 codes bit-exact (a zero code's sign aside), every
+    other token of the pools untouched."""
+    wl = W.make_workload("append", kind="mla", seed=109, seq_lens=[70, 300, 2100, 1, 65], q_lens=[70, 3, 1, 1, 2],
+                         topk=64, spare_blocks=3)
+    dev = torch.device("cuda")
+    rng = np.random.default_rng(110 + k_bf16)
+    kv_new, k_in, fmt = _append_inputs(wl.total_q, rng, k_bf16)
+    bt, sl, cu = (_dev_copy(a.astype(np.int32), dev) for a in (wl.block_table, wl.seq_lens, wl.cu_q))
+    batch = B.make_batch(bt, sl, cu, num_blocks=wl.num_blocks, page_size=64, total_q=wl.total_q,
+                         max_q_per_seq=wl.max_q_per_seq, max_seq_len=wl.max_seq_len)
+    kv_pool, kI_pool, kS_pool = _dev_copy(wl.kv_pool, dev), _dev_copy(wl.kI_pool, dev), _dev_copy(wl.kS_pool, dev)
+    ws = torch.zeros(B.dsa_workspace_size(B.DSA_OP_CACHE_APPEND, batch), dtype=torch.uint8, device=dev)
+    n0 = B.dsa_launch_count()
+    B.dsa_cache_append(_dev_copy(kv_new, dev), B.DSA_BF16, _dev_copy(k_in, dev), B.DSA_BF16 if k_bf16 else B.DSA_F32,
+                       576, 128, batch, kv_pool, kI_pool, kS_pool, ws, ws.numel())
+    torch.cuda.synchronize()
+    B.dsa_read_device_status(ws)
+    assert B.dsa_launch_count() == n0 + 1
+    k_oracle = k_in.view(np.uint16) if k_bf16 else k_in
+    ekv, ekI, ekS = oracle.cache_append(wl, kv_new.view(np.uint16), k_oracle, fmt)
+    assert np.array_equal(kv_pool.cpu().numpy().view(np.uint16), ekv)
+    assert np.array_equal(kS_pool.cpu().numpy().view(np.uint32), ekS.view(np.uint32))
+    zero = lambda c: np.where((c & 0x7F) == 0, 0, c)
+    assert np.array_equal(zero(kI_pool.cpu().numpy()), zero(ekI))
+
+
+def test_cache_append_reports_bad_block_ids():
+    """A block id outside the pool: those tokens are skipped and the status word says so; the rest of
+    the batch is written."""
+    wl = W.make_workload("append_bad", kind="mla", seed=111, seq_lens=[130, 64], q_lens=[2, 1], topk=64)
+    bt_host = wl.block_table.astype(np.int32).copy()
+    bt_host[0, 2] = wl.num_blocks + 5                               # positions 128, 129 of sequence 0
+    dev = torch.device("cuda")
+    bt, sl, cu = (_dev_copy(a.astype(np.int32), dev) for a in (bt_host, wl.seq_lens, wl.cu_q))
+    batch = B.make_batch(bt, sl, cu, num_blocks=wl.num_blocks, page_size=64, total_q=wl.total_q,
+                         max_q_per_seq=wl.max_q_per_seq, max_seq_len=wl.max_seq_len)
+    kv_pool, kI_pool, kS_pool = _dev_copy(wl.kv_pool, dev), _dev_copy(wl.kI_pool, dev), _dev_copy(wl.kS_pool, dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    kv_new, k_in, _ = _append_inputs(wl.total_q + 4, np.random.default_rng(112), False)
+    B.dsa_cache_append(_dev_copy(kv_new[: wl.total_q], dev), B.DSA_BF16, _dev_copy(k_in[4:], dev), B.DSA_F32, 576, 128,
+                       batch, kv_pool, kI_pool, kS_pool, ws, 256)
+    with pytest.raises(B.DSAError) as e:
+        B.dsa_read_device_status(ws)
+    assert e.value.status == B.DSA_ERR_DEVICE_CHECK
+    changed = np.argwhere((kI_pool.cpu().numpy() != wl.kI_pool).any(axis=2)).tolist()
+    blk, slot = oracle.token_slots(bt_host[1], np.array([63]), 64)
+    assert changed == [[int(blk[0]), int(slot[0])]]                 # only sequence 1's token was written

@@ -63,3 +63,94 @@ def test_two_gloo_ranks_slowest_rank_time_and_weak_scaling_value():
     assert res[0]["shapes"][0][:2] == res[0]["shapes"][1][:2] == [32, 32]
     assert res[0]["seq_lens"] != res[1]["seq_lens"]
     assert np.all(np.asarray(res[0]["seq_lens"]) >= 4096) and np.all(np.asarray(res[1]["seq_lens"]) <= 32768)
+
+
+# ----------------------------------------------------------------------------- overlapped e2e leg
+def _fake_cuda(step_ms):
+    """Stand-ins for the CUDA stream/event calls the overlapped e2e leg makes, so that its multi-rank
+    agreement logic runs on CPU: every recorded event advances a clock by `step_ms`."""
+    import contextlib
+
+    class Ev:
+        clock = 0.0
+
+        def __init__(self, enable_timing=False):
+            self.t = None
+
+        def record(self, stream=None):
+            Ev.clock += step_ms
+            self.t = Ev.clock
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    class St:
+        cuda_stream = 0
+
+        def wait_event(self, ev):
+            pass
+
+    empty = torch.empty
+    torch.empty = lambda *a, pin_memory=False, **k: empty(*a, **k)
+    torch.cuda.Stream = lambda device=None: St()
+    torch.cuda.Event = Ev
+    torch.cuda.stream = lambda s: contextlib.nullcontext()
+    torch.cuda.synchronize = lambda device=None: None
+
+
+class _FakeBatch:
+    def __init__(self):
+        self.inputs = {n: torch.zeros(4, 3) for n in ("q", "qI", "w", "block_table", "seq_lens", "cu_q")}
+        self.out = torch.zeros(2, 8, dtype=torch.bfloat16)
+        self.lse = torch.zeros(2, 8)
+        self.n = 0
+
+    def run(self, stream):
+        self.n += 1
+        self.out.fill_(self.n)
+        self.lse.fill_(self.n)
+
+
+def _e2e_rank_main(rank, world, port, results, sets_per_rank):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import types
+        import bench
+        _fake_cuda(step_ms=1.0 + rank)                         # rank 1 is the slower one
+        args = types.SimpleNamespace(steps=6, warmup=3)
+        wl = types.SimpleNamespace(total_q=32)
+        sets = [_FakeBatch() for _ in range(sets_per_rank[rank])]
+        res = bench.run_e2e_overlapped(args, wl, sets, "cpu", world)
+        results[rank] = None if res is None else {"ms_per_step": res["ms_per_step"], "value": res["value"]}
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("sets_per_rank", [(2, 2), (2, 1)])
+def test_overlapped_e2e_ranks_agree(sets_per_rank):
+    """Both ranks report the slowest rank's time, or both drop the overlapped leg when one rank cannot
+    run it (so that neither waits in a collective the other never enters)."""
+    world = 2
+    port = 31500 + (os.getpid() % 2000) + 7 * sets_per_rank[1]
+    with mp.Manager() as mgr:
+        results = mgr.dict()
+        ctx = mp.get_context("spawn")
+        procs = [ctx.Process(target=_e2e_rank_main, args=(r, world, port, results, sets_per_rank))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(120)
+            assert p.exitcode == 0, f"rank process exited with {p.exitcode}"
+        res = dict(results)
+    assert set(res) == {0, 1}
+    if sets_per_rank == (2, 1):
+        assert res[0] is None and res[1] is None
+    else:
+        assert res[0] == res[1]
+        # the timed region spans 3 events per step for 6 steps plus the closing one; rank 1's events are
+        # 2 ms apart (rank 0's 1 ms), so the job's time is rank 1's: 19 * 2 ms over 6 steps
+        assert res[0]["ms_per_step"] == pytest.approx(19 * 2.0 / 6)
+        assert res[0]["value"] == pytest.approx(2 * 32 / (res[0]["ms_per_step"] / 1e3))

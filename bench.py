@@ -77,6 +77,23 @@ def work_of(wl):
                 attention=dict(bytes=attn_bytes, flops=attn_flops), tokens=T, selected_rows=attn_rows)
 
 
+def step_roofline(work, peaks, ms_per_step):
+    """Roofline of one whole step: T_roof = max(fp8 flops / P_fp8 + bf16 flops / P_bf16, bytes / BW) over
+    the indexer and the attention (the scores / idx round trip between stages is not credited), with
+    the measured HBM copy bandwidth, the burst bf16 GEMM peak and FP8 at twice bf16; frac = T_roof over
+    the measured step time."""
+    bf16 = peaks["bf16_tflops"] * 1e12
+    fp8 = 2.0 * bf16
+    bw = peaks["hbm_gbs"] * 1e9
+    nbytes = work["indexer"]["bytes"] + work["attention"]["bytes"]
+    t_flops = work["indexer"]["flops"] / fp8 + work["attention"]["flops"] / bf16
+    t_bytes = nbytes / bw
+    t = max(t_flops, t_bytes)
+    return {"t_roof_us": t * 1e6, "bound": "hbm" if t_bytes >= t_flops else "tensor", "frac": t / (ms_per_step / 1e3),
+            "bytes": nbytes, "flops_fp8": work["indexer"]["flops"], "flops_bf16": work["attention"]["flops"],
+            "peaks": "hbm_gbs, bf16_tflops (burst), fp8 = 2 x bf16"}
+
+
 # ---------------------------------------------------------------------------------------------- clocks
 class ClockSampler:
     """Polls NVML for SM clock and throttle reasons in a background thread."""
@@ -254,6 +271,8 @@ def run_ours(args, rank, world, local_rank):
         "stages_ms": stage_avg, "roofline": roof, "e2e": e2e, "gpu_launches": int(launches),
         "clocks": clocks, "impl": "ours",
     }
+    if wl.kind == "mla":
+        res["step_roofline"] = step_roofline(work, peaks, ms_per_step)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     return res

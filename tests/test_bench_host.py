@@ -1,0 +1,40 @@
+"""Host-side accounting of bench.py (no GPU): the algorithmic bytes and flops credited per stage follow the
+definitions (each causal indexer key once, each selected latent row once, plus q, w and out), and the
+whole-step roofline combines them as max(fp8 / P_fp8 + bf16 / P_bf16, bytes / BW)."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from sparse_attention_long_dsa_b200 import workloads as W  # noqa: E402
+
+
+def test_work_of_two_decode_rows_by_hand():
+    # contexts 100 and 3000, one query each (the last token), top-k 2048
+    wl = W.make_workload("acct", kind="mla", seed=1, seq_lens=[100, 3000], q_lens=[1, 1], topk=2048)
+    w = bench.work_of(wl)
+    keys = 100 + 3000                                  # causal indexer keys, 128 e4m3 + 4-byte scale each
+    assert w["indexer"]["bytes"] == keys * 132 + 2 * 64 * (128 + 4)      # + qI rows and w
+    assert w["indexer"]["flops"] == keys * 2 * 64 * 128
+    rows = 100 + 2048                                  # selected latent rows (all 100 of the short context)
+    assert w["selected_rows"] == rows
+    assert w["attention"]["bytes"] == rows * 1152 + 2 * 128 * (576 * 2 + 512 * 2)   # + q and out, bf16
+    assert w["attention"]["flops"] == rows * 2 * 128 * (576 + 512)
+    assert w["topk"]["bytes"] == keys * 4 + 2 * 2048 * 4
+
+
+def test_step_roofline_tensor_and_hbm_bound():
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 100.0, "bf16_tflops_sustained": 90.0}
+    work = {"indexer": {"bytes": 1e9, "flops": 2e12}, "topk": {"bytes": 5e9, "flops": 0.0},
+            "attention": {"bytes": 1e9, "flops": 1e12}}
+    r = bench.step_roofline(work, peaks, 40.0)
+    # fp8 at 200 TF/s: 10 ms; bf16: 10 ms; bytes 2 GB (top-k's round trip not credited) at 1 TB/s: 2 ms
+    assert r["bound"] == "tensor" and r["t_roof_us"] == pytest.approx(20e3) and r["frac"] == pytest.approx(0.5)
+    work["attention"]["bytes"] = 29e9
+    r = bench.step_roofline(work, peaks, 60.0)
+    assert r["bound"] == "hbm" and r["t_roof_us"] == pytest.approx(30e3) and r["frac"] == pytest.approx(0.5)

@@ -16,6 +16,30 @@ def _dev(a, device):
     return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device)
 
 
+def check_inputs_finite(wl) -> None:
+    """Optional host pre-check of a workload's inputs: the library requires finite values (and positive key
+    scales) and does not test them on the device.  Raises ValueError naming the first offending array.
+    bf16 and fp32 values are checked by their exponent bits, E4M3 codes by the two NaN codes (0x7F, 0xFF)."""
+    def bad(name, mask):
+        if np.any(mask):
+            raise ValueError(f"input {name} holds {int(np.count_nonzero(mask))} non-finite value(s)")
+
+    fp8 = wl.kind == "mla"
+    for name in ("q", "kv_pool", "v_pool", "qI", "kI_pool", "w", "kS_pool"):
+        a = getattr(wl, name, None)
+        if a is None:
+            continue
+        a = np.asarray(a)
+        if a.dtype == np.uint16:                                   # bf16 bits
+            bad(name, (a & 0x7F80) == 0x7F80)
+        elif a.dtype == np.uint8 and fp8:                          # e4m3 codes
+            bad(name, (a & 0x7F) == 0x7F)
+        else:
+            bad(name, ~np.isfinite(a.astype(np.float32, copy=False)))
+    if getattr(wl, "kS_pool", None) is not None and np.any(np.asarray(wl.kS_pool) <= 0):
+        raise ValueError("input kS_pool holds a key scale <= 0")
+
+
 class DeviceBatch:
     """One workload resident in HBM plus its outputs.
 
@@ -24,7 +48,7 @@ class DeviceBatch:
     query row) over dsa_sparse_attn_prefill; default: decode when that holds.
     """
 
-    def __init__(self, wl, device="cuda", decode=None, inputs=None):
+    def __init__(self, wl, device="cuda", decode=None, inputs=None, check_finite=False):
         self.wl = wl
         self.device = torch.device(device)
         dv = self.device
@@ -32,6 +56,8 @@ class DeviceBatch:
         self.mla = mla
         self.dt = B.DSA_BF16 if mla else B.DSA_F32
         self.idx_dt = B.DSA_FP8_E4M3 if mla else B.DSA_F32
+        if check_finite:
+            check_inputs_finite(wl)
         if inputs is None:
             inputs = self.upload_inputs(wl, dv)
         self.inputs = inputs

@@ -134,3 +134,23 @@ def test_cache_append_rejects_before_launch():
             B.dsa_cache_append(a["kv_new"], a["kv_dt"], a["k_new"], a["k_dt"], a["Dqk"], a["Di"], b, a["kv_pool"],
                                a["k_idx_pool"], a["k_scale_pool"], a["ws"], a["ws_bytes"], 0)
         assert e.value.status == status, bad
+
+
+def test_host_precheck_rejects_non_finite_inputs():
+    """The optional host pre-check names the first array holding a NaN / Inf (bf16 bits, E4M3 NaN codes,
+    fp32) or a non-positive key scale; clean workloads pass."""
+    from sparse_attention_long_dsa_b200 import workloads as W
+    from sparse_attention_long_dsa_b200.pipeline import check_inputs_finite
+    wl = W.make_workload("chk", kind="mla", seed=3, seq_lens=[130, 70], q_lens=[2, 1], topk=64)
+    check_inputs_finite(wl)
+    check_inputs_finite(W.tiny_f32())
+    plants = [("q", 0x7FC0), ("kv_pool", 0xFF80), ("qI", 0x7F), ("kI_pool", 0xFF), ("w", np.nan), ("kS_pool", np.inf),
+              ("kS_pool", 0.0)]
+    for name, val in plants:
+        a = getattr(wl, name)
+        keep = a.flat[5]
+        a.flat[5] = val
+        with pytest.raises(ValueError, match=name):
+            check_inputs_finite(wl)
+        a.flat[5] = keep
+    check_inputs_finite(wl)

@@ -297,7 +297,7 @@ def workload_config(wl, args):
 # ncu capture (profiles/), valid only while the kernel's sources are the ones that were captured.
 MEASURED_TRAFFIC = {
     ("attention", "decode_batch"): {"bytes": 84244992 + 4310784,
-                                    "sources": ("attn_mla_tc.cu", "tc.cuh", "common.cuh"), "sha256_16": "00dad19e2a1db298"},
+                                    "sources": ("attn_mla_tc.cu", "tc.cuh", "common.cuh"), "sha256_16": "ee6a0cc8aa2fe8fa"},
 }
 
 

@@ -211,6 +211,14 @@ DSA_API dsa_status_t dsa_cache_append(const void *kv_new, dsa_dtype_t kv_dt, con
  * workspace used by the calls above: DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK. */
 DSA_API dsa_status_t dsa_read_device_status(void *ws, void *stream);
 
+/* Self-test of the bounded device waits: enqueues one kernel whose thread waits on an mbarrier that
+ * nothing completes, through the wait routine every tensor-core kernel uses, with a budget of
+ * `budget_cycles` SM cycles (1 .. 4e9; the kernels' own budget is 8e9).  The wait gives up, sets the
+ * timeout bit of the workspace status word (ws: at least 256 bytes, 256-byte aligned) and the kernel
+ * returns, so dsa_read_device_status(ws) then reports DSA_ERR_TIMEOUT and the context stays usable.
+ * No GPU fault is involved. */
+DSA_API dsa_status_t dsa_selftest_wait_timeout(uint64_t budget_cycles, void *ws, size_t ws_bytes, void *stream);
+
 DSA_API const char *dsa_status_string(dsa_status_t s);
 DSA_API const char *dsa_last_error(void);
 

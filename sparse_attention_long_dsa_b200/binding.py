@@ -21,7 +21,7 @@ DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_ATTN_PREFILL, DSA_OP_ATTN_DECODE, DSA_OP_CAC
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn_prefill",
            "dsa_sparse_attn_decode", "dsa_read_device_status", "dsa_status_string", "dsa_last_error",
-           "dsa_version", "dsa_launch_count", "dsa_topk_noalloc", "dsa_cache_append")
+           "dsa_version", "dsa_launch_count", "dsa_topk_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout")
 
 
 class dsa_batch_t(ctypes.Structure):
@@ -67,6 +67,7 @@ def load(path: str = LIB_PATH):
         "dsa_sparse_attn_prefill": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
         "dsa_sparse_attn_decode": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
         "dsa_cache_append": [P, I32, P, I32, I32, I32, B, P, P, P, P, SZ, P],
+        "dsa_selftest_wait_timeout": [ctypes.c_uint64, P, SZ, P],
         "dsa_read_device_status": [P, P],
     }
     for name, args in sig.items():
@@ -160,6 +161,11 @@ def dsa_cache_append(kv_new, kv_dt: int, k_new, k_dt: int, Dqk: int, Di: int, ba
     _check(load().dsa_cache_append(_ptr(kv_new), kv_dt, _ptr(k_new), k_dt, Dqk, Di, ctypes.byref(batch), _ptr(kv_pool),
                                    _ptr(k_idx_pool), _ptr(k_scale_pool), _ptr(ws), ws_bytes, _stream(stream)),
            "dsa_cache_append")
+
+
+def dsa_selftest_wait_timeout(budget_cycles: int, ws, ws_bytes: int, stream=None):
+    _check(load().dsa_selftest_wait_timeout(budget_cycles, _ptr(ws), ws_bytes, _stream(stream)),
+           "dsa_selftest_wait_timeout")
 
 
 def dsa_read_device_status(ws, stream=None):

@@ -29,6 +29,7 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
 size_t attn_workspace_bytes(int T, int k, bool decode);
 dsa_status_t cache_append_launch(const void *kv_new, const void *k_new, bool k_bf16, const dsa_batch_t *b,
                                  void *kv_pool, void *kI_pool, float *kS_pool, void *ws, cudaStream_t stream);
+dsa_status_t selftest_wait_launch(long long budget, void *ws, cudaStream_t stream);
 dsa_status_t attn_simt_launch(const void *q, dsa_dtype_t dt, const void *kv, const void *v, int H, int Dqk, int Dv,
                               float scale, const int32_t *idx, int k, const dsa_batch_t *b, void *out, float *lse,
                               cudaStream_t stream);
@@ -299,6 +300,16 @@ dsa_status_t dsa_cache_append(const void *kv_new, dsa_dtype_t kv_dt, const void 
   if ((st = current_device(&dev)) != DSA_OK) return st;
   return cache_append_launch(kv_new, k_new, k_dt == DSA_BF16, b, kv_pool, k_idx_pool, k_scale_pool, ws,
                              (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_selftest_wait_timeout(uint64_t budget_cycles, void *ws, size_t ws_bytes, void *stream) {
+  CHECK_ARG(budget_cycles >= 1 && budget_cycles <= 4000000000ull,
+            "budget_cycles must be in [1, 4e9] (got %llu)", (unsigned long long)budget_cycles);
+  dsa_status_t st = check_ws(ws, ws_bytes, kWsHeader);
+  if (st != DSA_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return selftest_wait_launch((long long)budget_cycles, ws, (cudaStream_t)stream);
 }
 
 dsa_status_t dsa_read_device_status(void *ws, void *stream) {

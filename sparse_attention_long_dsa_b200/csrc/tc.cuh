@@ -39,7 +39,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // another role has raised `abort`.  On giving up it raises `abort` and the workspace timeout bit.
 constexpr long long kWaitBudget = 8000000000LL;
 
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int *abort, uint32_t *status,
+                                              long long budget) {
   if (mbar_try_wait(bar, parity)) return true;
   if (*abort) return false;
   const long long t0 = clock64();
@@ -47,13 +48,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0u) {
       if (*abort) return false;
-      if (clock64() - t0 > kWaitBudget) {
+      if (clock64() - t0 > budget) {
         *abort = 1;
         set_status(status, kStatusTimeout);
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+  return mbar_wait_for(bar, parity, abort, status, kWaitBudget);
 }
 
 // ------------------------------------------------------------------------------------------ copies

@@ -154,3 +154,12 @@ def test_host_precheck_rejects_non_finite_inputs():
             check_inputs_finite(wl)
         a.flat[5] = keep
     check_inputs_finite(wl)
+
+
+def test_wait_selftest_rejects_before_launch():
+    P = 1 << 24
+    for budget, ws_bytes, status in [(0, 256, B.DSA_ERR_INVALID_ARG), (5_000_000_000, 256, B.DSA_ERR_INVALID_ARG),
+                                     (1000, 128, B.DSA_ERR_WORKSPACE)]:
+        with pytest.raises(B.DSAError) as e:
+            B.dsa_selftest_wait_timeout(budget, P, ws_bytes, 0)
+        assert e.value.status == status

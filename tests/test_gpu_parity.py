@@ -339,3 +339,23 @@ def test_cache_append_reports_bad_block_ids():
     changed = np.argwhere((kI_pool.cpu().numpy() != wl.kI_pool).any(axis=2)).tolist()
     blk, slot = oracle.token_slots(bt_host[1], np.array([63]), 64)
     assert changed == [[int(blk[0]), int(slot[0])]]                 # only sequence 1's token was written
+
+
+# --------------------------------------------------------------------------------------- bounded waits
+def test_bounded_wait_gives_up_and_reports_timeout():
+    """A device wait on a barrier that nothing completes (the wait routine of the tensor-core kernels, with a
+    budget of 2e7 SM cycles) gives up and raises the timeout bit; reading the status clears it, and the
+    context still runs a batch that matches the oracle."""
+    import time
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    t0 = time.time()
+    B.dsa_selftest_wait_timeout(20_000_000, ws, 256)
+    with pytest.raises(B.DSAError) as e:
+        B.dsa_read_device_status(ws)
+    assert e.value.status == B.DSA_ERR_TIMEOUT
+    assert time.time() - t0 < 60
+    B.dsa_read_device_status(ws)                                    # cleared by the read
+    wl = W.make_workload("after_timeout", kind="mla", seed=113, seq_lens=[300, 2100], q_lens=[1, 1], topk=2048,
+                         grid=True)
+    db = _run(wl)
+    compare_rows(wl, db, list(range(wl.total_q)))

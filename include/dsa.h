@@ -211,6 +211,33 @@ DSA_API dsa_status_t dsa_cache_append(const void *kv_new, dsa_dtype_t kv_dt, con
  * workspace used by the calls above: DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK. */
 DSA_API dsa_status_t dsa_read_device_status(void *ws, void *stream);
 
+/* Context-parallel decode ("Engineering Practices ...", Four Key Layers 3: partial attention over
+ * disjoint key sets merged by a log-sum-exp reduction, here across GPUs).  Every sequence of a decode
+ * batch (one query row per sequence, T rows) is spread over G ranks, rank r holding the contiguous token
+ * range [lo[t], hi[t]) of row t's sequence, ranks in ascending order of their ranges.  Each rank runs
+ * dsa_indexer_scores and dsa_topk on a batch of its own ranges (local positions), then:
+ *
+ * dsa_cp_candidates: cand_score[t, j] = scores[t, idx[t, j]], cand_gidx[t, j] = idx[t, j] + offsets[t]
+ *   (offsets = lo); idx entries outside [0, ld_scores) give (-inf, -1).  All arrays [T, k], device.
+ * After an all-gather of both into [G, T, k]:
+ * dsa_cp_rows: rows[t, r*k + j] = g_score[r, t, j], rows [T, ld_rows], ld_rows >= G*k.  dsa_topk over these
+ *   rows (a batch of T sequences of G*k candidates, one query row each) picks the global top-k; ties go
+ *   to the lower candidate position, which is the lower global position.
+ * dsa_cp_select_local: local_idx[t, j] = g - lo[t] where g = g_gidx[p / k, t, p % k] for p = sel[t, j],
+ *   if lo[t] <= g < hi[t], else -1.  dsa_sparse_attn_decode over local_idx gives this rank's o_r, lse_r.
+ * After an all-gather of those into part_out [G, T, H, Dv] (bf16) and part_lse [G, T, H]:
+ * dsa_cp_merge: lse = log sum_r exp(lse_r), out = sum_r exp(lse_r - lse) o_r in fp32, stored as bf16;
+ *   ranks with lse_r = -inf contribute nothing; lse may be NULL.
+ * Each call only enqueues; T = 0 returns DSA_OK at once. */
+DSA_API dsa_status_t dsa_cp_candidates(const float *scores, int64_t ld_scores, const int32_t *idx, int32_t T, int32_t k,
+                                       const int32_t *offsets, float *cand_score, int32_t *cand_gidx, void *stream);
+DSA_API dsa_status_t dsa_cp_rows(const float *g_score, int32_t G, int32_t T, int32_t k, float *rows, int64_t ld_rows,
+                                 void *stream);
+DSA_API dsa_status_t dsa_cp_select_local(const int32_t *sel, const int32_t *g_gidx, int32_t G, int32_t T, int32_t k,
+                                         const int32_t *lo, const int32_t *hi, int32_t *local_idx, void *stream);
+DSA_API dsa_status_t dsa_cp_merge(const void *part_out, dsa_dtype_t dt, const float *part_lse, int32_t G, int32_t T,
+                                  int32_t H, int32_t Dv, void *out, float *lse, void *stream);
+
 /* Self-test of the bounded device waits: enqueues one kernel whose thread waits on an mbarrier that
  * nothing completes, through the wait routine every tensor-core kernel uses, with a budget of
  * `budget_cycles` SM cycles (1 .. 4e9; the kernels' own budget is 8e9).  The wait gives up, sets the

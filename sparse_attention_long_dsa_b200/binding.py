@@ -21,7 +21,8 @@ DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_ATTN_PREFILL, DSA_OP_ATTN_DECODE, DSA_OP_CAC
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn_prefill",
            "dsa_sparse_attn_decode", "dsa_read_device_status", "dsa_status_string", "dsa_last_error",
-           "dsa_version", "dsa_launch_count", "dsa_topk_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout")
+           "dsa_version", "dsa_launch_count", "dsa_topk_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout",
+           "dsa_cp_candidates", "dsa_cp_rows", "dsa_cp_select_local", "dsa_cp_merge")
 
 
 class dsa_batch_t(ctypes.Structure):
@@ -68,6 +69,10 @@ def load(path: str = LIB_PATH):
         "dsa_sparse_attn_decode": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
         "dsa_cache_append": [P, I32, P, I32, I32, I32, B, P, P, P, P, SZ, P],
         "dsa_selftest_wait_timeout": [ctypes.c_uint64, P, SZ, P],
+        "dsa_cp_candidates": [P, I64, P, I32, I32, P, P, P, P],
+        "dsa_cp_rows": [P, I32, I32, I32, P, I64, P],
+        "dsa_cp_select_local": [P, P, I32, I32, I32, P, P, P, P],
+        "dsa_cp_merge": [P, I32, P, I32, I32, I32, I32, P, P, P],
         "dsa_read_device_status": [P, P],
     }
     for name, args in sig.items():
@@ -166,6 +171,25 @@ def dsa_cache_append(kv_new, kv_dt: int, k_new, k_dt: int, Dqk: int, Di: int, ba
 def dsa_selftest_wait_timeout(budget_cycles: int, ws, ws_bytes: int, stream=None):
     _check(load().dsa_selftest_wait_timeout(budget_cycles, _ptr(ws), ws_bytes, _stream(stream)),
            "dsa_selftest_wait_timeout")
+
+
+def dsa_cp_candidates(scores, ld_scores: int, idx, T: int, k: int, offsets, cand_score, cand_gidx, stream=None):
+    _check(load().dsa_cp_candidates(_ptr(scores), ld_scores, _ptr(idx), T, k, _ptr(offsets), _ptr(cand_score),
+                                    _ptr(cand_gidx), _stream(stream)), "dsa_cp_candidates")
+
+
+def dsa_cp_rows(g_score, G: int, T: int, k: int, rows, ld_rows: int, stream=None):
+    _check(load().dsa_cp_rows(_ptr(g_score), G, T, k, _ptr(rows), ld_rows, _stream(stream)), "dsa_cp_rows")
+
+
+def dsa_cp_select_local(sel, g_gidx, G: int, T: int, k: int, lo, hi, local_idx, stream=None):
+    _check(load().dsa_cp_select_local(_ptr(sel), _ptr(g_gidx), G, T, k, _ptr(lo), _ptr(hi), _ptr(local_idx),
+                                      _stream(stream)), "dsa_cp_select_local")
+
+
+def dsa_cp_merge(part_out, dt: int, part_lse, G: int, T: int, H: int, Dv: int, out, lse, stream=None):
+    _check(load().dsa_cp_merge(_ptr(part_out), dt, _ptr(part_lse), G, T, H, Dv, _ptr(out), _ptr(lse),
+                               _stream(stream)), "dsa_cp_merge")
 
 
 def dsa_read_device_status(ws, stream=None):

@@ -30,6 +30,14 @@ size_t attn_workspace_bytes(int T, int k, bool decode);
 dsa_status_t cache_append_launch(const void *kv_new, const void *k_new, bool k_bf16, const dsa_batch_t *b,
                                  void *kv_pool, void *kI_pool, float *kS_pool, void *ws, cudaStream_t stream);
 dsa_status_t selftest_wait_launch(long long budget, void *ws, cudaStream_t stream);
+dsa_status_t cp_candidates_launch(const float *scores, int64_t ld, const int32_t *idx, int T, int k,
+                                  const int32_t *offsets, float *cand_score, int32_t *cand_gidx, cudaStream_t stream);
+dsa_status_t cp_rows_launch(const float *g_score, int G, int T, int k, float *rows, int64_t ld_rows,
+                            cudaStream_t stream);
+dsa_status_t cp_select_local_launch(const int32_t *sel, const int32_t *g_gidx, int G, int T, int k, const int32_t *lo,
+                                    const int32_t *hi, int32_t *local, cudaStream_t stream);
+dsa_status_t cp_merge_launch(const void *part_out, const float *part_lse, int G, int T, int H, int Dv, void *out,
+                             float *lse, cudaStream_t stream);
 dsa_status_t attn_simt_launch(const void *q, dsa_dtype_t dt, const void *kv, const void *v, int H, int Dqk, int Dv,
                               float scale, const int32_t *idx, int k, const dsa_batch_t *b, void *out, float *lse,
                               cudaStream_t stream);
@@ -310,6 +318,55 @@ dsa_status_t dsa_selftest_wait_timeout(uint64_t budget_cycles, void *ws, size_t 
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
   return selftest_wait_launch((long long)budget_cycles, ws, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_cp_candidates(const float *scores, int64_t ld_scores, const int32_t *idx, int32_t T, int32_t k,
+                               const int32_t *offsets, float *cand_score, int32_t *cand_gidx, void *stream) {
+  CHECK_ARG(T >= 0 && k >= 1 && ld_scores >= 1, "T must be >= 0, k and ld_scores >= 1");
+  if (T == 0) return DSA_OK;
+  CHECK_ARG(scores && idx && offsets && cand_score && cand_gidx, "scores, idx, offsets, cand_score and cand_gidx are required");
+  DeviceInfo dev;
+  dsa_status_t st;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return cp_candidates_launch(scores, ld_scores, idx, T, k, offsets, cand_score, cand_gidx, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_cp_rows(const float *g_score, int32_t G, int32_t T, int32_t k, float *rows, int64_t ld_rows,
+                         void *stream) {
+  CHECK_ARG(G >= 1 && T >= 0 && k >= 1, "G and k must be >= 1, T >= 0");
+  CHECK_ARG(ld_rows >= (int64_t)G * k, "ld_rows (%lld) must be >= G * k", (long long)ld_rows);
+  if (T == 0) return DSA_OK;
+  CHECK_ARG(g_score && rows, "g_score and rows are required");
+  DeviceInfo dev;
+  dsa_status_t st;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return cp_rows_launch(g_score, G, T, k, rows, ld_rows, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_cp_select_local(const int32_t *sel, const int32_t *g_gidx, int32_t G, int32_t T, int32_t k,
+                                 const int32_t *lo, const int32_t *hi, int32_t *local_idx, void *stream) {
+  CHECK_ARG(G >= 1 && T >= 0 && k >= 1, "G and k must be >= 1, T >= 0");
+  CHECK_ARG((int64_t)G * k <= 0x7FFFFFFF, "G * k must fit in int32");
+  if (T == 0) return DSA_OK;
+  CHECK_ARG(sel && g_gidx && lo && hi && local_idx, "sel, g_gidx, lo, hi and local_idx are required");
+  DeviceInfo dev;
+  dsa_status_t st;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return cp_select_local_launch(sel, g_gidx, G, T, k, lo, hi, local_idx, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_cp_merge(const void *part_out, dsa_dtype_t dt, const float *part_lse, int32_t G, int32_t T, int32_t H,
+                          int32_t Dv, void *out, float *lse, void *stream) {
+  CHECK_ARG(G >= 1 && T >= 0 && H >= 1 && H <= 65535, "G and H must be >= 1 (H <= 65535), T >= 0");
+  CHECK_SUP(dt == DSA_BF16 && Dv >= 4 && Dv <= 1024 && Dv % 4 == 0,
+            "merge supports bf16 partial outputs with Dv a multiple of 4 in [4, 1024]");
+  if (T == 0) return DSA_OK;
+  CHECK_ARG(part_out && part_lse && out, "part_out, part_lse and out are required");
+  CHECK_ARG((((uintptr_t)part_out | (uintptr_t)out) & 7) == 0, "part_out and out must be 8-byte aligned");
+  DeviceInfo dev;
+  dsa_status_t st;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return cp_merge_launch(part_out, part_lse, G, T, H, Dv, out, lse, (cudaStream_t)stream);
 }
 
 dsa_status_t dsa_read_device_status(void *ws, void *stream) {

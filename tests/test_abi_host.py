@@ -163,3 +163,26 @@ def test_wait_selftest_rejects_before_launch():
         with pytest.raises(B.DSAError) as e:
             B.dsa_selftest_wait_timeout(budget, P, ws_bytes, 0)
         assert e.value.status == status
+
+
+def test_context_parallel_entries_validate_before_launch():
+    P = 1 << 24
+    # empty batches are no-ops without a device
+    B.dsa_cp_candidates(None, 128, None, 0, 16, None, None, None, 0)
+    B.dsa_cp_rows(None, 2, 0, 16, None, 32, 0)
+    B.dsa_cp_select_local(None, None, 2, 0, 16, None, None, None, 0)
+    B.dsa_cp_merge(None, B.DSA_BF16, None, 2, 0, 128, 512, None, None, 0)
+    bad = [
+        (lambda: B.dsa_cp_candidates(P, 128, P, 2, 0, P, P, P, 0), B.DSA_ERR_INVALID_ARG),        # k = 0
+        (lambda: B.dsa_cp_candidates(P, 128, None, 2, 16, P, P, P, 0), B.DSA_ERR_INVALID_ARG),    # NULL idx
+        (lambda: B.dsa_cp_rows(P, 0, 2, 16, P, 32, 0), B.DSA_ERR_INVALID_ARG),                     # G = 0
+        (lambda: B.dsa_cp_rows(P, 2, 2, 16, P, 31, 0), B.DSA_ERR_INVALID_ARG),                     # ld < G*k
+        (lambda: B.dsa_cp_select_local(P, P, 2, 2, 16, None, P, P, 0), B.DSA_ERR_INVALID_ARG),     # NULL lo
+        (lambda: B.dsa_cp_merge(P, B.DSA_F32, P, 2, 2, 128, 512, P, P, 0), B.DSA_ERR_UNSUPPORTED),  # f32 parts
+        (lambda: B.dsa_cp_merge(P, B.DSA_BF16, P, 2, 2, 128, 6, P, P, 0), B.DSA_ERR_UNSUPPORTED),   # Dv % 4
+        (lambda: B.dsa_cp_merge(P + 2, B.DSA_BF16, P, 2, 2, 128, 512, P, P, 0), B.DSA_ERR_INVALID_ARG),  # align
+    ]
+    for call, status in bad:
+        with pytest.raises(B.DSAError) as e:
+            call()
+        assert e.value.status == status

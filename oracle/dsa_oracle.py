@@ -36,6 +36,13 @@ What each step follows (page titles and sections of the source pages):
   o = sum p V / sum p, lse = m + ln(sum p).
 * Split combine -- "Engineering Practices ...", Four Key Layers 3 (partial
   results over candidate KV blocks followed by a cross-block reduction).
+* Block-granular selection -- "Day-0 Adaptation: Running Trillion-Parameter
+  Models on Domestic AI Accelerators", 3.1 (the selection operator's top-k
+  counts key-value blocks): a page's score is taken as the largest token
+  score in it (the pages do not say how token scores make a block score),
+  the best kb pages are kept with ties to the lower page, and attention runs
+  over all their causal tokens.  An approximation of the token-granular
+  path, with this oracle of its own.
 * Cache append -- "Engineering Practices ...", Four Key Layers 3 (the decode
   step writes the new token into the KV cache, merged with its attention
   launch) and 2 (the block table places a token in its block); the indexer
@@ -220,6 +227,33 @@ def topk_row(scores: np.ndarray, k: int) -> np.ndarray:
         sel = np.sort(order[:k])
     out = np.full(k, -1, dtype=np.int32)
     out[: sel.size] = sel
+    return out
+
+
+def block_scores_row(scores: np.ndarray, page_size: int) -> np.ndarray:
+    """Score of each page of a row's candidates: the largest token score in it (the last page may be
+    partial)."""
+    scores = np.asarray(scores, dtype=np.float64)
+    n = scores.size
+    nb = (n + page_size - 1) // page_size
+    padded = np.full(nb * page_size, -np.inf)
+    padded[:n] = scores
+    return padded.reshape(nb, page_size).max(axis=1)
+
+
+def block_topk_row(scores: np.ndarray, kb: int, page_size: int) -> np.ndarray:
+    """Block-granular selection: the kb best pages by block score (ties to the lower page, every page when
+    there are at most kb), each expanded to its token positions.  Selected page i (in ascending page order)
+    fills entries [i*page_size, (i+1)*page_size) with its positions, -1 past the last candidate; unused
+    entries are -1.  Length kb*page_size."""
+    n = np.asarray(scores).size
+    pages = topk_row(block_scores_row(scores, page_size), kb)
+    out = np.full(kb * page_size, -1, dtype=np.int32)
+    for i, p in enumerate(pages):
+        if p < 0:
+            continue
+        pos = p * page_size + np.arange(page_size)
+        out[i * page_size: (i + 1) * page_size] = np.where(pos < n, pos, -1)
     return out
 
 

@@ -412,3 +412,43 @@ def test_cache_append_places_tokens_by_hand():
     assert np.array_equal(kv[~touched], case.kv_pool[~touched])
     assert np.array_equal(kI[~touched], case.kI_pool[~touched])
     assert np.array_equal(kS[~touched], case.kS_pool[~touched])
+
+
+# ----------------------------------------------------------------------------- block-granular selection
+
+def test_block_topk_hand():
+    g = _golden("block_topk_hand.json")
+    for c in g["cases"]:
+        sc = np.array(c["scores"], dtype=np.float64)
+        assert oracle.block_scores_row(sc, c["page"]).tolist() == c["block_scores"], c["note"]
+        assert oracle.block_topk_row(sc, c["kb"], c["page"]).tolist() == c["positions"], c["note"]
+
+
+def test_block_topk_brute_force():
+    """Independent brute force: page maxima by a Python loop, pages ranked by sorting (-max, page)."""
+    rng = np.random.default_rng(31)
+    for it in range(300):
+        n = int(rng.integers(1, 400))
+        page = int(rng.choice([1, 2, 4, 64]))
+        kb = int(rng.integers(1, 12))
+        sc = (rng.integers(-5, 6, n) if it % 2 else rng.standard_normal(n)).astype(np.float64)
+        maxima = [max(sc[p:p + page]) for p in range(0, n, page)]
+        ranked = sorted(range(len(maxima)), key=lambda p: (-maxima[p], p))[:kb]
+        exp = []
+        for p in sorted(ranked):
+            exp += [x if x < n else -1 for x in range(p * page, p * page + page)]
+        exp += [-1] * (kb * page - len(exp))
+        assert oracle.block_topk_row(sc, kb, page).tolist() == exp
+
+
+def test_block_topk_reduces_to_token_topk():
+    """One-token pages select exactly the token top-k; with every page selected the result is every
+    candidate in order, the token path's layout for k >= n."""
+    rng = np.random.default_rng(32)
+    for _ in range(100):
+        n = int(rng.integers(1, 300))
+        sc = rng.integers(-3, 4, n).astype(np.float64)
+        kb = int(rng.integers(1, 40))
+        assert np.array_equal(oracle.block_topk_row(sc, kb, 1), oracle.topk_row(sc, kb))
+        nb = (n + 63) // 64
+        assert np.array_equal(oracle.block_topk_row(sc, nb, 64), oracle.topk_row(sc, nb * 64))

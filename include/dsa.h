@@ -211,6 +211,23 @@ DSA_API dsa_status_t dsa_cache_append(const void *kv_new, dsa_dtype_t kv_dt, con
  * workspace used by the calls above: DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK. */
 DSA_API dsa_status_t dsa_read_device_status(void *ws, void *stream);
 
+/* Block-granular selection ("Day-0 Adaptation: Running Trillion-Parameter Models on Domestic AI
+ * Accelerators", 3.1: the selection operator's top-k counts key-value blocks).  A variant of the
+ * token-granular path, approximate by design:
+ * dsa_block_scores: for every query row, blk_scores[row, p] = max over the causal tokens s of page p
+ *   (s <= pos(row)) of scores[row, s], for p < ceil((pos + 1) / page_size), and blk_lens[row] = that page
+ *   count.  blk_scores [total_q, ld_blk] f32 (ld_blk >= pages of max_seq_len, multiple of 4, 16-byte
+ *   aligned), blk_lens [total_q] int32.
+ * dsa_topk over blk_scores, with a batch of total_q sequences of blk_lens[row] candidates (one query row
+ *   each, cu_q = 0..total_q), keeps kb pages per row, ties to the lower page.
+ * dsa_expand_blocks: idx[row, i*page_size + j] = blk_idx[row, i]*page_size + j when blk_idx[row, i] is a
+ *   page of the row and that position is <= pos(row), else -1.  idx [total_q, kb*page_size] feeds either
+ *   attention call with k = kb*page_size. */
+DSA_API dsa_status_t dsa_block_scores(const float *scores, int64_t ld_scores, const dsa_batch_t *b, float *blk_scores,
+                                      int64_t ld_blk, int32_t *blk_lens, void *stream);
+DSA_API dsa_status_t dsa_expand_blocks(const int32_t *blk_idx, int32_t kb, const dsa_batch_t *b, int32_t *idx,
+                                       void *stream);
+
 /* Context-parallel decode ("Engineering Practices ...", Four Key Layers 3: partial attention over
  * disjoint key sets merged by a log-sum-exp reduction, here across GPUs).  Every sequence of a decode
  * batch (one query row per sequence, T rows) is spread over G ranks, rank r holding the contiguous token

@@ -22,7 +22,8 @@ DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_ATTN_PREFILL, DSA_OP_ATTN_DECODE, DSA_OP_CAC
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn_prefill",
            "dsa_sparse_attn_decode", "dsa_read_device_status", "dsa_status_string", "dsa_last_error",
            "dsa_version", "dsa_launch_count", "dsa_topk_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout",
-           "dsa_cp_candidates", "dsa_cp_rows", "dsa_cp_select_local", "dsa_cp_merge")
+           "dsa_cp_candidates", "dsa_cp_rows", "dsa_cp_select_local", "dsa_cp_merge", "dsa_block_scores",
+           "dsa_expand_blocks")
 
 
 class dsa_batch_t(ctypes.Structure):
@@ -69,6 +70,8 @@ def load(path: str = LIB_PATH):
         "dsa_sparse_attn_decode": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
         "dsa_cache_append": [P, I32, P, I32, I32, I32, B, P, P, P, P, SZ, P],
         "dsa_selftest_wait_timeout": [ctypes.c_uint64, P, SZ, P],
+        "dsa_block_scores": [P, I64, B, P, I64, P, P],
+        "dsa_expand_blocks": [P, I32, B, P, P],
         "dsa_cp_candidates": [P, I64, P, I32, I32, P, P, P, P],
         "dsa_cp_rows": [P, I32, I32, I32, P, I64, P],
         "dsa_cp_select_local": [P, P, I32, I32, I32, P, P, P, P],
@@ -171,6 +174,16 @@ def dsa_cache_append(kv_new, kv_dt: int, k_new, k_dt: int, Dqk: int, Di: int, ba
 def dsa_selftest_wait_timeout(budget_cycles: int, ws, ws_bytes: int, stream=None):
     _check(load().dsa_selftest_wait_timeout(budget_cycles, _ptr(ws), ws_bytes, _stream(stream)),
            "dsa_selftest_wait_timeout")
+
+
+def dsa_block_scores(scores, ld_scores: int, batch: dsa_batch_t, blk_scores, ld_blk: int, blk_lens, stream=None):
+    _check(load().dsa_block_scores(_ptr(scores), ld_scores, ctypes.byref(batch), _ptr(blk_scores), ld_blk,
+                                   _ptr(blk_lens), _stream(stream)), "dsa_block_scores")
+
+
+def dsa_expand_blocks(blk_idx, kb: int, batch: dsa_batch_t, idx, stream=None):
+    _check(load().dsa_expand_blocks(_ptr(blk_idx), kb, ctypes.byref(batch), _ptr(idx), _stream(stream)),
+           "dsa_expand_blocks")
 
 
 def dsa_cp_candidates(scores, ld_scores: int, idx, T: int, k: int, offsets, cand_score, cand_gidx, stream=None):

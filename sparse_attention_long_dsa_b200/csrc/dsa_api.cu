@@ -30,6 +30,10 @@ size_t attn_workspace_bytes(int T, int k, bool decode);
 dsa_status_t cache_append_launch(const void *kv_new, const void *k_new, bool k_bf16, const dsa_batch_t *b,
                                  void *kv_pool, void *kI_pool, float *kS_pool, void *ws, cudaStream_t stream);
 dsa_status_t selftest_wait_launch(long long budget, void *ws, cudaStream_t stream);
+dsa_status_t block_scores_launch(const float *scores, int64_t ld, const dsa_batch_t *b, float *blk, int64_t ld_blk,
+                                 int32_t *blk_lens, cudaStream_t stream);
+dsa_status_t expand_blocks_launch(const int32_t *blk_idx, int kb, const dsa_batch_t *b, int32_t *idx,
+                                  cudaStream_t stream);
 dsa_status_t cp_candidates_launch(const float *scores, int64_t ld, const int32_t *idx, int T, int k,
                                   const int32_t *offsets, float *cand_score, int32_t *cand_gidx, cudaStream_t stream);
 dsa_status_t cp_rows_launch(const float *g_score, int G, int T, int k, float *rows, int64_t ld_rows,
@@ -318,6 +322,32 @@ dsa_status_t dsa_selftest_wait_timeout(uint64_t budget_cycles, void *ws, size_t 
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
   return selftest_wait_launch((long long)budget_cycles, ws, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_block_scores(const float *scores, int64_t ld_scores, const dsa_batch_t *b, float *blk_scores,
+                              int64_t ld_blk, int32_t *blk_lens, void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
+  CHECK_ARG(scores && blk_scores && blk_lens, "scores, blk_scores and blk_lens are required");
+  CHECK_ARG(ld_scores >= b->max_seq_len, "ld_scores (%lld) must be >= max_seq_len", (long long)ld_scores);
+  CHECK_ARG(ld_blk >= (b->max_seq_len + b->page_size - 1) / b->page_size && ld_blk % 4 == 0,
+            "ld_blk (%lld) must be >= the pages of max_seq_len and a multiple of 4", (long long)ld_blk);
+  CHECK_ARG(((uintptr_t)blk_scores & 15) == 0, "blk_scores must be 16-byte aligned");
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return block_scores_launch(scores, ld_scores, b, blk_scores, ld_blk, blk_lens, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_expand_blocks(const int32_t *blk_idx, int32_t kb, const dsa_batch_t *b, int32_t *idx, void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
+  CHECK_ARG(kb >= 1 && (int64_t)kb * b->page_size <= 1 << 20, "kb must be >= 1 with kb * page_size <= 2^20");
+  CHECK_ARG(blk_idx && idx, "blk_idx and idx are required");
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return expand_blocks_launch(blk_idx, kb, b, idx, (cudaStream_t)stream);
 }
 
 dsa_status_t dsa_cp_candidates(const float *scores, int64_t ld_scores, const int32_t *idx, int32_t T, int32_t k,

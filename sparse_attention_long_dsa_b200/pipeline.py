@@ -100,11 +100,43 @@ class DeviceBatch:
         B.dsa_topk(self.scores if scores is None else scores, self.ld, self.batch, self.wl.topk, self.idx, self.ws,
                    self.ws_bytes, stream)
 
-    def attention(self, stream=None, idx=None):
+    def attention(self, stream=None, idx=None, k=None):
         wl = self.wl
         fn = B.dsa_sparse_attn_decode if self.decode else B.dsa_sparse_attn_prefill
         fn(self.q, self.dt, self.kv_pool, self.v_pool, wl.H, wl.Dqk, wl.Dv, wl.softmax_scale,
-           self.idx if idx is None else idx, wl.topk, self.batch, self.out, self.lse, self.ws, self.ws_bytes, stream)
+           self.idx if idx is None else idx, wl.topk if k is None else k, self.batch, self.out, self.lse, self.ws,
+           self.ws_bytes, stream)
+
+    def block_select(self, kb, stream=None):
+        """Block-granular selection from the current scores: page scores, the kb best pages per row (the
+        usual top-k on a batch of the rows' page lists) and their token positions.  Returns the index
+        array [total_q, kb * page_size] for attention(idx=..., k=kb * page_size); the page scores, page
+        counts and kept pages stay in blk_scores, blk_lens and blk_idx."""
+        wl, dv, T, P = self.wl, self.device, self.wl.total_q, self.wl.page_size
+        max_pages = (wl.max_seq_len + P - 1) // P
+        if getattr(self, "_blk_kb", None) != kb:
+            self.ld_blk = (max_pages + 3) // 4 * 4
+            self.blk_scores = torch.empty((T, self.ld_blk), dtype=torch.float32, device=dv)
+            self.blk_lens = torch.empty((T,), dtype=torch.int32, device=dv)
+            self._blk_bt = torch.zeros((T, (max_pages + P - 1) // P), dtype=torch.int32, device=dv)
+            self._blk_cu = torch.arange(T + 1, dtype=torch.int32, device=dv)
+            self.blk_batch = B.make_batch(self._blk_bt, self.blk_lens, self._blk_cu, num_blocks=1, page_size=P,
+                                          total_q=T, max_q_per_seq=1 if T else 0, max_seq_len=max(max_pages, 1))
+            self._blk_ws_bytes = B.dsa_workspace_size(B.DSA_OP_TOPK, self.blk_batch, kb)
+            self._blk_ws = torch.zeros(self._blk_ws_bytes, dtype=torch.uint8, device=dv)
+            self.blk_idx = torch.empty((T, kb), dtype=torch.int32, device=dv)
+            self.idx_blk = torch.empty((T, kb * P), dtype=torch.int32, device=dv)
+            op_attn = B.DSA_OP_ATTN_DECODE if self.decode else B.DSA_OP_ATTN_PREFILL
+            need = B.dsa_workspace_size(op_attn, self.batch, kb * P, wl.H, wl.Dv)
+            if need > self.ws_bytes:
+                self.ws_bytes = need
+                self.ws = torch.zeros(need, dtype=torch.uint8, device=dv)
+            self._blk_kb = kb
+        B.dsa_block_scores(self.scores, self.ld, self.batch, self.blk_scores, self.ld_blk, self.blk_lens, stream)
+        B.dsa_topk(self.blk_scores, self.ld_blk, self.blk_batch, kb, self.blk_idx, self._blk_ws, self._blk_ws_bytes,
+                   stream)
+        B.dsa_expand_blocks(self.blk_idx, kb, self.batch, self.idx_blk, stream)
+        return self.idx_blk
 
     def run(self, stream=None):
         self.indexer(stream)

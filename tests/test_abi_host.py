@@ -186,3 +186,23 @@ def test_context_parallel_entries_validate_before_launch():
         with pytest.raises(B.DSAError) as e:
             call()
         assert e.value.status == status
+
+
+def test_block_selection_entries_validate_before_launch():
+    b = _batch()                                       # max_seq_len 100 -> 2 pages
+    P = 1 << 24
+    B.dsa_block_scores(None, 128, _batch(total_q=0, max_q_per_seq=0), None, 4, None, 0)      # empty: no-op
+    B.dsa_expand_blocks(None, 2, _batch(total_q=0, max_q_per_seq=0), None, 0)
+    bad = [
+        (lambda: B.dsa_block_scores(P, 64, b, P, 4, P, 0), B.DSA_ERR_INVALID_ARG),          # ld_scores < 100
+        (lambda: B.dsa_block_scores(P, 128, b, P, 1, P, 0), B.DSA_ERR_INVALID_ARG),         # ld_blk < 2 pages
+        (lambda: B.dsa_block_scores(P, 128, b, P, 6, P, 0), B.DSA_ERR_INVALID_ARG),         # ld_blk % 4
+        (lambda: B.dsa_block_scores(P, 128, b, P + 4, 4, P, 0), B.DSA_ERR_INVALID_ARG),     # alignment
+        (lambda: B.dsa_block_scores(P, 128, b, P, 4, None, 0), B.DSA_ERR_INVALID_ARG),      # NULL blk_lens
+        (lambda: B.dsa_expand_blocks(P, 0, b, P, 0), B.DSA_ERR_INVALID_ARG),                # kb = 0
+        (lambda: B.dsa_expand_blocks(None, 2, b, P, 0), B.DSA_ERR_INVALID_ARG),
+    ]
+    for call, status in bad:
+        with pytest.raises(B.DSAError) as e:
+            call()
+        assert e.value.status == status

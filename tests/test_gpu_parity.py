@@ -407,3 +407,40 @@ def test_context_parallel_decode_1m_planted():
     sel, out, lse = _cp_run(wl, 4)
     assert np.array_equal(sel[0], np.sort(wl.planted))
     _cp_check(wl, [0], sel, out, lse)
+
+
+# --------------------------------------------------------------------------------------- block-granular selection
+def _block_case(kind, grid):
+    if kind == "prefill":
+        return W.make_workload("blocks", kind="mla", seed=115, seq_lens=[70, 300, 2100, 2600], q_lens=[70, 37, 300, 5],
+                               topk=2048, grid=grid)
+    return W.make_workload("blocks_decode", kind="mla", seed=116, seq_lens=[1, 64, 65, 2049, 9000, 15000],
+                           q_lens=[1] * 6, topk=2048, grid=grid)
+
+
+@pytest.mark.parametrize("kind,grid,kb", [("prefill", True, 8), ("prefill", False, 8), ("decode", True, 32),
+                                          ("decode", False, 5)])
+def test_block_selection_matches_oracle(kind, grid, kb):
+    """Page scores bit-exact (a max of the same fp32 scores), kept pages and their positions exact (the
+    oracle decides on the GPU's fp32 scores), attention over that set within the MLA tolerances."""
+    wl = _block_case(kind, grid)
+    db = DeviceBatch(wl)
+    db.indexer()
+    idx = db.block_select(kb)
+    db.attention(idx=idx, k=kb * 64)
+    torch.cuda.synchronize()
+    db.check_status()
+    sc = db.scores.cpu().numpy()
+    blk = db.blk_scores.cpu().numpy()
+    lens = db.blk_lens.cpu().numpy()
+    got = idx.cpu().numpy()
+    out, lse = db.out.float().cpu().numpy(), db.lse.cpu().numpy()
+    for r in range(wl.total_q):
+        _, pos = oracle.row_location(wl.seq_lens, wl.cu_q, r)
+        s = sc[r, : pos + 1].astype(np.float64)
+        bs = oracle.block_scores_row(s, 64)
+        assert lens[r] == bs.size and np.array_equal(blk[r, : bs.size].astype(np.float64), bs), f"row {r}: page scores"
+        exp = oracle.block_topk_row(s, kb, 64)
+        assert np.array_equal(got[r], exp), f"row {r}: block selection differs"
+        ref_o, ref_l = oracle.sparse_attention_row(wl, r, exp)
+        check_attention(wl, r, out[r], lse[r], ref_o, ref_l)

@@ -1,6 +1,6 @@
 """Context-parallel decode on the CPU: the range split, the local batches and the exchange schedule of
 `context_parallel`, with every local step done by the oracle (test-only rank objects), against the
-single-GPU oracle.  The CUDA kernels of the same steps are checked in tests/test_gpu_parity.py."""
+single-GPU oracle.  The CUDA kernels of the same steps are checked in tests/test_zz_widened_paths_gpu.py."""
 import datetime
 import os
 import sys

@@ -43,6 +43,13 @@ What each step follows (page titles and sections of the source pages):
   the best kb pages are kept with ties to the lower page, and attention runs
   over all their causal tokens.  An approximation of the token-granular
   path, with this oracle of its own.
+* Decode index reuse -- "Day-0 Adaptation: Running Trillion-Parameter Models
+  on Domestic AI Accelerators", 3.3 (the decode path keeps its indices
+  incrementally and reuses the previous step's result): the candidates of a
+  step are an earlier selection plus every token added since, scored by the
+  same indexer at those positions only, and the k best are kept (ties to the
+  lower position).  An approximation of a full selection, exact on its own
+  definition.
 * Cache append -- "Engineering Practices ...", Four Key Layers 3 (the decode
   step writes the new token into the KV cache, merged with its attention
   launch) and 2 (the block table places a token in its block); the indexer
@@ -255,6 +262,30 @@ def block_topk_row(scores: np.ndarray, kb: int, page_size: int) -> np.ndarray:
         pos = p * page_size + np.arange(page_size)
         out[i * page_size: (i + 1) * page_size] = np.where(pos < n, pos, -1)
     return out
+
+
+def reuse_candidates(prev_idx: np.ndarray, prev_len: int, pos: int) -> np.ndarray:
+    """Candidates of a decode step that reuses an earlier selection: that selection's positions (made when
+    the sequence held prev_len tokens) followed by every position added since, prev_len .. pos.  -1 entries
+    of the earlier selection stay as -1 slots."""
+    prev_idx = np.asarray(prev_idx, dtype=np.int64)
+    return np.concatenate([prev_idx, np.arange(prev_len, pos + 1, dtype=np.int64)])
+
+
+def candidate_scores_row(case, row: int, cands: np.ndarray) -> np.ndarray:
+    """Indexer scores of one query row at the given candidate positions (-1 gives -inf), from the full
+    scorer: the same definition, evaluated only where asked."""
+    cands = np.asarray(cands, dtype=np.int64)
+    full = indexer_scores_row(case, row)
+    return np.where(cands >= 0, full[np.maximum(cands, 0)], -np.inf)
+
+
+def candidate_topk(cand_scores: np.ndarray, cands: np.ndarray, k: int) -> np.ndarray:
+    """The k best candidates by score (ties to the earlier candidate slot, which is the lower position when
+    the candidates are in ascending position order), returned as positions in slot order, -1 padded."""
+    slots = topk_row(cand_scores, k)
+    cands = np.asarray(cands, dtype=np.int64)
+    return np.where(slots >= 0, cands[np.maximum(slots, 0)], -1).astype(np.int32)
 
 
 # ----------------------------------------------------------------------------

@@ -452,3 +452,44 @@ def test_block_topk_reduces_to_token_topk():
         assert np.array_equal(oracle.block_topk_row(sc, kb, 1), oracle.topk_row(sc, kb))
         nb = (n + 63) // 64
         assert np.array_equal(oracle.block_topk_row(sc, nb, 64), oracle.topk_row(sc, nb * 64))
+
+
+# ----------------------------------------------------------------------------- decode index reuse
+
+def test_reuse_candidates_and_selection_by_hand():
+    # an earlier selection {2, 5, 9} (one -1 slot) made at 12 tokens; the query now sits at position 14
+    cands = oracle.reuse_candidates(np.array([2, 5, 9, -1]), 12, 14)
+    assert cands.tolist() == [2, 5, 9, -1, 12, 13, 14]
+    sc = np.array([0.5, 3.0, 3.0, -np.inf, 1.0, 3.0, -2.0])
+    # k = 3: the three 3.0's (slots 1, 2, 5 -> positions 5, 9, 13)
+    assert oracle.candidate_topk(sc, cands, 3).tolist() == [5, 9, 13]
+    # k = 2: the tie at 3.0 goes to the earlier slots (positions 5 and 9)
+    assert oracle.candidate_topk(sc, cands, 2).tolist() == [5, 9]
+    # k = 8 >= 7 candidates: every slot in slot order (the empty slot stays -1), then -1 padding
+    assert oracle.candidate_topk(sc, cands, 8).tolist() == [2, 5, 9, -1, 12, 13, 14, -1]
+
+
+def test_reuse_with_every_position_is_the_full_selection():
+    """When the earlier selection held every earlier position, reuse selects exactly what a full top-k
+    selects (the candidates are then all positions, in order)."""
+    wl = _tiny_case(topk=20)
+    for row in (30, 70, 95):
+        _, pos = oracle.row_location(wl.seq_lens, wl.cu_q, row)
+        prev = np.arange(0, pos - 3)
+        cands = oracle.reuse_candidates(prev, pos - 3, pos)
+        sc = oracle.candidate_scores_row(wl, row, cands)
+        full = oracle.indexer_scores_row(wl, row)
+        assert np.array_equal(sc, full)
+        assert np.array_equal(oracle.candidate_topk(sc, cands, 20), oracle.topk_row(full, 20))
+
+
+def test_reuse_of_the_same_step_is_idempotent():
+    """Reusing a selection made at the same position with no new tokens returns that selection."""
+    wl = _tiny_case(topk=16)
+    for row in (10, 40, 95):
+        full = oracle.indexer_scores_row(wl, row)
+        sel = oracle.topk_row(full, 16)
+        _, pos = oracle.row_location(wl.seq_lens, wl.cu_q, row)
+        cands = oracle.reuse_candidates(sel, pos + 1, pos)
+        got = oracle.candidate_topk(oracle.candidate_scores_row(wl, row, cands), cands, 16)
+        assert np.array_equal(np.sort(got[got >= 0]), sel[sel >= 0])

@@ -228,6 +228,27 @@ DSA_API dsa_status_t dsa_block_scores(const float *scores, int64_t ld_scores, co
 DSA_API dsa_status_t dsa_expand_blocks(const int32_t *blk_idx, int32_t kb, const dsa_batch_t *b, int32_t *idx,
                                        void *stream);
 
+/* Decode index reuse ("Day-0 Adaptation: Running Trillion-Parameter Models on Domestic AI Accelerators",
+ * 3.3: the decode path maintains its indices incrementally and reuses the previous step's result).  A
+ * variant of the full selection, approximate by design, for decode batches (one row per sequence):
+ * dsa_reuse_candidates: cand[row, j] = prev_idx[row, j] for j < k (entries >= prev_lens[row] become -1),
+ *   then prev_lens[row] + (j - k) for the positions added since, -1 past the row's position.  cand
+ *   [T, k + max_new]; a row with more than max_new new positions is reported by dsa_read_device_status
+ *   as DSA_ERR_DEVICE_CHECK (its extra positions are not candidates).
+ * dsa_indexer_scores_at: cand_scores[row, j] = the indexer score I(row, cand[row, j]) (same definition
+ *   as dsa_indexer_scores), -inf for -1 or positions past the row.  e4m3 indexer, Hi = 64, Di = 128.
+ * dsa_topk over cand_scores (a batch of T sequences of m candidates, one query row each; m a multiple of
+ *   4) keeps k slots, ties to the earlier slot (the lower position).
+ * dsa_gather_positions: idx[row, j] = cand[row, sel[row, j]] (-1 for -1), for either attention call. */
+DSA_API dsa_status_t dsa_reuse_candidates(const int32_t *prev_idx, int32_t k, const int32_t *prev_lens, int32_t max_new,
+                                          const dsa_batch_t *b, int32_t *cand, void *ws, size_t ws_bytes, void *stream);
+DSA_API dsa_status_t dsa_indexer_scores_at(const void *q_idx, dsa_dtype_t q_dt, const float *w, const void *k_idx_pool,
+                                           dsa_dtype_t k_dt, const float *k_scale_pool, int32_t Hi, int32_t Di,
+                                           const dsa_batch_t *b, const int32_t *cand, int32_t m, float *cand_scores,
+                                           void *ws, size_t ws_bytes, void *stream);
+DSA_API dsa_status_t dsa_gather_positions(const int32_t *sel, int32_t k, const int32_t *cand, int32_t m, int32_t T,
+                                          int32_t *idx, void *stream);
+
 /* Context-parallel decode ("Engineering Practices ...", Four Key Layers 3: partial attention over
  * disjoint key sets merged by a log-sum-exp reduction, here across GPUs).  Every sequence of a decode
  * batch (one query row per sequence, T rows) is spread over G ranks, rank r holding the contiguous token

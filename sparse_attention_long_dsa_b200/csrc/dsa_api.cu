@@ -30,6 +30,13 @@ size_t attn_workspace_bytes(int T, int k, bool decode);
 dsa_status_t cache_append_launch(const void *kv_new, const void *k_new, bool k_bf16, const dsa_batch_t *b,
                                  void *kv_pool, void *kI_pool, float *kS_pool, void *ws, cudaStream_t stream);
 dsa_status_t selftest_wait_launch(long long budget, void *ws, cudaStream_t stream);
+dsa_status_t reuse_candidates_launch(const int32_t *prev_idx, int k, const int32_t *prev_lens, int max_new,
+                                     const dsa_batch_t *b, int32_t *cand, void *ws, cudaStream_t stream);
+dsa_status_t indexer_at_launch(const uint8_t *qI, const float *w, const uint8_t *kpool, const float *kscale,
+                               const dsa_batch_t *b, const int32_t *cand, int m, float *out, void *ws,
+                               cudaStream_t stream);
+dsa_status_t gather_positions_launch(const int32_t *sel, int k, const int32_t *cand, int m, int T, int32_t *idx,
+                                     cudaStream_t stream);
 dsa_status_t block_scores_launch(const float *scores, int64_t ld, const dsa_batch_t *b, float *blk, int64_t ld_blk,
                                  int32_t *blk_lens, cudaStream_t stream);
 dsa_status_t expand_blocks_launch(const int32_t *blk_idx, int kb, const dsa_batch_t *b, int32_t *idx,
@@ -322,6 +329,50 @@ dsa_status_t dsa_selftest_wait_timeout(uint64_t budget_cycles, void *ws, size_t 
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
   return selftest_wait_launch((long long)budget_cycles, ws, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_reuse_candidates(const int32_t *prev_idx, int32_t k, const int32_t *prev_lens, int32_t max_new,
+                                  const dsa_batch_t *b, int32_t *cand, void *ws, size_t ws_bytes, void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
+  CHECK_ARG(b->total_q == b->num_seqs && b->max_q_per_seq == 1, "index reuse takes decode batches (one row per sequence)");
+  CHECK_ARG(k >= 1 && max_new >= 0 && (int64_t)k + max_new <= 1 << 24, "k >= 1, max_new >= 0, k + max_new <= 2^24");
+  CHECK_ARG(prev_idx && prev_lens && cand, "prev_idx, prev_lens and cand are required");
+  if ((st = check_ws(ws, ws_bytes, kWsHeader)) != DSA_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return reuse_candidates_launch(prev_idx, k, prev_lens, max_new, b, cand, ws, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_indexer_scores_at(const void *q_idx, dsa_dtype_t q_dt, const float *w, const void *k_idx_pool,
+                                   dsa_dtype_t k_dt, const float *k_scale_pool, int32_t Hi, int32_t Di,
+                                   const dsa_batch_t *b, const int32_t *cand, int32_t m, float *cand_scores, void *ws,
+                                   size_t ws_bytes, void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
+  CHECK_SUP(q_dt == DSA_FP8_E4M3 && k_dt == DSA_FP8_E4M3 && Hi == 64 && Di == 128,
+            "scores at positions support the e4m3 indexer with Hi = 64, Di = 128");
+  CHECK_ARG(m >= 1, "m must be >= 1");
+  CHECK_ARG(q_idx && w && k_idx_pool && k_scale_pool && cand && cand_scores, "every pointer is required");
+  CHECK_ARG(((uintptr_t)k_idx_pool & 15) == 0, "k_idx_pool must be 16-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, kWsHeader)) != DSA_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return indexer_at_launch((const uint8_t *)q_idx, w, (const uint8_t *)k_idx_pool, k_scale_pool, b, cand, m, cand_scores,
+                           ws, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_gather_positions(const int32_t *sel, int32_t k, const int32_t *cand, int32_t m, int32_t T,
+                                  int32_t *idx, void *stream) {
+  CHECK_ARG(T >= 0 && k >= 1 && m >= 1, "T >= 0, k and m >= 1");
+  if (T == 0) return DSA_OK;
+  CHECK_ARG(sel && cand && idx, "sel, cand and idx are required");
+  DeviceInfo dev;
+  dsa_status_t st;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  return gather_positions_launch(sel, k, cand, m, T, idx, (cudaStream_t)stream);
 }
 
 dsa_status_t dsa_block_scores(const float *scores, int64_t ld_scores, const dsa_batch_t *b, float *blk_scores,

@@ -107,6 +107,33 @@ class DeviceBatch:
            self.idx if idx is None else idx, wl.topk if k is None else k, self.batch, self.out, self.lse, self.ws,
            self.ws_bytes, stream)
 
+    def reuse_select(self, prev_idx, prev_lens, max_new, stream=None):
+        """Decode index reuse: candidates = an earlier selection prev_idx [T, k] (made at prev_lens [T]
+        tokens) plus the positions added since (at most max_new per row), scored at those positions only,
+        the k best kept.  Returns the index array [T, k] for attention(); the candidate list and scores stay
+        in cand and cand_scores."""
+        wl, dv, T, k = self.wl, self.device, self.wl.total_q, self.wl.topk
+        m = (k + max_new + 3) // 4 * 4                      # slots past k + max_new stay -1
+        if getattr(self, "_reuse_m", None) != m:
+            self.cand = torch.empty((T, m), dtype=torch.int32, device=dv)
+            self.cand_scores = torch.empty((T, m), dtype=torch.float32, device=dv)
+            self._cand_bt = torch.zeros((T, (m + 63) // 64), dtype=torch.int32, device=dv)
+            self._cand_len = torch.full((T,), m, dtype=torch.int32, device=dv)
+            self._cand_cu = torch.arange(T + 1, dtype=torch.int32, device=dv)
+            self.cand_batch = B.make_batch(self._cand_bt, self._cand_len, self._cand_cu, num_blocks=1,
+                                           page_size=wl.page_size, total_q=T, max_q_per_seq=1, max_seq_len=m)
+            self._cand_ws_bytes = B.dsa_workspace_size(B.DSA_OP_TOPK, self.cand_batch, k)
+            self._cand_ws = torch.zeros(self._cand_ws_bytes, dtype=torch.uint8, device=dv)
+            self._cand_sel = torch.empty((T, k), dtype=torch.int32, device=dv)
+            self.idx_reuse = torch.empty((T, k), dtype=torch.int32, device=dv)
+            self._reuse_m = m
+        B.dsa_reuse_candidates(prev_idx, k, prev_lens, m - k, self.batch, self.cand, self.ws, self.ws_bytes, stream)
+        B.dsa_indexer_scores_at(self.qI, self.idx_dt, self.w, self.kI_pool, self.idx_dt, self.kS_pool, wl.Hi, wl.Di,
+                                self.batch, self.cand, m, self.cand_scores, self.ws, self.ws_bytes, stream)
+        B.dsa_topk(self.cand_scores, m, self.cand_batch, k, self._cand_sel, self._cand_ws, self._cand_ws_bytes, stream)
+        B.dsa_gather_positions(self._cand_sel, k, self.cand, m, T, self.idx_reuse, stream)
+        return self.idx_reuse
+
     def block_select(self, kb, stream=None):
         """Block-granular selection from the current scores: page scores, the kb best pages per row (the
         usual top-k on a batch of the rows' page lists) and their token positions.  Returns the index

@@ -206,3 +206,27 @@ def test_block_selection_entries_validate_before_launch():
         with pytest.raises(B.DSAError) as e:
             call()
         assert e.value.status == status
+
+
+def test_reuse_entries_validate_before_launch():
+    b = _batch(total_q=2, max_q_per_seq=1)
+    P = 1 << 24
+    empty = _batch(total_q=0, max_q_per_seq=0)
+    B.dsa_reuse_candidates(None, 16, None, 4, empty, None, None, 0, 0)
+    B.dsa_indexer_scores_at(None, B.DSA_FP8_E4M3, None, None, B.DSA_FP8_E4M3, None, 64, 128, empty, None, 20, None,
+                            None, 0, 0)
+    B.dsa_gather_positions(None, 16, None, 20, 0, None, 0)
+    bad = [
+        (lambda: B.dsa_reuse_candidates(P, 16, P, 4, _batch(), P, P, 256, 0), B.DSA_ERR_INVALID_ARG),   # 2 rows/seq
+        (lambda: B.dsa_reuse_candidates(P, 0, P, 4, b, P, P, 256, 0), B.DSA_ERR_INVALID_ARG),           # k = 0
+        (lambda: B.dsa_reuse_candidates(P, 16, P, 4, b, P, P, 128, 0), B.DSA_ERR_WORKSPACE),
+        (lambda: B.dsa_indexer_scores_at(P, B.DSA_F32, P, P, B.DSA_F32, None, 2, 32, b, P, 20, P, P, 256, 0),
+         B.DSA_ERR_UNSUPPORTED),
+        (lambda: B.dsa_indexer_scores_at(P, B.DSA_FP8_E4M3, P, P + 4, B.DSA_FP8_E4M3, P, 64, 128, b, P, 20, P, P, 256, 0),
+         B.DSA_ERR_INVALID_ARG),
+        (lambda: B.dsa_gather_positions(P, 16, None, 20, 2, P, 0), B.DSA_ERR_INVALID_ARG),
+    ]
+    for call, status in bad:
+        with pytest.raises(B.DSAError) as e:
+            call()
+        assert e.value.status == status

@@ -232,3 +232,47 @@ def test_block_selection_matches_oracle(kind, grid, kb):
         assert np.array_equal(got[r], exp), f"row {r}: block selection differs"
         ref_o, ref_l = oracle.sparse_attention_row(wl, r, exp)
         check_attention(wl, r, out[r], lse[r], ref_o, ref_l)
+
+
+# --------------------------------------------------------------------------------------- decode index reuse
+@pytest.mark.parametrize("grid", [True, False])
+def test_decode_index_reuse_matches_oracle(grid):
+    """An earlier selection (this step's own, cut to the positions before prev_len) plus the positions
+    added since: the candidate list exact, the scores at the candidates within the indexer tolerance
+    (bit-exact on the integer grid), the kept positions exact (the oracle decides on the GPU's fp32
+    candidate scores), attention over them within the MLA tolerances."""
+    from parity import SCORE_REL, abs_case
+    seq_lens = np.array([300, 2100, 5000, 9000])
+    delta = np.array([1, 7, 64, 300])                                # tokens added since the earlier selection
+    wl = W.make_workload("reuse", kind="mla", seed=117, seq_lens=seq_lens, q_lens=[1] * 4, topk=2048, grid=grid)
+    db = _run(wl)
+    prev_lens = seq_lens - delta
+    prev = db.idx.clone()
+    prev_lens_d = torch.from_numpy(prev_lens.astype(np.int32)).cuda()
+    prev[prev >= prev_lens_d[:, None]] = -1
+    idx = db.reuse_select(prev, prev_lens_d, int(delta.max()))
+    db.attention(idx=idx)
+    torch.cuda.synchronize()
+    db.check_status()
+    cand, cs, got = db.cand.cpu().numpy(), db.cand_scores.cpu().numpy(), idx.cpu().numpy()
+    out, lse = db.out.float().cpu().numpy(), db.lse.cpu().numpy()
+    prev_h = prev.cpu().numpy()
+    acase = abs_case(wl)
+    m = cand.shape[1]
+    for r in range(wl.total_q):
+        _, pos = oracle.row_location(wl.seq_lens, wl.cu_q, r)
+        exp_c = oracle.reuse_candidates(prev_h[r], int(prev_lens[r]), pos)
+        exp_c = np.concatenate([exp_c, np.full(m - exp_c.size, -1)])
+        assert np.array_equal(cand[r], exp_c), f"row {r}: candidate list differs"
+        osc = oracle.candidate_scores_row(wl, r, exp_c)
+        fin = np.isfinite(osc)
+        assert np.array_equal(np.isfinite(cs[r]), fin), f"row {r}: empty candidate slots differ"
+        if grid:
+            assert np.array_equal(cs[r][fin].astype(np.float64), osc[fin]), f"row {r}: grid scores inexact"
+        else:
+            A = oracle.candidate_scores_row(acase, r, exp_c)
+            assert np.all(np.abs(cs[r][fin] - osc[fin]) <= SCORE_REL["mla"] * A[fin] + 1e-30), f"row {r}: scores"
+        exp = oracle.candidate_topk(cs[r].astype(np.float64), exp_c, wl.topk)
+        assert np.array_equal(got[r], exp), f"row {r}: kept positions differ"
+        ref_o, ref_l = oracle.sparse_attention_row(wl, r, exp)
+        check_attention(wl, r, out[r], lse[r], ref_o, ref_l)

@@ -228,6 +228,18 @@ DSA_API dsa_status_t dsa_block_scores(const float *scores, int64_t ld_scores, co
 DSA_API dsa_status_t dsa_expand_blocks(const int32_t *blk_idx, int32_t kb, const dsa_batch_t *b, int32_t *idx,
                                        void *stream);
 
+/* Cache append fused with the indexer ("Engineering Practices ...", Four Key Layers 3: the decode step
+ * merges the KV cache update into its sparse-attention launches): dsa_cache_append's writes (new tokens'
+ * latent rows and quantised indexer keys, same arguments and layouts) and then dsa_indexer_scores over
+ * the updated pools, in one call.  For batches of up to 256 query rows the append runs inside the
+ * indexer's first kernel; larger batches get a separate append launch ahead of it.  The workspace is the
+ * indexer's (dsa_workspace_size(DSA_OP_INDEXER)); its status word also reports the append's bad block ids. */
+DSA_API dsa_status_t dsa_indexer_scores_append(const void *kv_new, dsa_dtype_t kv_dt, const void *k_new,
+                                               dsa_dtype_t k_new_dt, void *kv_pool, const void *q_idx, dsa_dtype_t q_dt,
+                                               const float *w, void *k_idx_pool, dsa_dtype_t k_dt, float *k_scale_pool,
+                                               int32_t Hi, int32_t Di, const dsa_batch_t *b, float *scores,
+                                               int64_t ld_scores, void *ws, size_t ws_bytes, void *stream);
+
 /* Decode index reuse ("Day-0 Adaptation: Running Trillion-Parameter Models on Domestic AI Accelerators",
  * 3.3: the decode path maintains its indices incrementally and reuses the previous step's result).  A
  * variant of the full selection, approximate by design, for decode batches (one row per sequence):

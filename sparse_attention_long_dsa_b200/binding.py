@@ -23,7 +23,8 @@ EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_a
            "dsa_sparse_attn_decode", "dsa_read_device_status", "dsa_status_string", "dsa_last_error",
            "dsa_version", "dsa_launch_count", "dsa_topk_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout",
            "dsa_cp_candidates", "dsa_cp_rows", "dsa_cp_select_local", "dsa_cp_merge", "dsa_block_scores",
-           "dsa_expand_blocks", "dsa_reuse_candidates", "dsa_indexer_scores_at", "dsa_gather_positions")
+           "dsa_expand_blocks", "dsa_reuse_candidates", "dsa_indexer_scores_at", "dsa_gather_positions",
+           "dsa_indexer_scores_append")
 
 
 class dsa_batch_t(ctypes.Structure):
@@ -72,6 +73,7 @@ def load(path: str = LIB_PATH):
         "dsa_selftest_wait_timeout": [ctypes.c_uint64, P, SZ, P],
         "dsa_block_scores": [P, I64, B, P, I64, P, P],
         "dsa_reuse_candidates": [P, I32, P, I32, B, P, P, SZ, P],
+        "dsa_indexer_scores_append": [P, I32, P, I32, P, P, I32, P, P, I32, P, I32, I32, B, P, I64, P, SZ, P],
         "dsa_indexer_scores_at": [P, I32, P, P, I32, P, I32, I32, B, P, I32, P, P, SZ, P],
         "dsa_gather_positions": [P, I32, P, I32, I32, P, P],
         "dsa_expand_blocks": [P, I32, B, P, P],
@@ -177,6 +179,15 @@ def dsa_cache_append(kv_new, kv_dt: int, k_new, k_dt: int, Dqk: int, Di: int, ba
 def dsa_selftest_wait_timeout(budget_cycles: int, ws, ws_bytes: int, stream=None):
     _check(load().dsa_selftest_wait_timeout(budget_cycles, _ptr(ws), ws_bytes, _stream(stream)),
            "dsa_selftest_wait_timeout")
+
+
+def dsa_indexer_scores_append(kv_new, kv_dt: int, k_new, k_new_dt: int, kv_pool, q_idx, q_dt: int, w, k_idx_pool,
+                              k_dt: int, k_scale_pool, Hi: int, Di: int, batch: dsa_batch_t, scores, ld_scores: int,
+                              ws, ws_bytes: int, stream=None):
+    _check(load().dsa_indexer_scores_append(_ptr(kv_new), kv_dt, _ptr(k_new), k_new_dt, _ptr(kv_pool), _ptr(q_idx),
+                                            q_dt, _ptr(w), _ptr(k_idx_pool), k_dt, _ptr(k_scale_pool), Hi, Di,
+                                            ctypes.byref(batch), _ptr(scores), ld_scores, _ptr(ws), ws_bytes,
+                                            _stream(stream)), "dsa_indexer_scores_append")
 
 
 def dsa_reuse_candidates(prev_idx, k: int, prev_lens, max_new: int, batch: dsa_batch_t, cand, ws, ws_bytes: int,

@@ -6,6 +6,7 @@
 #include <atomic>
 #include <mutex>
 
+#include "append.cuh"
 #include "common.cuh"
 
 namespace dsa {
@@ -21,7 +22,7 @@ dsa_status_t indexer_simt_launch(const void *qI, dsa_dtype_t dt, const float *w,
                                  int64_t ld, cudaStream_t stream);
 dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t *kpool, const float *kscale,
                                const dsa_batch_t *b, float *scores, int64_t ld, void *ws, cudaStream_t stream,
-                               int num_sms);
+                               int num_sms, const AppendArgs *app);
 size_t indexer_workspace_bytes(int num_seqs, int total_q);
 dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, int k, float softmax_scale,
                              const dsa_batch_t *b, void *out, float *lse, void *ws, bool decode, cudaStream_t stream,
@@ -219,7 +220,7 @@ dsa_status_t dsa_indexer_scores(const void *q_idx, dsa_dtype_t q_dt, const float
   if ((st = current_device(&dev)) != DSA_OK) return st;
   if (mla)
     return indexer_tc_launch((const uint8_t *)q_idx, w, (const uint8_t *)k_idx_pool, k_scale_pool, b, scores,
-                             ld_scores, ws, (cudaStream_t)stream, dev.num_sms);
+                             ld_scores, ws, (cudaStream_t)stream, dev.num_sms, nullptr);
   return indexer_simt_launch(q_idx, q_dt, w, k_idx_pool, k_scale_pool, Hi, Di, b, scores, ld_scores,
                              (cudaStream_t)stream);
 }
@@ -329,6 +330,33 @@ dsa_status_t dsa_selftest_wait_timeout(uint64_t budget_cycles, void *ws, size_t 
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
   return selftest_wait_launch((long long)budget_cycles, ws, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_indexer_scores_append(const void *kv_new, dsa_dtype_t kv_dt, const void *k_new, dsa_dtype_t k_new_dt,
+                                       void *kv_pool, const void *q_idx, dsa_dtype_t q_dt, const float *w,
+                                       void *k_idx_pool, dsa_dtype_t k_dt, float *k_scale_pool, int32_t Hi, int32_t Di,
+                                       const dsa_batch_t *b, float *scores, int64_t ld_scores, void *ws,
+                                       size_t ws_bytes, void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
+  CHECK_ARG(kv_new && k_new && kv_pool && q_idx && w && k_idx_pool && k_scale_pool && scores,
+            "kv_new, k_new, kv_pool, q_idx, w, k_idx_pool, k_scale_pool and scores are required");
+  CHECK_SUP(kv_dt == DSA_BF16 && (k_new_dt == DSA_F32 || k_new_dt == DSA_BF16) && q_dt == DSA_FP8_E4M3 &&
+                k_dt == DSA_FP8_E4M3 && Hi == 64 && Di == 128,
+            "the fused append supports the MLA path: bf16 latent rows, f32 or bf16 new keys, e4m3 indexer 64 x 128");
+  CHECK_ARG(ld_scores >= b->max_seq_len && ld_scores % 4 == 0,
+            "ld_scores (%lld) must be >= max_seq_len and a multiple of 4", (long long)ld_scores);
+  CHECK_ARG((((uintptr_t)kv_new | (uintptr_t)k_new | (uintptr_t)kv_pool | (uintptr_t)q_idx | (uintptr_t)w |
+              (uintptr_t)k_idx_pool | (uintptr_t)k_scale_pool | (uintptr_t)scores) & 15) == 0,
+            "every buffer must be 16-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, indexer_workspace_bytes(b->num_seqs, b->total_q))) != DSA_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  const AppendArgs app{(const uint4 *)kv_new, k_new, k_new_dt == DSA_BF16 ? 1 : 0, (uint4 *)kv_pool,
+                       (uint32_t *)k_idx_pool, k_scale_pool};
+  return indexer_tc_launch((const uint8_t *)q_idx, w, (const uint8_t *)k_idx_pool, k_scale_pool, b, scores, ld_scores,
+                           ws, (cudaStream_t)stream, dev.num_sms, &app);
 }
 
 dsa_status_t dsa_reuse_candidates(const int32_t *prev_idx, int32_t k, const int32_t *prev_lens, int32_t max_new,

@@ -22,6 +22,7 @@
 //   warps 2..5   epilogue: tcgen05.ld 64 heads per row, ReLU, weight, sum, key scale, causal store
 // Work units are (row group, key tile) pairs in group order, split evenly over the CTAs; a one-CTA
 // plan kernel enumerates the groups and their tile counts in the workspace first.
+#include "append.cuh"
 #include "tc.cuh"
 
 namespace dsa {
@@ -71,12 +72,10 @@ static IdxPlanView plan_view(void *ws, int num_seqs, int total_q) {
   return v;
 }
 
-__global__ void __launch_bounds__(1024) indexer_plan_kernel(BatchView bv, IdxPlanView pv) {
-  __shared__ uint32_t tmp[64];
-  __shared__ uint32_t s_carry;
+// the plan, by one CTA of 1024 threads (tmp: 64 words of scan scratch, s_carry: one shared word)
+__device__ __forceinline__ void indexer_plan_body(const BatchView &bv, const IdxPlanView &pv, uint32_t *tmp,
+                                                  uint32_t &s_carry) {
   const int tid = threadIdx.x;
-  pdl_wait();
-  pdl_trigger();
   if (tid == 0) s_carry = 0;
   __syncthreads();
   // groups per sequence -> seq_goff (exclusive prefix)
@@ -131,6 +130,30 @@ __global__ void __launch_bounds__(1024) indexer_plan_kernel(BatchView bv, IdxPla
     pv.hdr[0] = G;
     pv.hdr[1] = (int)s_carry;
   }
+}
+
+__global__ void __launch_bounds__(1024) indexer_plan_kernel(BatchView bv, IdxPlanView pv) {
+  __shared__ uint32_t tmp[64];
+  __shared__ uint32_t s_carry;
+  pdl_wait();
+  pdl_trigger();
+  indexer_plan_body(bv, pv, tmp, s_carry);
+}
+
+// The decode step's cache update fused into its first kernel: the 32 warps append the batch's new tokens
+// (one warp per token, append.cuh), then the CTA builds the plan.  The indexer's main kernel, which reads
+// the new keys, starts its work only once this kernel has completed.
+constexpr int kIdxFusedAppendMaxRows = 256;
+
+__global__ void __launch_bounds__(1024) indexer_plan_append_kernel(BatchView bv, IdxPlanView pv, AppendArgs app, int T,
+                                                                   uint32_t *status) {
+  __shared__ uint32_t tmp[64];
+  __shared__ uint32_t s_carry;
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int row = warp; row < T; row += 32) append_token_warp(app, bv, row, lane, status);
+  indexer_plan_body(bv, pv, tmp, s_carry);
 }
 
 // ------------------------------------------------------------------------------------------------ main
@@ -463,9 +486,12 @@ static size_t indexer_tc_smem() {
          sizeof(IdxSmem);
 }
 
+dsa_status_t cache_append_launch(const void *kv_new, const void *k_new, bool k_bf16, const dsa_batch_t *b,
+                                 void *kv_pool, void *kI_pool, float *kS_pool, void *ws, cudaStream_t stream);
+
 dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t *kpool, const float *kscale,
                                const dsa_batch_t *b, float *scores, int64_t ld, void *ws, cudaStream_t stream,
-                               int num_sms) {
+                               int num_sms, const AppendArgs *app) {
   BatchView bv = view_of(b);
   IdxPlanView pv = plan_view(ws, b->num_seqs, b->total_q);
   CUtensorMap tm_k, tm_q;
@@ -474,7 +500,17 @@ dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t 
     set_error("indexer: cuTensorMapEncodeTiled failed");
     return DSA_ERR_CUDA;
   }
-  DSA_LAUNCH_PDL("indexer_plan_kernel", indexer_plan_kernel, dim3(1), dim3(1024), 0, stream, bv, pv);
+  if (app != nullptr && b->total_q <= kIdxFusedAppendMaxRows) {
+    DSA_LAUNCH_PDL("indexer_plan_append_kernel", indexer_plan_append_kernel, dim3(1), dim3(1024), 0, stream, bv, pv,
+                   *app, b->total_q, (uint32_t *)ws);
+  } else {
+    if (app != nullptr) {
+      const dsa_status_t st = cache_append_launch(app->kv_new, app->k_new, app->k_bf16 != 0, b, app->kv_pool,
+                                                  app->kI_pool, app->kS_pool, ws, stream);
+      if (st != DSA_OK) return st;
+    }
+    DSA_LAUNCH_PDL("indexer_plan_kernel", indexer_plan_kernel, dim3(1), dim3(1024), 0, stream, bv, pv);
+  }
   const size_t smem = indexer_tc_smem();
   cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   DSA_LAUNCH_PDL("indexer_tc_kernel", indexer_tc_kernel, dim3(num_sms), dim3(kIdxThreads), smem, stream, tm_k, tm_q,

@@ -96,6 +96,14 @@ class DeviceBatch:
         B.dsa_indexer_scores(self.qI, self.idx_dt, self.w, self.kI_pool, self.idx_dt, self.kS_pool, wl.Hi, wl.Di,
                              self.batch, self.scores, self.ld, self.ws, self.ws_bytes, stream)
 
+    def append_and_indexer(self, kv_new, k_new, k_dt, stream=None):
+        """The decode step's cache update fused with the indexer: writes the batch's new tokens (kv_new
+        [T, 576] bf16 bits, k_new [T, 128] of k_dt) into this batch's pools, then scores."""
+        wl = self.wl
+        B.dsa_indexer_scores_append(kv_new, self.dt, k_new, k_dt, self.kv_pool, self.qI, self.idx_dt, self.w,
+                                    self.kI_pool, self.idx_dt, self.kS_pool, wl.Hi, wl.Di, self.batch, self.scores,
+                                    self.ld, self.ws, self.ws_bytes, stream)
+
     def topk(self, stream=None, scores=None):
         B.dsa_topk(self.scores if scores is None else scores, self.ld, self.batch, self.wl.topk, self.idx, self.ws,
                    self.ws_bytes, stream)

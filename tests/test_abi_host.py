@@ -230,3 +230,26 @@ def test_reuse_entries_validate_before_launch():
         with pytest.raises(B.DSAError) as e:
             call()
         assert e.value.status == status
+
+
+def test_fused_append_validates_before_launch():
+    b = _batch(total_q=2, max_q_per_seq=1)
+    P = 1 << 24
+    F8, BF, F32 = B.DSA_FP8_E4M3, B.DSA_BF16, B.DSA_F32
+    B.dsa_indexer_scores_append(None, BF, None, F32, None, None, F8, None, None, F8, None, 64, 128,
+                                _batch(total_q=0, max_q_per_seq=0), None, 128, None, 0, 0)          # empty: no-op
+    bad = [
+        (dict(k_new_dt=F8), B.DSA_ERR_UNSUPPORTED),
+        (dict(Hi=32), B.DSA_ERR_UNSUPPORTED),
+        (dict(kv_pool=None), B.DSA_ERR_INVALID_ARG),
+        (dict(ld=64), B.DSA_ERR_INVALID_ARG),                # < max_seq_len 100
+        (dict(k_new=P + 8), B.DSA_ERR_INVALID_ARG),          # alignment
+        (dict(ws_bytes=16), B.DSA_ERR_WORKSPACE),
+    ]
+    for over, status in bad:
+        a = dict(kv_new=P, k_new=P, k_new_dt=F32, kv_pool=P, Hi=64, ld=128, ws_bytes=1 << 20)
+        a.update(over)
+        with pytest.raises(B.DSAError) as e:
+            B.dsa_indexer_scores_append(a["kv_new"], BF, a["k_new"], a["k_new_dt"], a["kv_pool"], P, F8, P, P, F8, P,
+                                        a["Hi"], 128, b, P, a["ld"], P, a["ws_bytes"], 0)
+        assert e.value.status == status, over

@@ -276,3 +276,44 @@ def test_decode_index_reuse_matches_oracle(grid):
         assert np.array_equal(got[r], exp), f"row {r}: kept positions differ"
         ref_o, ref_l = oracle.sparse_attention_row(wl, r, exp)
         check_attention(wl, r, out[r], lse[r], ref_o, ref_l)
+
+
+# --------------------------------------------------------------------------------------- append fused with the indexer
+def _own_pools(wl, dev):
+    inputs = DeviceBatch.upload_inputs(wl, dev)
+    inputs["kv_pool"] = torch.from_numpy(np.ascontiguousarray(wl.kv_pool).view(np.int16)).to(dev)
+    return inputs
+
+
+@pytest.mark.parametrize("shape", ["decode", "chunk"])
+def test_append_fused_with_indexer_matches_separate_calls(shape):
+    """The fused call (inside the indexer's first kernel for <= 256 rows; a separate launch for the 305-row
+    chunk) leaves the same pools and scores, bit for bit, as dsa_cache_append followed by dsa_indexer_scores,
+    and the pools equal the oracle's append."""
+    if shape == "decode":
+        seq_lens, q_lens = [300, 2100, 5000, 65], [1, 1, 1, 1]
+    else:
+        seq_lens, q_lens = [2100, 700], [300, 5]
+    wl = W.make_workload("fused_append", kind="mla", seed=118, seq_lens=seq_lens, q_lens=q_lens, topk=2048)
+    dev = torch.device("cuda")
+    kv_new, k_in, fmt = _append_inputs(wl.total_q, np.random.default_rng(119), False)
+    kv_d, k_d = _dev_copy(kv_new, dev), _dev_copy(k_in, dev)
+    a = DeviceBatch(wl, inputs=_own_pools(wl, dev))
+    b = DeviceBatch(wl, inputs=_own_pools(wl, dev))
+    a.append_and_indexer(kv_d, k_d, B.DSA_F32)
+    B.dsa_cache_append(kv_d, B.DSA_BF16, k_d, B.DSA_F32, 576, 128, b.batch, b.kv_pool, b.kI_pool, b.kS_pool, b.ws,
+                       b.ws_bytes)
+    b.indexer()
+    torch.cuda.synchronize()
+    a.check_status()
+    b.check_status()
+    for name in ("kv_pool", "kI_pool", "kS_pool"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), f"{name} differs between fused and separate calls"
+    for r in range(wl.total_q):
+        _, pos = oracle.row_location(wl.seq_lens, wl.cu_q, r)
+        assert torch.equal(a.scores[r, : pos + 1], b.scores[r, : pos + 1]), f"row {r}: scores differ"
+    ekv, ekI, ekS = oracle.cache_append(wl, kv_new.view(np.uint16), k_in, fmt)
+    assert np.array_equal(a.kv_pool.cpu().numpy().view(np.uint16), ekv)
+    assert np.array_equal(a.kS_pool.cpu().numpy().view(np.uint32), ekS.view(np.uint32))
+    zero = lambda c: np.where((c & 0x7F) == 0, 0, c)
+    assert np.array_equal(zero(a.kI_pool.cpu().numpy()), zero(ekI))

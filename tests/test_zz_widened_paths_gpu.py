@@ -317,3 +317,22 @@ def test_append_fused_with_indexer_matches_separate_calls(shape):
     assert np.array_equal(a.kS_pool.cpu().numpy().view(np.uint32), ekS.view(np.uint32))
     zero = lambda c: np.where((c & 0x7F) == 0, 0, c)
     assert np.array_equal(zero(a.kI_pool.cpu().numpy()), zero(ekI))
+
+
+# --------------------------------------------------------------------------------------- zig-zag prefill
+@pytest.mark.parametrize("world", [2, 3])
+def test_zigzag_prefill_ranks_match_one_batch(world):
+    """Each rank's zig-zag share of a prompt, run as its own batch, gives its rows exactly the scores, picks,
+    outputs and lse that the whole prompt run as one batch gives them (every step is per row)."""
+    from sparse_attention_long_dsa_b200 import prefill_parallel as PP
+    wl = W.make_workload("zz_gpu", kind="mla", seed=120, seq_lens=[3000], q_lens=[2600], topk=2048, grid=True)
+    whole = _run(wl)
+    for rank in range(world):
+        loc, rows = PP.local_prefill_workload(wl, rank, world)
+        db = _run(loc)
+        rt = torch.from_numpy(rows).cuda()
+        assert torch.equal(db.idx, whole.idx[rt]), f"rank {rank}: picks differ"
+        assert torch.equal(db.out, whole.out[rt]) and torch.equal(db.lse, whole.lse[rt]), f"rank {rank}: attention"
+        for i in range(0, loc.total_q, 97):
+            _, pos = oracle.row_location(loc.seq_lens, loc.cu_q, i)
+            assert torch.equal(db.scores[i, : pos + 1], whole.scores[int(rows[i]), : pos + 1]), f"rank {rank} row {i}"

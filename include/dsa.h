@@ -20,6 +20,12 @@
  * Million-Token Context Models on Domestic AI Chips", Four Key Layers 3:
  * separate prefill and decode paths.)
  *
+ * Around them: dsa_indexer_scores_append (the cache append fused into the indexer's first kernel); two
+ * approximate selection variants, block-granular (dsa_block_scores, dsa_expand_blocks) and decode index
+ * reuse (dsa_reuse_candidates, dsa_indexer_scores_at, dsa_gather_positions), both ending in dsa_topk;
+ * the steps of context-parallel decode across GPUs (dsa_cp_*); and a self-test of the bounded device
+ * waits (dsa_selftest_wait_timeout).
+ *
  * Conventions shared by every call
  * --------------------------------
  * Ownership: the caller owns every buffer.  Pointers inside dsa_batch_t and all

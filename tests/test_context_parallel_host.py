@@ -142,9 +142,9 @@ def _gloo_rank(rank, world, port, results):
 def test_two_gloo_ranks_match_single_gpu_oracle():
     world = 2
     port = 33500 + (os.getpid() % 2000)
-    with mp.Manager() as mgr:
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
         results = mgr.dict()
-        ctx = mp.get_context("spawn")
         procs = [ctx.Process(target=_gloo_rank, args=(r, world, port, results)) for r in range(world)]
         for p in procs:
             p.start()

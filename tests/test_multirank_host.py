@@ -44,9 +44,9 @@ def _rank_main(rank, world, port, results):
 def test_two_gloo_ranks_slowest_rank_time_and_weak_scaling_value():
     world = 2
     port = 29500 + (os.getpid() % 2000)
-    with mp.Manager() as mgr:
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
         results = mgr.dict()
-        ctx = mp.get_context("spawn")
         procs = [ctx.Process(target=_rank_main, args=(r, world, port, results)) for r in range(world)]
         for p in procs:
             p.start()
@@ -134,9 +134,9 @@ def test_overlapped_e2e_ranks_agree(sets_per_rank):
     run it (so that neither waits in a collective the other never enters)."""
     world = 2
     port = 31500 + (os.getpid() % 2000) + 7 * sets_per_rank[1]
-    with mp.Manager() as mgr:
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
         results = mgr.dict()
-        ctx = mp.get_context("spawn")
         procs = [ctx.Process(target=_e2e_rank_main, args=(r, world, port, results, sets_per_rank))
                  for r in range(world)]
         for p in procs:

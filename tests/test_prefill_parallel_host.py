@@ -75,9 +75,9 @@ def _gloo_pages(rank, world, port, results):
 def test_two_gloo_ranks_fill_the_pool():
     world = 2
     port = 35500 + (os.getpid() % 2000)
-    with mp.Manager() as mgr:
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
         results = mgr.dict()
-        ctx = mp.get_context("spawn")
         procs = [ctx.Process(target=_gloo_pages, args=(r, world, port, results)) for r in range(world)]
         for p in procs:
             p.start()

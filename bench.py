@@ -280,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
 
 def _seed(args, rank):
     base = {"decode_batch": 20260002, "prefill_16k": 20260003, "decode_1m_planted": 20260004,
-            "mixed_batch": 20260005}[args.workload]
+            "mixed_batch": 20260005, "prefill_4k": 20260003}[args.workload]
     return base + 1000 * rank
 
 
@@ -525,7 +525,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="decode_batch",
-                    choices=["decode_batch", "prefill_16k", "decode_1m_planted", "mixed_batch", "tiny_f32"])
+                    choices=["decode_batch", "prefill_16k", "prefill_4k", "decode_1m_planted", "mixed_batch", "tiny_f32"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--replicas", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")

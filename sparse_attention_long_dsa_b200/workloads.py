@@ -33,7 +33,7 @@ import numpy as np
 
 __all__ = [
     "Workload", "make_workload", "bf16_encode", "e4m3_encode",
-    "tiny_f32", "decode_batch", "prefill_16k", "decode_1m_planted", "mixed_batch",
+    "tiny_f32", "decode_batch", "prefill_16k", "prefill_4k", "decode_1m_planted", "mixed_batch",
     "BENCH_WORKLOADS",
 ]
 
@@ -356,6 +356,12 @@ def prefill_16k(seed: int = 20260003, grid: bool = False) -> Workload:
                          topk=2048, grid=grid)
 
 
+def prefill_4k(seed: int = 20260003, grid: bool = False) -> Workload:
+    """The prefill workload at a quarter of the length (4096-token causal prompt): small enough for a
+    full profiler capture, the same shapes otherwise."""
+    return make_workload("prefill_4k", kind="mla", seed=seed, seq_lens=[4096], q_lens=[4096], topk=2048, grid=grid)
+
+
 def decode_1m_planted(seed: int = 20260004, attention: bool = True) -> Workload:
     """Long-context decode: one query over a 1,048,576-token paged cache, with 2048
     planted positions whose indexer keys align with the query."""
@@ -378,6 +384,7 @@ BENCH_WORKLOADS = {
     "tiny_f32": tiny_f32,
     "decode_batch": decode_batch,
     "prefill_16k": prefill_16k,
+    "prefill_4k": prefill_4k,
     "decode_1m_planted": decode_1m_planted,
     "mixed_batch": mixed_batch,
 }

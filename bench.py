@@ -401,19 +401,46 @@ def run_e2e_overlapped(args, wl, sets, dev, world):
     ms = slowest_rank_ms(res["ms"], world, dev)
     return {"value": job_tokens_per_s(wl.total_q, world, ms / args.steps), "unit": "tokens/s",
             "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"], "ms_per_step": ms / args.steps,
-            "pipeline": "copy-in, compute and copy-out of neighbouring steps overlapped on three streams, "
-                        "two device input/output sets"}
+            "pipeline": "copy-in (one packed copy), compute and copy-out of neighbouring steps overlapped on three "
+                        "streams, two device input/output sets"}
 
 
-def _e2e_overlapped_local(args, wl, sets, dev):
+def _packed_step_inputs(wl, replicas, dev):
+    """A step's inputs (q, qI, w and the batch descriptor's arrays) packed into one pinned host buffer, and for
+    each replica a batch whose per-step inputs are views into one device buffer of the same layout (its pools
+    stay the replica's), so that a step's copy-in is a single copy."""
     import torch
-    names = ("q", "qI", "w", "block_table", "seq_lens", "cu_q")
-    host_in = {n: torch.empty(sets[0].inputs[n].shape, dtype=sets[0].inputs[n].dtype, pin_memory=True) for n in names}
-    for n in names:
-        host_in[n].copy_(sets[0].inputs[n].cpu())
+    from sparse_attention_long_dsa_b200.pipeline import DeviceBatch
+    arrays = {"q": wl.q, "qI": wl.qI, "w": wl.w, "block_table": wl.block_table.astype(np.int32),
+              "seq_lens": wl.seq_lens.astype(np.int32), "cu_q": wl.cu_q.astype(np.int32)}
+    tdt = {np.dtype(np.uint16): torch.int16, np.dtype(np.uint8): torch.uint8, np.dtype(np.float32): torch.float32,
+           np.dtype(np.int32): torch.int32}
+    layout, total = {}, 0
+    for n, a in arrays.items():
+        a = np.ascontiguousarray(a)
+        layout[n] = (total, a)
+        total += (a.nbytes + 255) // 256 * 256
+    host = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    hn = host.numpy()
+    for n, (o, a) in layout.items():
+        hn[o: o + a.nbytes] = a.reshape(-1).view(np.uint8)
+    batches, bufs = [], []
+    for db in replicas:
+        dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
+        inputs = dict(db.inputs)
+        for n, (o, a) in layout.items():
+            inputs[n] = dbuf[o: o + a.nbytes].view(tdt[a.dtype]).view(a.shape)
+        batches.append(DeviceBatch(wl, device=dev, decode=db.decode, inputs=inputs))
+        bufs.append(dbuf)
+    return host, bufs, batches
+
+
+def _e2e_overlapped_local(args, wl, replicas, dev):
+    import torch
+    host_in, dev_in, sets = _packed_step_inputs(wl, replicas[:2], dev)
     host_out = [(torch.empty(db.out.shape, dtype=db.out.dtype, pin_memory=True),
-                 torch.empty(db.lse.shape, dtype=db.lse.dtype, pin_memory=True)) for db in sets[:2]]
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+                 torch.empty(db.lse.shape, dtype=db.lse.dtype, pin_memory=True)) for db in sets]
+    h2d = host_in.numel()
     d2h = sum(t.numel() * t.element_size() for t in host_out[0])
     s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
     in_done = [torch.cuda.Event() for _ in range(2)]       # set j's inputs are on the device
@@ -427,8 +454,7 @@ def _e2e_overlapped_local(args, wl, sets, dev):
             if i >= 2:
                 s_in.wait_event(cmp_done[j])
             with torch.cuda.stream(s_in):
-                for name in names:
-                    db.inputs[name].copy_(host_in[name], non_blocking=True)
+                dev_in[j].copy_(host_in, non_blocking=True)
             in_done[j].record(s_in)
             s_cmp.wait_event(in_done[j])
             if i >= 2:

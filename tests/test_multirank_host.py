@@ -119,6 +119,10 @@ def _e2e_rank_main(rank, world, port, results, sets_per_rank):
         import types
         import bench
         _fake_cuda(step_ms=1.0 + rank)                         # rank 1 is the slower one
+        # the packed copy-in buffers and their batches: plain CPU buffers around the fake batches
+        bench._packed_step_inputs = lambda wl, reps, dev: (torch.zeros(512, dtype=torch.uint8),
+                                                             [torch.zeros(512, dtype=torch.uint8) for _ in reps],
+                                                             list(reps))
         args = types.SimpleNamespace(steps=6, warmup=3)
         wl = types.SimpleNamespace(total_q=32)
         sets = [_FakeBatch() for _ in range(sets_per_rank[rank])]

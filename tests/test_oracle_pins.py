@@ -307,6 +307,56 @@ def test_block_table_permutation_invariance():
             assert np.array_equal(ref[row][key], got[row][key])
 
 
+def _bf16_bits_by_torch(x):
+    """bf16 bit patterns of x through torch's own fp32 -> bf16 cast (the values used here are exact)."""
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_mla_value_slice_hand():
+    """MLA layout: keys are the whole latent row, values its leading Dv entries.  The rope dims carry values
+    that a trailing slice, the whole row, or a dropped rope term in the keys would turn into other outputs."""
+    g = _golden("mla_attention_hand.json")
+    P, Dqk = g["page_size"], g["Dqk"]
+    kv = np.zeros((1, P, Dqk), np.float32)
+    kv[0, : len(g["kv"])] = g["kv"]
+    case = SimpleNamespace(kind="mla", page_size=P, seq_lens=np.array([len(g["kv"])], np.int32),
+                           cu_q=np.array([0, 1], np.int32), block_table=np.zeros((1, 1), np.int32),
+                           q=_bf16_bits_by_torch(np.array(g["q"], np.float32)[None]), kv_pool=_bf16_bits_by_torch(kv),
+                           v_pool=None, Dqk=Dqk, Dv=g["Dv"], softmax_scale=math.log(3.0))
+    for c in g["cases"]:
+        o, lse = oracle.sparse_attention_row(case, 0, np.array(c["idx"]))
+        assert o.shape == (2, g["Dv"])
+        assert np.allclose(o, c["out"], rtol=0, atol=1e-14)
+        assert np.allclose(lse, c["lse"], rtol=0, atol=1e-14)
+
+
+def test_mla_attention_matches_torch_sdpa_on_bf16_rows():
+    """The oracle's MLA attention (its own bf16 decoder, paged lookup and value slice) against torch's fp64
+    SDPA over the same rows decoded by torch's bf16 view: K = the whole latent row, V = its first Dv
+    entries, a boolean mask for the selected set."""
+    wl = _small_mla(grid=False)
+    assert wl.Dqk > wl.Dv and wl.v_pool is None
+    for row in range(wl.total_q):
+        b, pos = oracle.row_location(wl.seq_lens, wl.cu_q, row)
+        r = oracle.run_rows(wl, [row])[row]
+        idx = r["idx"][r["idx"] >= 0]
+        allpos = np.arange(int(wl.seq_lens[b]))
+        blk, slot = wl.block_table[b, allpos // wl.page_size], allpos % wl.page_size
+        lat = torch.from_numpy(np.ascontiguousarray(wl.kv_pool[blk, slot]).view(np.int16)).view(torch.bfloat16)
+        lat = lat.to(torch.float64)
+        q = torch.from_numpy(np.ascontiguousarray(wl.q[row]).view(np.int16)).view(torch.bfloat16).to(torch.float64)
+        K, V = lat, lat[:, : wl.Dv]
+        H = q.shape[0]
+        mask = torch.zeros(allpos.size, dtype=torch.bool)
+        mask[torch.from_numpy(idx)] = True
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[:, None, :], K.expand(H, -1, -1), V.expand(H, -1, -1),
+            attn_mask=mask[None, None, :].expand(H, 1, -1), scale=wl.softmax_scale)[:, 0, :]
+        assert np.allclose(r["out"], ref.numpy(), rtol=0, atol=1e-12)
+        lse_ref = torch.logsumexp(wl.softmax_scale * (q @ K.T)[:, torch.from_numpy(idx)], dim=1)
+        assert np.allclose(r["lse"], lse_ref.numpy(), rtol=0, atol=1e-12)
+
+
 def test_lse_is_log_normaliser():
     wl = _tiny_case(topk=20)
     r = oracle.run_rows(wl, [70])[70]

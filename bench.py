@@ -176,21 +176,12 @@ def job_tokens_per_s(tokens_per_rank_step, world, ms_per_step):
     return world * tokens_per_rank_step / (ms_per_step / 1e3)
 
 
-def run_ours(args, rank, world, local_rank):
+def _time_steps(replicas, stream, steps, warmup, world, dev, sampler=None):
+    """W untimed warm-up steps, then K steps bracketed by a barrier and a device synchronise, timed with
+    CUDA events on the launching stream (per-stage events inside the timed region).  Returns the slowest
+    rank's total milliseconds, the per-stage averages, the library launches and the clock summary."""
     import torch
     from sparse_attention_long_dsa_b200 import binding as B
-    from sparse_attention_long_dsa_b200 import workloads as W
-    from sparse_attention_long_dsa_b200.pipeline import DeviceBatch
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    B.load()
-    wl = W.BENCH_WORKLOADS[args.workload](**({} if args.workload == "tiny_f32" else {"seed": _seed(args, rank)}))
-    work = work_of(wl)
-    replicas = []
-    for r in range(args.replicas):
-        replicas.append(DeviceBatch(wl, device=dev))
-    stream = torch.cuda.Stream(device=dev)
     stages = ("indexer", "topk", "attention")
 
     def step(db, ev=None):
@@ -206,16 +197,13 @@ def run_ours(args, rank, world, local_rank):
         if ev is not None:
             ev[3].record(stream)
 
-    sampler = ClockSampler(local_rank)
-    sampler.start()
     with torch.cuda.stream(stream):
-        for i in range(args.warmup):
+        for i in range(warmup):
             step(replicas[i % len(replicas)])
     torch.cuda.synchronize(dev)
     for db in replicas:
         db.check_status(stream)
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -224,7 +212,7 @@ def run_ours(args, rank, world, local_rank):
     launches0 = B.dsa_launch_count()
     w0 = time.perf_counter()
     t_start.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(replicas[i % len(replicas)], evs[i])
     t_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -232,10 +220,8 @@ def run_ours(args, rank, world, local_rank):
     launches = B.dsa_launch_count() - launches0
     if world > 1:
         torch.distributed.barrier()
-    sampler.stop()
     for db in replicas:
         db.check_status(stream)
-
     total_ms = t_start.elapsed_time(t_end)
     stage_ms = {s: [] for s in stages}
     for e in evs:
@@ -243,6 +229,66 @@ def run_ours(args, rank, world, local_rank):
             stage_ms[s].append(e[j].elapsed_time(e[j + 1]))
     stage_avg = {s: float(np.mean(v)) for s, v in stage_ms.items()}
     total_ms = slowest_rank_ms(total_ms, world, dev)
+    clocks = sampler.summary(w0, w1) if sampler is not None else None
+    return total_ms, stage_avg, int(launches), clocks
+
+
+# the other MLA workloads timed by the default run, each a 1-GPU figure of its own
+EXTRA_WORKLOADS = ("prefill_16k", "decode_1m_planted", "mixed_batch")
+
+
+def run_extra_workload(name, args, dev, stream, sampler):
+    """One more workload of the same path, timed like the headline (inputs larger than L2, one device
+    replica), reported with its own stage times, the roofline of its dominant stage against the burst peaks
+    and the whole step's roofline."""
+    import torch
+    from sparse_attention_long_dsa_b200 import workloads as W
+    from sparse_attention_long_dsa_b200.pipeline import DeviceBatch
+
+    wl = W.BENCH_WORKLOADS[name](seed=_seed_of(name, 0))
+    work = work_of(wl)
+    db = DeviceBatch(wl, device=dev)
+    # enough steps for a timed region of about 0.2 s (clock samples under load), at least --extra-steps
+    probe_ms, _, _, _ = _time_steps([db], stream, 1, args.warmup, 1, dev, None)
+    steps = int(min(2000, max(args.extra_steps, math.ceil(200.0 / max(probe_ms, 1e-3)))))
+    total_ms, stage_avg, launches, clocks = _time_steps([db], stream, steps, 1, 1, dev, sampler)
+    ms_per_step = total_ms / steps
+    peaks, peak_src = load_peaks()
+    decode = bool(np.all(wl.q_lens == 1))
+    dom = max(stage_avg, key=stage_avg.get)
+    res = {"metric": "sparse-attn decode tokens/s" if decode else "sparse-attn prefill tokens/s",
+           "value": job_tokens_per_s(work["tokens"], 1, ms_per_step), "unit": "tokens/s", "steps": steps,
+           "warmup": args.warmup, "ms_per_step": ms_per_step, "stages_ms": stage_avg,
+           "roofline": roofline_entry(dom, stage_avg[dom], work, peaks, peak_src, name, decode),
+           "stage_rooflines": {s: roofline_entry(s, stage_avg[s], work, peaks, peak_src, name, decode)
+                               for s in ("indexer", "attention")},
+           "step_roofline": step_roofline(work, peaks, ms_per_step), "gpu_launches": launches, "clocks": clocks,
+           "config": workload_config(wl, replicas=1, l2="inputs larger than L2 (one device replica)")}
+    del db
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from sparse_attention_long_dsa_b200 import binding as B
+    from sparse_attention_long_dsa_b200 import workloads as W
+    from sparse_attention_long_dsa_b200.pipeline import DeviceBatch
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    B.load()
+    wl = W.BENCH_WORKLOADS[args.workload](**({} if args.workload == "tiny_f32" else {"seed": _seed(args, rank)}))
+    work = work_of(wl)
+    replicas = []
+    for r in range(args.replicas):
+        replicas.append(DeviceBatch(wl, device=dev))
+    stream = torch.cuda.Stream(device=dev)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    total_ms, stage_avg, launches, clocks = _time_steps(replicas, stream, args.steps, args.warmup, world, dev, sampler)
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(work["tokens"], world, ms_per_step)
 
@@ -259,37 +305,51 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     dom = max(stage_avg, key=stage_avg.get)
     decode = bool(np.all(wl.q_lens == 1))
-    roof = roofline_entry(dom, stage_avg[dom], work, peaks, peak_src, args, decode)
-    clocks = sampler.summary(w0, w1)
+    roof = roofline_entry(dom, stage_avg[dom], work, peaks, peak_src, args.workload, decode)
     res = {
         "metric": "sparse-attn decode tokens/s" if wl.kind == "mla" and np.all(wl.q_lens == 1)
         else "sparse-attn prefill tokens/s",
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16+e4m3" if wl.kind == "mla" else "f32", "data": "synthetic",
-        "config": workload_config(wl, args),
+        "config": workload_config(wl, replicas=args.replicas),
         "stages_ms": stage_avg, "roofline": roof, "e2e": e2e, "gpu_launches": int(launches),
         "clocks": clocks, "impl": "ours",
     }
     if wl.kind == "mla":
         res["step_roofline"] = step_roofline(work, peaks, ms_per_step)
+    del replicas
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    # the other MLA workloads (1 GPU only: under torchrun the ranks would each repeat them)
+    extras = [] if (world > 1 or args.workload != "decode_batch") else \
+        [w for w in (args.extra_workloads.split(",") if args.extra_workloads else []) if w]
+    if extras:
+        res["workloads"] = {}
+        for name in extras:
+            res["workloads"][name] = run_extra_workload(name, args, dev, stream, sampler)
+    sampler.stop()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     return res
 
 
-def _seed(args, rank):
+def _seed_of(workload, rank):
     base = {"decode_batch": 20260002, "prefill_16k": 20260003, "decode_1m_planted": 20260004,
-            "mixed_batch": 20260005, "prefill_4k": 20260003}[args.workload]
+            "mixed_batch": 20260005, "prefill_4k": 20260003}[workload]
     return base + 1000 * rank
 
 
-def workload_config(wl, args):
+def _seed(args, rank):
+    return _seed_of(args.workload, rank)
+
+
+def workload_config(wl, replicas=1, l2=None):
     d = {"workload": wl.name, "batch_seqs": wl.num_seqs, "query_rows": wl.total_q,
          "context": f"{int(wl.seq_lens.min())}..{int(wl.seq_lens.max())}", "topk": wl.topk, "heads": wl.H,
          "d_qk": wl.Dqk, "d_v": wl.Dv, "indexer": f"{wl.Hi}x{wl.Di} {'e4m3' if wl.kind == 'mla' else 'f32'}",
-         "page": wl.page_size, "l2": f"{args.replicas} rotating device replicas of all inputs (> L2 touched "
-                                     f"between reuses)"}
+         "page": wl.page_size,
+         "l2": l2 or f"{replicas} rotating device replicas of all inputs (> L2 touched between reuses)"}
     return d
 
 
@@ -313,9 +373,10 @@ def measured_traffic(stage, workload):
     return rec["bytes"] if m.hexdigest()[:16] == rec["sha256_16"] else None
 
 
-def roofline_entry(stage, ms, work, peaks, src, args, decode):
+def roofline_entry(stage, ms, work, peaks, src, workload, decode):
     """Decode stages are HBM-bound (bytes / HBM copy bandwidth); prefill attention and indexer are
-    tensor-bound (flops / dense peak: bf16 for attention, 2x bf16 for the FP8 indexer)."""
+    tensor-bound (flops / the burst dense peak: bf16 for attention, 2x bf16 for the FP8 indexer; each stage
+    is timed as one call of milliseconds, not as a seconds-long loop)."""
     w = work[stage]
     secs = ms / 1e3
     tag = f"{src} (MEASURED_PEAKS.json)" if src == "measured" else "fallback"
@@ -324,15 +385,15 @@ def roofline_entry(stage, ms, work, peaks, src, args, decode):
         peak = peaks["hbm_gbs"]
         return {"kernel": stage, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "peak_source": f"{tag} hbm_gbs", "algorithmic_bytes_per_launch": w["bytes"],
-                "avg_launch_ms": ms, "traffic": measured_traffic(stage, args.workload),
+                "avg_launch_ms": ms, "traffic": measured_traffic(stage, workload),
                 "tflops": w["flops"] / secs / 1e12}
     ach = w["flops"] / secs / 1e12
     fp8 = stage == "indexer"
-    peak = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
+    peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
     return {"kernel": stage, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-            "peak_source": f"{tag} bf16_tflops_sustained" + (" x2 (fp8 = 2x bf16 dense ratio)" if fp8 else ""),
+            "peak_source": f"{tag} bf16_tflops (burst)" + (" x2 (fp8 = 2x bf16 dense ratio)" if fp8 else ""),
             "algorithmic_flops_per_launch": w["flops"], "avg_launch_ms": ms,
-            "traffic": measured_traffic(stage, args.workload),
+            "traffic": measured_traffic(stage, workload),
             "gbs": w["bytes"] / secs / 1e9}
 
 
@@ -508,7 +569,9 @@ def cpu_baseline(wl, budget_s=15.0, rows=None):
                 break
         passes += 1
     dt = time.perf_counter() - t0
-    return {"value": done / dt, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+    return {"value": done / dt, "unit": "tokens/s", "cores": _blas_threads(), "host_cores": os.cpu_count(),
+            "threads": "one Python thread walks the rows; numpy's BLAS calls inside it use up to `cores` threads",
+            "kind": "oracle",
             "sample": f"{done} query-row evaluations over {len(order)} rows of {wl.name} (full path per row: "
                       f"scores, top-k, attention), {dt:.1f} s wall"}
 
@@ -537,8 +600,10 @@ def run_reference(args, rank, world):
     line = {"metric": "sparse-attn decode tokens/s" if np.all(wl.q_lens == 1) else "sparse-attn prefill tokens/s",
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic", "config": workload_config(wl, args), "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "dtype": "f64", "data": "synthetic", "config": workload_config(wl, replicas=args.replicas), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "host_cores": os.cpu_count(),
+                             "threads": "one Python thread walks the rows; numpy's BLAS calls inside it use up to "
+                                        "`cores` threads", "kind": "oracle",
                              "sample": f"{rows_per_step} query rows of {wl.name} per step (bounded sample)"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     return line
@@ -556,6 +621,9 @@ def main():
     ap.add_argument("--replicas", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--extra-workloads", default=",".join(EXTRA_WORKLOADS),
+                    help="comma-separated MLA workloads timed after the decode batch at N=1 ('' for none)")
+    ap.add_argument("--extra-steps", type=int, default=10)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -77,6 +77,22 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
     return code | sign
 
 
+def _e4m3_encode_chunked(x: np.ndarray) -> np.ndarray:
+    """e4m3_encode over a large array, element for element the same codes, computed in pieces of
+    2^20 values on the thread pool (small temporaries, several cores)."""
+    x = np.ascontiguousarray(x)
+    out = np.empty(x.shape, dtype=np.uint8)
+    fx, fo = x.reshape(-1), out.reshape(-1)
+    step = 1 << 20
+
+    def work(lo):
+        fo[lo: lo + step] = e4m3_encode(fx[lo: lo + step])
+
+    with ThreadPoolExecutor(_THREADS) as ex:
+        list(ex.map(work, range(0, fx.size, step)))
+    return out
+
+
 # ----------------------------------------------------------------------------
 # chunked, thread-parallel draws
 # ----------------------------------------------------------------------------
@@ -139,7 +155,7 @@ def _quantise_tokens(k: np.ndarray):
     flat_k = k.reshape(-1, k.shape[-1])
     flat_s = scale.reshape(-1)
     flat_c = codes.reshape(-1, k.shape[-1])
-    step = max(1, _CHUNK // k.shape[-1])
+    step = max(1, (1 << 20) // k.shape[-1])
 
     def work(lo):
         hi = min(lo + step, flat_k.shape[0])
@@ -267,8 +283,8 @@ def make_workload(name: str, *, kind: str, seed: int, seq_lens, q_lens, topk: in
         if kind == "f32":
             qI, kI_pool, kS_pool = qI_real, kI_real, None
         else:
-            qI = e4m3_encode(qI_real)
-            kI_pool = e4m3_encode(kI_real)
+            qI = _e4m3_encode_chunked(qI_real)
+            kI_pool = _e4m3_encode_chunked(kI_real)
             kS_pool = np.exp2(_grid_int(seed, "kS", (NB, P), -2, 2).astype(np.float32)).astype(np.float32)
     else:
         if w_dist == "uniform":
@@ -280,7 +296,7 @@ def make_workload(name: str, *, kind: str, seed: int, seq_lens, q_lens, topk: in
             kI_pool = _normal_f32(seed, "kI", (NB, P, Di))
             kS_pool = None
         else:
-            qI = e4m3_encode(_normal_f32(seed, "qI", (T, Hi, Di)))
+            qI = _e4m3_encode_chunked(_normal_f32(seed, "qI", (T, Hi, Di)))
             k_real = _normal_f32(seed, "kI", (NB, P, Di))
             planted = None
             if planted_k:

@@ -97,7 +97,8 @@ typedef enum {
   DSA_OP_TOPK = 1,
   DSA_OP_ATTN_PREFILL = 2,
   DSA_OP_ATTN_DECODE = 3,
-  DSA_OP_CACHE_APPEND = 4
+  DSA_OP_CACHE_APPEND = 4,
+  DSA_OP_INDEXER_TOPK = 5
 } dsa_op_t;
 
 /* Batch descriptor shared by every call.  The three host integers at the end are
@@ -149,6 +150,24 @@ DSA_API dsa_status_t dsa_indexer_scores(const void *q_idx, dsa_dtype_t q_dt, con
 DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_batch_t *b, int32_t k,
                       int32_t *idx, void *ws, size_t ws_bytes, void *stream);
 
+/* Indexer scores and top-k selection in one call, the selection fused into the scoring ("Day-0 Adaptation:
+ * Running Trillion-Parameter Models on Domestic AI Accelerators", 3.1 Index Selection Operator: scoring,
+ * threshold filtering and index gathering in one operator so that the scores are not walked repeatedly in
+ * global memory; "Engineering Practices ...", Four Key Layers 1).  Same arguments and results as
+ * dsa_indexer_scores followed by dsa_topk: scores[row, s] for s <= pos(row) as dsa_indexer_scores writes
+ * them (kept, so callers may reuse them), and idx [total_q, k] as dsa_topk defines it (bit for bit the same
+ * selection).  For the e4m3 indexer, the scoring kernel also counts the leading 11 bits of every score's
+ * order-preserving key per row (a 2048-bin histogram in the workspace), so the selection starts from the
+ * threshold digit and reads each row's scores once, keeping only the keys at or above it.  The f32 indexer
+ * takes the same selection kernel, which then counts the leading digit itself first.
+ * Workspace: dsa_workspace_size(DSA_OP_INDEXER_TOPK) (the indexer's plus 8 KB per query row); its status
+ * word also reports a selection that ran past its shared-memory capacity (DSA_ERR_DEVICE_CHECK; cannot
+ * happen with a histogram written by this call). */
+DSA_API dsa_status_t dsa_indexer_topk(const void *q_idx, dsa_dtype_t q_dt, const float *w, const void *k_idx_pool,
+                                      dsa_dtype_t k_dt, const float *k_scale_pool, int32_t Hi, int32_t Di,
+                                      const dsa_batch_t *b, int32_t k, float *scores, int64_t ld_scores, int32_t *idx,
+                                      void *ws, size_t ws_bytes, void *stream);
+
 /* Allocation-free top-k.  There is no counterpart in the pages: this entry point exists for callers
  * that cannot allocate device memory for a workspace -- code that runs where cudaMalloc is not allowed
  * or not wanted (a plugin or custom operator handed only a stream, a framework whose memory is owned
@@ -157,9 +176,12 @@ DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_
  * inside the library (about 2.3 MB per device, held until the process exits) instead of a caller
  * workspace.  Limits: total_q <= 256 rows and max_seq_len <= 1,048,576 candidates; larger batches return
  * DSA_ERR_UNSUPPORTED with nothing enqueued.  The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) and caches it; make that first call outside any stream capture.  All
- * calls share the one array, so calls whose GPU work overlaps (different streams, concurrent host
- * threads) race on it; serialise them on one stream.  Allocates nothing: no cudaMalloc/cudaFree. */
+ * address (cudaGetSymbolAddress) and caches it for that device's current context; make that first call
+ * outside any stream capture.  After a device reset (cudaDeviceReset) the next call finds a new context
+ * and looks the address up again, so that call, too, should come before any capture.  All calls share
+ * the one array, so calls whose GPU work overlaps (different streams, concurrent host threads) race on
+ * it; serialise them on one stream.  The selection kernels report no device status, so there is no
+ * status word to read back.  Allocates nothing: no cudaMalloc/cudaFree. */
 DSA_API dsa_status_t dsa_topk_noalloc(const float *scores, int64_t ld_scores, const dsa_batch_t *b, int32_t k,
                                       int32_t *idx, void *stream);
 

@@ -24,6 +24,8 @@
 #include <algorithm>
 #include <mutex>
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace dsa {
@@ -491,7 +493,7 @@ dsa_status_t topk_launch(const float *scores, int64_t ld, const dsa_batch_t *b, 
 // header) is one file-scope device array, sized for at most kNoAllocMaxRows query rows and rows of at
 // most kNoAllocMaxSeqLen candidates.  Every device that loads the library holds it until the process
 // exits.  Host code must not hand the array's host-side name to a kernel: it is only a stand-in there,
-// so the device address is looked up with cudaGetSymbolAddress once per device and cached.
+// so the device address is looked up with cudaGetSymbolAddress once per device (and context) and cached.
 // ------------------------------------------------------------------------------------------------
 constexpr int kNoAllocMaxRows = 256;
 constexpr int kNoAllocMaxSeqLen = 1 << 20;
@@ -503,27 +505,60 @@ constexpr size_t kNoAllocBytes =
 
 static __device__ __align__(256) unsigned char g_topk_scratch[kNoAllocBytes];
 
-static void *g_topk_scratch_addr[kMaxDevices];
+// Device address of the array in the current context.  Looked up once per device and context: a device
+// reset (or any other teardown of the context) unloads the module, and the array's address in the new
+// context may differ, so the cached address is keyed on the context's unique ID as well.
+struct ScratchAddr {
+  unsigned long long ctx_id;
+  void *ptr;
+};
+static ScratchAddr g_topk_scratch_addr[kMaxDevices];
 static std::mutex g_topk_scratch_mu;
 
-// device address of the scratch array on the current device (looked up on first use per device)
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// unique ID of the calling thread's current context (0 if there is none or the driver cannot say)
+static unsigned long long current_ctx_id() {
+  static const CtxGetCurrentFn get_cur = []() -> CtxGetCurrentFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+                   q == cudaDriverEntryPointSuccess ? (CtxGetCurrentFn)p : nullptr;
+  }();
+  static const CtxGetIdFn get_id = []() -> CtxGetIdFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+                   q == cudaDriverEntryPointSuccess ? (CtxGetIdFn)p : nullptr;
+  }();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur && get_id && get_cur(&ctx) == CUDA_SUCCESS && ctx != nullptr && get_id(ctx, &id) == CUDA_SUCCESS) return id;
+  return 0;
+}
+
 static dsa_status_t topk_scratch_address(void **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     set_error("dsa_topk_noalloc: no current CUDA device");
     return DSA_ERR_CUDA;
   }
+  // the runtime makes the device's primary context current on its first call above
+  const unsigned long long ctx = current_ctx_id();
   std::lock_guard<std::mutex> g(g_topk_scratch_mu);
-  if (g_topk_scratch_addr[dev] == nullptr) {
+  ScratchAddr &c = g_topk_scratch_addr[dev];
+  if (c.ptr == nullptr || ctx == 0 || c.ctx_id != ctx) {
     void *p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_topk_scratch);
     if (e != cudaSuccess || p == nullptr) {
       set_error("dsa_topk_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
       return DSA_ERR_CUDA;
     }
-    g_topk_scratch_addr[dev] = p;
+    c.ptr = p;
+    c.ctx_id = ctx;
   }
-  *out = g_topk_scratch_addr[dev];
+  *out = c.ptr;
   return DSA_OK;
 }
 

@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from sparse_attention_long_dsa_b200 import binding as B
 
 pytestmark = pytest.mark.gpu
@@ -57,6 +58,11 @@ def test_noalloc_topk_matches_workspace_topk_on_consecutive_calls(k):
         B.dsa_topk_noalloc(scores, ld, batch, k, got)
         torch.cuda.synchronize()
         assert torch.equal(got, ref), f"call {call}: rows differ {torch.nonzero((got != ref).any(dim=1)).flatten().tolist()}"
+        # and directly against the oracle's selection on the same fp32 scores (exact: same values both sides)
+        sc = scores.cpu().numpy()
+        g = got.cpu().numpy()
+        for i, n in enumerate(lengths):
+            assert np.array_equal(g[i], oracle.topk_row(sc[i, :n].astype(np.float64), k)), f"call {call}, row {i}"
 
 
 def test_noalloc_topk_rejects_oversized_batches():
@@ -68,3 +74,18 @@ def test_noalloc_topk_rejects_oversized_batches():
         B.dsa_topk_noalloc(scores, 100, batch, 8, idx)
     assert e.value.status == B.DSA_ERR_UNSUPPORTED
     assert "256 rows" in B.load().dsa_last_error().decode()
+
+
+def test_noalloc_topk_rejects_rows_past_the_candidate_limit_and_writes_nothing():
+    n = (1 << 20) + 1                                                 # one candidate over the built-in limit
+    batch, keep = _batch([n, 10])
+    ld = (n + 3) // 4 * 4
+    scores = torch.zeros((2, ld), dtype=torch.float32, device="cuda")
+    idx = torch.full((2, 16), -5, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    with pytest.raises(B.DSAError) as e:
+        B.dsa_topk_noalloc(scores, ld, batch, 16, idx)
+    assert e.value.status == B.DSA_ERR_UNSUPPORTED
+    assert "max_seq_len" in B.load().dsa_last_error().decode()
+    torch.cuda.synchronize()
+    assert bool((idx == -5).all()), "a rejected call must enqueue nothing"

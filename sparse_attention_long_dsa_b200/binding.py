@@ -17,14 +17,15 @@ LIB_PATH = os.path.join(PKG, "libdsa.so")
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_DEVICE_CHECK, \
     DSA_ERR_TIMEOUT = range(7)
 DSA_F32, DSA_BF16, DSA_FP8_E4M3 = 0, 1, 2
-DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_ATTN_PREFILL, DSA_OP_ATTN_DECODE, DSA_OP_CACHE_APPEND = 0, 1, 2, 3, 4
+DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_ATTN_PREFILL, DSA_OP_ATTN_DECODE, DSA_OP_CACHE_APPEND, DSA_OP_INDEXER_TOPK = \
+    0, 1, 2, 3, 4, 5
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn_prefill",
            "dsa_sparse_attn_decode", "dsa_read_device_status", "dsa_status_string", "dsa_last_error",
            "dsa_version", "dsa_launch_count", "dsa_topk_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout",
            "dsa_cp_candidates", "dsa_cp_rows", "dsa_cp_select_local", "dsa_cp_merge", "dsa_block_scores",
            "dsa_expand_blocks", "dsa_reuse_candidates", "dsa_indexer_scores_at", "dsa_gather_positions",
-           "dsa_indexer_scores_append")
+           "dsa_indexer_scores_append", "dsa_indexer_topk")
 
 
 class dsa_batch_t(ctypes.Structure):
@@ -66,6 +67,7 @@ def load(path: str = LIB_PATH):
         "dsa_workspace_size": [I32, B, I32, I32, I32, ctypes.POINTER(SZ)],
         "dsa_indexer_scores": [P, I32, P, P, I32, P, I32, I32, B, P, I64, P, SZ, P],
         "dsa_topk": [P, I64, B, I32, P, P, SZ, P],
+        "dsa_indexer_topk": [P, I32, P, P, I32, P, I32, I32, B, I32, P, I64, P, P, SZ, P],
         "dsa_topk_noalloc": [P, I64, B, I32, P, P],
         "dsa_sparse_attn_prefill": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
         "dsa_sparse_attn_decode": [P, I32, P, P, I32, I32, I32, F, P, I32, B, P, P, P, SZ, P],
@@ -147,6 +149,14 @@ def dsa_indexer_scores(q_idx, q_dt: int, w, k_idx_pool, k_dt: int, k_scale_pool,
 def dsa_topk(scores, ld_scores: int, batch: dsa_batch_t, k: int, idx, ws, ws_bytes: int, stream=None):
     _check(load().dsa_topk(_ptr(scores), ld_scores, ctypes.byref(batch), k, _ptr(idx), _ptr(ws), ws_bytes,
                            _stream(stream)), "dsa_topk")
+
+
+def dsa_indexer_topk(q_idx, q_dt: int, w, k_idx_pool, k_dt: int, k_scale_pool, Hi: int, Di: int,
+                     batch: dsa_batch_t, k: int, scores, ld_scores: int, idx, ws, ws_bytes: int, stream=None):
+    """Indexer scores and the top-k selection in one call (the selection fused into the scoring)."""
+    _check(load().dsa_indexer_topk(_ptr(q_idx), q_dt, _ptr(w), _ptr(k_idx_pool), k_dt, _ptr(k_scale_pool), Hi, Di,
+                                   ctypes.byref(batch), k, _ptr(scores), ld_scores, _ptr(idx), _ptr(ws), ws_bytes,
+                                   _stream(stream)), "dsa_indexer_topk")
 
 
 def dsa_topk_noalloc(scores, ld_scores: int, batch: dsa_batch_t, k: int, idx, stream=None):

@@ -22,8 +22,11 @@ dsa_status_t indexer_simt_launch(const void *qI, dsa_dtype_t dt, const float *w,
                                  int64_t ld, cudaStream_t stream);
 dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t *kpool, const float *kscale,
                                const dsa_batch_t *b, float *scores, int64_t ld, void *ws, cudaStream_t stream,
-                               int num_sms, const AppendArgs *app);
+                               int num_sms, const AppendArgs *app, uint32_t *hist);
 size_t indexer_workspace_bytes(int num_seqs, int total_q);
+size_t indexer_hist_bytes(int total_q);
+dsa_status_t select_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx,
+                           const uint32_t *hist, uint32_t *status, cudaStream_t stream, int num_sms);
 dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, int k, float softmax_scale,
                              const dsa_batch_t *b, void *out, float *lse, void *ws, bool decode, cudaStream_t stream,
                              int num_sms);
@@ -148,6 +151,11 @@ static bool is_f32_attn(dsa_dtype_t dt, int H, int Dqk, int Dv, const void *v) {
   return dt == DSA_F32 && H >= 1 && H <= 16 && Dqk >= 1 && Dqk <= 128 && Dv >= 1 && Dv <= 128 && v != nullptr;
 }
 
+// the fused scores + selection call: the indexer's workspace, then the rows' leading-digit histograms
+static size_t indexer_topk_ws_bytes(const dsa_batch_t *b) {
+  return indexer_workspace_bytes(b->num_seqs, b->total_q) + indexer_hist_bytes(b->total_q);
+}
+
 static size_t attn_ws_bytes(const dsa_batch_t *b, int k, int H, int Dv, bool decode) {
   return H == 128 && Dv == 512 ? attn_workspace_bytes(b->total_q, k, decode) : kWsHeader;
 }
@@ -191,6 +199,7 @@ dsa_status_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t *b, int32_t k, in
     case DSA_OP_ATTN_PREFILL: *bytes = attn_ws_bytes(b, k, H, Dv, false); return DSA_OK;
     case DSA_OP_ATTN_DECODE: *bytes = attn_ws_bytes(b, k, H, Dv, true); return DSA_OK;
     case DSA_OP_CACHE_APPEND: *bytes = kWsHeader; return DSA_OK;
+    case DSA_OP_INDEXER_TOPK: *bytes = indexer_topk_ws_bytes(b); return DSA_OK;
   }
   set_error("unknown op %d", (int)op);
   return DSA_ERR_INVALID_ARG;
@@ -220,7 +229,7 @@ dsa_status_t dsa_indexer_scores(const void *q_idx, dsa_dtype_t q_dt, const float
   if ((st = current_device(&dev)) != DSA_OK) return st;
   if (mla)
     return indexer_tc_launch((const uint8_t *)q_idx, w, (const uint8_t *)k_idx_pool, k_scale_pool, b, scores,
-                             ld_scores, ws, (cudaStream_t)stream, dev.num_sms, nullptr);
+                             ld_scores, ws, (cudaStream_t)stream, dev.num_sms, nullptr, nullptr);
   return indexer_simt_launch(q_idx, q_dt, w, k_idx_pool, k_scale_pool, Hi, Di, b, scores, ld_scores,
                              (cudaStream_t)stream);
 }
@@ -239,6 +248,42 @@ dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_batch_t 
   DeviceInfo dev;
   if ((st = current_device(&dev)) != DSA_OK) return st;
   return topk_launch(scores, ld_scores, b, k, idx, ws, (cudaStream_t)stream, dev.num_sms);
+}
+
+dsa_status_t dsa_indexer_topk(const void *q_idx, dsa_dtype_t q_dt, const float *w, const void *k_idx_pool,
+                              dsa_dtype_t k_dt, const float *k_scale_pool, int32_t Hi, int32_t Di, const dsa_batch_t *b,
+                              int32_t k, float *scores, int64_t ld_scores, int32_t *idx, void *ws, size_t ws_bytes,
+                              void *stream) {
+  dsa_status_t st = check_batch(b);
+  if (st != DSA_OK) return st;
+  if (b->total_q == 0) return DSA_OK;   // empty batch: nothing to enqueue, data pointers may be NULL
+  CHECK_ARG(q_idx && w && k_idx_pool && scores && idx, "q_idx, w, k_idx_pool, scores and idx are required");
+  CHECK_ARG(q_dt == k_dt, "query and key dtypes differ");
+  CHECK_SUP(k >= 1 && k <= 16384, "k must be in [1, 16384] (got %d)", k);
+  CHECK_ARG(ld_scores >= b->max_seq_len && ld_scores % 4 == 0,
+            "ld_scores (%lld) must be >= max_seq_len and a multiple of 4", (long long)ld_scores);
+  CHECK_ARG(((uintptr_t)scores & 15) == 0, "scores must be 16-byte aligned");
+  const bool mla = q_dt == DSA_FP8_E4M3 && Hi == 64 && Di == 128;
+  const bool f32 = q_dt == DSA_F32 && Hi >= 1 && Hi <= 16 && Di >= 1 && Di <= 128;
+  CHECK_SUP(mla || f32, "indexer supports e4m3 with Hi=64, Di=128 or f32 with Hi<=16, Di<=128");
+  CHECK_ARG(mla ? k_scale_pool != nullptr : k_scale_pool == nullptr,
+            "k_scale_pool is required for e4m3 keys and must be NULL for f32 keys");
+  CHECK_ARG((((uintptr_t)q_idx | (uintptr_t)w | (uintptr_t)k_idx_pool | (uintptr_t)k_scale_pool) & 15) == 0,
+            "q_idx, w, k_idx_pool and k_scale_pool must be 16-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, indexer_topk_ws_bytes(b))) != DSA_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != DSA_OK) return st;
+  if (mla) {
+    uint32_t *hist = (uint32_t *)((char *)ws + indexer_workspace_bytes(b->num_seqs, b->total_q));
+    st = indexer_tc_launch((const uint8_t *)q_idx, w, (const uint8_t *)k_idx_pool, k_scale_pool, b, scores, ld_scores,
+                           ws, (cudaStream_t)stream, dev.num_sms, nullptr, hist);
+    if (st != DSA_OK) return st;
+    return select_launch(scores, ld_scores, b, k, idx, hist, (uint32_t *)ws, (cudaStream_t)stream, dev.num_sms);
+  }
+  // fp32 indexer (CUDA cores): the selection counts the leading digit itself
+  st = indexer_simt_launch(q_idx, q_dt, w, k_idx_pool, k_scale_pool, Hi, Di, b, scores, ld_scores, (cudaStream_t)stream);
+  if (st != DSA_OK) return st;
+  return select_launch(scores, ld_scores, b, k, idx, nullptr, (uint32_t *)ws, (cudaStream_t)stream, dev.num_sms);
 }
 
 dsa_status_t dsa_topk_noalloc(const float *scores, int64_t ld_scores, const dsa_batch_t *b, int32_t k,
@@ -356,7 +401,7 @@ dsa_status_t dsa_indexer_scores_append(const void *kv_new, dsa_dtype_t kv_dt, co
   const AppendArgs app{(const uint4 *)kv_new, k_new, k_new_dt == DSA_BF16 ? 1 : 0, (uint4 *)kv_pool,
                        (uint32_t *)k_idx_pool, k_scale_pool};
   return indexer_tc_launch((const uint8_t *)q_idx, w, (const uint8_t *)k_idx_pool, k_scale_pool, b, scores, ld_scores,
-                           ws, (cudaStream_t)stream, dev.num_sms, &app);
+                           ws, (cudaStream_t)stream, dev.num_sms, &app, nullptr);
 }
 
 dsa_status_t dsa_reuse_candidates(const int32_t *prev_idx, int32_t k, const int32_t *prev_lens, int32_t max_new,

@@ -22,6 +22,8 @@
 //   warps 2..5   epilogue: tcgen05.ld 64 heads per row, ReLU, weight, sum, key scale, causal store
 // Work units are (row group, key tile) pairs in group order, split evenly over the CTAs; a one-CTA
 // plan kernel enumerates the groups and their tile counts in the workspace first.
+#include <algorithm>
+
 #include "append.cuh"
 #include "tc.cuh"
 
@@ -36,6 +38,11 @@ constexpr uint32_t kIdxTileBytes = kIdxTile * kIdxDi;         // 16 KB
 constexpr uint32_t kIdxPageBytes = 64 * kIdxDi;               // 8 KB
 constexpr uint32_t kIdxBSlotBytes = kIdxRows * kIdxHi * kIdxDi;  // 32 KB
 constexpr uint32_t kIdxWSlotBytes = kIdxRows * kIdxHi * 4;       // 1 KB
+// Leading-digit histograms for the selection step: per row of a group, 2048 bins of the top 11 bits of each
+// score's order-preserving key, as 16-bit counters packed in pairs; flushed to global memory (adds of the
+// non-zero bins) when the group changes and before a counter could pass 65535 (511 tiles of 128 keys).
+constexpr int kIdxHistBins = 2048;
+constexpr int kIdxHistFlushTiles = 511;
 
 // ------------------------------------------------------------------------------------------------ plan
 // workspace (after the header): int32 [0] = G, [1] = U, then arrays
@@ -140,6 +147,20 @@ __global__ void __launch_bounds__(1024) indexer_plan_kernel(BatchView bv, IdxPla
   indexer_plan_body(bv, pv, tmp, s_carry);
 }
 
+// The plan (CTA 0) and, over the whole grid, the zeroing of the rows' leading-digit histograms that the
+// main kernel's epilogue accumulates for the selection step (hist_words u32, a multiple of 4).
+__global__ void __launch_bounds__(1024) indexer_prep_kernel(BatchView bv, IdxPlanView pv, uint32_t *hist,
+                                                            int64_t hist_words) {
+  __shared__ uint32_t tmp[64];
+  __shared__ uint32_t s_carry;
+  pdl_wait();
+  pdl_trigger();
+  uint4 *h4 = reinterpret_cast<uint4 *>(hist);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < hist_words / 4; i += (int64_t)gridDim.x * blockDim.x)
+    h4[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (blockIdx.x == 0) indexer_plan_body(bv, pv, tmp, s_carry);
+}
+
 // The decode step's cache update fused into its first kernel: the 32 warps append the batch's new tokens
 // (one warp per token, append.cuh), then the CTA builds the plan.  The indexer's main kernel, which reads
 // the new keys, starts its work only once this kernel has completed.
@@ -180,14 +201,15 @@ __device__ __forceinline__ void unit_locate(const int32_t *tile_prefix, int G, i
 __global__ void __launch_bounds__(kIdxThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                   const float *__restrict__ kscale, const float *__restrict__ w, BatchView bv, IdxPlanView pv,
-                  float *__restrict__ scores, int64_t ld, uint32_t *status) {
+                  float *__restrict__ scores, int64_t ld, uint32_t *status, uint32_t *__restrict__ hist) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sA = smem;                                             // kIdxStages x 16 KB
   uint8_t *sB = sA + kIdxStages * kIdxTileBytes;                  // 2 x 32 KB
   float *sW = (float *)(sB + 2 * kIdxBSlotBytes);                 // 2 x 1 KB
   float *sKS = sW + 2 * (kIdxWSlotBytes / 4);                     // kIdxStages x 128 key scales
-  IdxSmem *S = (IdxSmem *)(sKS + kIdxStages * kIdxTile);
+  uint32_t *sHist = (uint32_t *)(sKS + kIdxStages * kIdxTile);    // kIdxRows x 2048 16-bit counters
+  IdxSmem *S = (IdxSmem *)(sHist + kIdxRows * (kIdxHistBins / 2));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -383,15 +405,47 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       // ------------------------------------------------------------------ epilogue
       const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
       const int key_local = quad * 32 + lane;
+      const int et = threadIdx.x - 64;           // 0..127 over the four epilogue warps
+      // With histograms on, the four warps meet at named barrier 1 around every flush, so the loop never
+      // leaves early then: after a timeout the waits return at once and the remaining units pass through
+      // without touching TMEM or global memory.
+      if (hist != nullptr) {
+        for (int j = et; j < kIdxRows * (kIdxHistBins / 2); j += 128) sHist[j] = 0u;
+        tc::named_bar_sync(1, 128);
+      }
       int gi, t;
       unit_locate(pv.tile_prefix, G, u0, &gi, &t);
-      int acc = 0, nb_groups = 0, bslot = 0, cur = -1;
+      int acc = 0, nb_groups = 0, bslot = 0, cur = -1, span = 0;
       uint32_t acc_phase = 0;
       int b = 0, row0 = 0, nr = 0, pos0 = 0;
+      bool ok = true;
+      // adds this CTA's counts of the current group's rows to their global histograms and clears them
+      auto flush = [&]() {
+        tc::named_bar_sync(1, 128);
+        for (int q = 0; q < nr; ++q) {
+          uint32_t *hg = hist + (int64_t)(row0 + q) * kIdxHistBins;
+          uint32_t *hs = sHist + q * (kIdxHistBins / 2);
+          for (int j = et; j < kIdxHistBins / 2; j += 128) {
+            const uint32_t v = hs[j];
+            if (v != 0u) {
+              if (ok) {
+                if (v & 0xFFFFu) atomicAdd(hg + 2 * j, v & 0xFFFFu);
+                if (v >> 16) atomicAdd(hg + 2 * j + 1, v >> 16);
+              }
+              hs[j] = 0u;
+            }
+          }
+        }
+        tc::named_bar_sync(1, 128);
+        span = 0;
+      };
       for (int u = u0; u < u1; ++u) {
         if (gi != cur) {
+          if (hist != nullptr && cur >= 0) flush();
           bslot = nb_groups & 1;
-          if (!__all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort, status))) break;
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort,
+                                                     status)) && ok;
+          if (!ok && hist == nullptr) break;
           ++nb_groups;
           cur = gi;
           b = pv.g_seq[gi];
@@ -399,47 +453,61 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           nr = pv.g_nrows[gi];
           const int c0 = __ldg(bv.cu_q + b);
           pos0 = __ldg(bv.seq_lens + b) - (__ldg(bv.cu_q + b + 1) - c0) + (row0 - c0);
+        } else if (hist != nullptr && span == kIdxHistFlushTiles) {
+          flush();
         }
         const int s = t * kIdxTile + key_local;
-        // the TMEM loads below are warp-collective: leave the loop together or not at all
-        if (!__all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->tfull[acc]), acc_phase, abort, status))) break;
-        tc::fence_after_sync();
-        // the tile's key scales arrived with it; the stage's fill has completed (the MMA consumed it), the
-        // wait below returns at once and orders the bulk copy before these reads
-        const int stage = (u - u0) % kIdxStages;
-        tc::mbar_wait(tc::smem_u32(&S->full[stage]), (uint32_t)((u - u0) / kIdxStages) & 1u, abort, status);
-        const float ks = sKS[stage * kIdxTile + key_local];
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->empty[stage]));
-        const float *wq = sW + bslot * (kIdxWSlotBytes / 4);
-        const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + acc * 256;
-        for (int q = 0; q < nr; ++q) {
-          float v0[32], v1[32];
-          tc::tmem_ld32(tbase + q * 64, v0);
-          tc::tmem_ld32(tbase + q * 64 + 32, v1);
-          tc::tmem_wait_ld();
-          const float *wr = wq + q * kIdxHi;
-          float a0 = 0.f, a1 = 0.f;
+        // the TMEM loads below are warp-collective: the warp takes them together or not at all
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->tfull[acc]), acc_phase, abort, status)) && ok;
+        if (!ok && hist == nullptr) break;
+        if (ok) {
+          tc::fence_after_sync();
+          // the tile's key scales arrived with it; the stage's fill has completed (the MMA consumed it), the
+          // wait below returns at once and orders the bulk copy before these reads
+          const int stage = (u - u0) % kIdxStages;
+          tc::mbar_wait(tc::smem_u32(&S->full[stage]), (uint32_t)((u - u0) / kIdxStages) & 1u, abort, status);
+          const float ks = sKS[stage * kIdxTile + key_local];
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->empty[stage]));
+          const float *wq = sW + bslot * (kIdxWSlotBytes / 4);
+          const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + acc * 256;
+          for (int q = 0; q < nr; ++q) {
+            float v0[32], v1[32];
+            tc::tmem_ld32(tbase + q * 64, v0);
+            tc::tmem_ld32(tbase + q * 64 + 32, v1);
+            tc::tmem_wait_ld();
+            const float *wr = wq + q * kIdxHi;
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-          for (int h = 0; h < 32; h += 2) {
-            a0 = fmaf(wr[h], fmaxf(v0[h], 0.f), a0);
-            a1 = fmaf(wr[h + 1], fmaxf(v0[h + 1], 0.f), a1);
-          }
+            for (int h = 0; h < 32; h += 2) {
+              a0 = fmaf(wr[h], fmaxf(v0[h], 0.f), a0);
+              a1 = fmaf(wr[h + 1], fmaxf(v0[h + 1], 0.f), a1);
+            }
 #pragma unroll
-          for (int h = 0; h < 32; h += 2) {
-            a0 = fmaf(wr[32 + h], fmaxf(v1[h], 0.f), a0);
-            a1 = fmaf(wr[33 + h], fmaxf(v1[h + 1], 0.f), a1);
+            for (int h = 0; h < 32; h += 2) {
+              a0 = fmaf(wr[32 + h], fmaxf(v1[h], 0.f), a0);
+              a1 = fmaf(wr[33 + h], fmaxf(v1[h + 1], 0.f), a1);
+            }
+            if (s <= pos0 + q) {
+              const float sc = (a0 + a1) * ks;
+              scores[(int64_t)(row0 + q) * ld + s] = sc;
+              if (hist != nullptr) {
+                const uint32_t d = ordered_key(sc) >> 21;
+                atomicAdd(&sHist[q * (kIdxHistBins / 2) + (d >> 1)], (d & 1u) ? 0x10000u : 1u);
+              }
+            }
           }
-          if (s <= pos0 + q) scores[(int64_t)(row0 + q) * ld + s] = (a0 + a1) * ks;
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->tempty[acc]));
+          const bool last_of_group = (t + 1 == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) || (u + 1 == u1);
+          if (last_of_group && lane == 0) tc::mbar_arrive(tc::smem_u32(&S->bempty[bslot]));
         }
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->tempty[acc]));
-        const bool last_of_group = (t + 1 == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) || (u + 1 == u1);
-        if (last_of_group && lane == 0) tc::mbar_arrive(tc::smem_u32(&S->bempty[bslot]));
+        ++span;
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         if (++t == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) { ++gi; t = 0; }
       }
+      if (hist != nullptr && cur >= 0) flush();
     }
   }
   tc::fence_before_sync();
@@ -483,15 +551,17 @@ static bool make_rows128_map(CUtensorMap *m, const void *base, uint64_t rows) {
 
 static size_t indexer_tc_smem() {
   return 1024 + kIdxStages * kIdxTileBytes + 2 * kIdxBSlotBytes + 2 * kIdxWSlotBytes + kIdxStages * kIdxTile * 4 +
-         sizeof(IdxSmem);
+         kIdxRows * (kIdxHistBins / 2) * 4 + sizeof(IdxSmem);
 }
+
+size_t indexer_hist_bytes(int total_q) { return al256((size_t)total_q * kIdxHistBins * 4); }
 
 dsa_status_t cache_append_launch(const void *kv_new, const void *k_new, bool k_bf16, const dsa_batch_t *b,
                                  void *kv_pool, void *kI_pool, float *kS_pool, void *ws, cudaStream_t stream);
 
 dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t *kpool, const float *kscale,
                                const dsa_batch_t *b, float *scores, int64_t ld, void *ws, cudaStream_t stream,
-                               int num_sms, const AppendArgs *app) {
+                               int num_sms, const AppendArgs *app, uint32_t *hist) {
   BatchView bv = view_of(b);
   IdxPlanView pv = plan_view(ws, b->num_seqs, b->total_q);
   CUtensorMap tm_k, tm_q;
@@ -500,7 +570,7 @@ dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t 
     set_error("indexer: cuTensorMapEncodeTiled failed");
     return DSA_ERR_CUDA;
   }
-  if (app != nullptr && b->total_q <= kIdxFusedAppendMaxRows) {
+  if (app != nullptr && hist == nullptr && b->total_q <= kIdxFusedAppendMaxRows) {
     DSA_LAUNCH_PDL("indexer_plan_append_kernel", indexer_plan_append_kernel, dim3(1), dim3(1024), 0, stream, bv, pv,
                    *app, b->total_q, (uint32_t *)ws);
   } else {
@@ -509,12 +579,19 @@ dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t 
                                                   app->kI_pool, app->kS_pool, ws, stream);
       if (st != DSA_OK) return st;
     }
-    DSA_LAUNCH_PDL("indexer_plan_kernel", indexer_plan_kernel, dim3(1), dim3(1024), 0, stream, bv, pv);
+    if (hist != nullptr) {
+      // the histograms are cleared here, a stream step ahead of the kernel that adds into them
+      const int64_t words = (int64_t)b->total_q * kIdxHistBins;
+      const int grid = (int)std::min<int64_t>(num_sms, std::max<int64_t>(1, words / (4 * 1024 * 4)));
+      DSA_LAUNCH_PDL("indexer_prep_kernel", indexer_prep_kernel, dim3(grid), dim3(1024), 0, stream, bv, pv, hist, words);
+    } else {
+      DSA_LAUNCH_PDL("indexer_plan_kernel", indexer_plan_kernel, dim3(1), dim3(1024), 0, stream, bv, pv);
+    }
   }
   const size_t smem = indexer_tc_smem();
   cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   DSA_LAUNCH_PDL("indexer_tc_kernel", indexer_tc_kernel, dim3(num_sms), dim3(kIdxThreads), smem, stream, tm_k, tm_q,
-                 kscale, w, bv, pv, scores, ld, (uint32_t *)ws);
+                 kscale, w, bv, pv, scores, ld, (uint32_t *)ws, hist);
   return DSA_OK;
 }
 

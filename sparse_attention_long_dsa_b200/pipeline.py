@@ -78,6 +78,7 @@ class DeviceBatch:
         op_attn = B.DSA_OP_ATTN_DECODE if decode else B.DSA_OP_ATTN_PREFILL
         self.ws_bytes = max(B.dsa_workspace_size(B.DSA_OP_INDEXER, self.batch),
                             B.dsa_workspace_size(B.DSA_OP_TOPK, self.batch, wl.topk),
+                            B.dsa_workspace_size(B.DSA_OP_INDEXER_TOPK, self.batch, wl.topk),
                             B.dsa_workspace_size(op_attn, self.batch, wl.topk, wl.H, wl.Dv))
         self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dv)
 
@@ -103,6 +104,13 @@ class DeviceBatch:
         B.dsa_indexer_scores_append(kv_new, self.dt, k_new, k_dt, self.kv_pool, self.qI, self.idx_dt, self.w,
                                     self.kI_pool, self.idx_dt, self.kS_pool, wl.Hi, wl.Di, self.batch, self.scores,
                                     self.ld, self.ws, self.ws_bytes, stream)
+
+    def indexer_topk(self, stream=None):
+        """Scores and selection in one call (the selection fused into the scoring): the same scores and idx
+        as indexer() followed by topk()."""
+        wl = self.wl
+        B.dsa_indexer_topk(self.qI, self.idx_dt, self.w, self.kI_pool, self.idx_dt, self.kS_pool, wl.Hi, wl.Di,
+                           self.batch, wl.topk, self.scores, self.ld, self.idx, self.ws, self.ws_bytes, stream)
 
     def topk(self, stream=None, scores=None):
         B.dsa_topk(self.scores if scores is None else scores, self.ld, self.batch, self.wl.topk, self.idx, self.ws,
@@ -173,9 +181,13 @@ class DeviceBatch:
         B.dsa_expand_blocks(self.blk_idx, kb, self.batch, self.idx_blk, stream)
         return self.idx_blk
 
-    def run(self, stream=None):
-        self.indexer(stream)
-        self.topk(stream)
+    def run(self, stream=None, fused=False):
+        """One pass of the path: scores, selection, attention (fused=True: scores and selection in one call)."""
+        if fused:
+            self.indexer_topk(stream)
+        else:
+            self.indexer(stream)
+            self.topk(stream)
         self.attention(stream)
 
     def check_status(self, stream=None):

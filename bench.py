@@ -185,12 +185,19 @@ def _time_steps(replicas, stream, steps, warmup, world, dev, sampler=None):
     stages = ("indexer", "topk", "attention")
 
     def step(db, ev=None):
+        # the first two steps as the pipeline runs them: one fused call for batches where that is faster
+        # (its time is then reported under "indexer", "topk" holding the empty interval), else two calls
+        fused = db.prefers_fused()
         if ev is not None:
             ev[0].record(stream)
-        db.indexer(stream)
+        if fused:
+            db.indexer_topk(stream)
+        else:
+            db.indexer(stream)
         if ev is not None:
             ev[1].record(stream)
-        db.topk(stream)
+        if not fused:
+            db.topk(stream)
         if ev is not None:
             ev[2].record(stream)
         db.attention(stream)
@@ -233,6 +240,60 @@ def _time_steps(replicas, stream, steps, warmup, world, dev, sampler=None):
     return total_ms, stage_avg, int(launches), clocks
 
 
+def time_widened(replicas, stream, dev, reps=50):
+    """Per-call device times (CUDA events, inputs rotating over the replicas) of the decode step's variants
+    against the calls they replace: the fused scores + selection (dsa_indexer_topk) against
+    dsa_indexer_scores + dsa_topk; the cache append fused into the indexer (dsa_indexer_scores_append)
+    against dsa_indexer_scores alone and against dsa_cache_append + dsa_indexer_scores; the block-granular
+    selection (32 pages of 64) and the decode index reuse (the previous selection plus the newest token)
+    against the full top-k.  Times in microseconds."""
+    import torch
+    from sparse_attention_long_dsa_b200 import binding as B
+    wl = replicas[0].wl
+    T = wl.total_q
+    g = torch.Generator(device="cpu").manual_seed(7)
+    kv_new = (torch.randn((T, wl.Dqk), generator=g) * 1.0).to(torch.bfloat16).to(dev)
+    k_new = torch.randn((T, wl.Di), generator=g).to(dev)
+    prev_lens = [torch.clamp(db.seq_lens - 1, min=1) for db in replicas]
+    for db in replicas:
+        db.indexer(stream)
+        db.topk(stream)
+    torch.cuda.synchronize(dev)
+    prev_idx = [db.idx.clone() for db in replicas]
+
+    def t(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for i in range(len(replicas)):
+                fn(i)
+            e0.record(stream)
+            for i in range(reps):
+                fn(i % len(replicas))
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps * 1e3
+
+    def append_sep(i):
+        db = replicas[i]
+        B.dsa_cache_append(kv_new, B.DSA_BF16, k_new, B.DSA_F32, wl.Dqk, wl.Di, db.batch, db.kv_pool, db.kI_pool,
+                           db.kS_pool, db.ws, db.ws_bytes, stream)
+        db.indexer(stream)
+
+    res = {
+        "indexer": t(lambda i: replicas[i].indexer(stream)),
+        "topk": t(lambda i: replicas[i].topk(stream)),
+        "indexer_topk_fused": t(lambda i: replicas[i].indexer_topk(stream)),
+        "cache_append_then_indexer": t(append_sep),
+        "indexer_with_fused_append": t(lambda i: replicas[i].append_and_indexer(kv_new, k_new, B.DSA_F32, stream)),
+        "block_select_32_pages": t(lambda i: replicas[i].block_select(32, stream)),
+        "index_reuse_select": t(lambda i: replicas[i].reuse_select(prev_idx[i], prev_lens[i], 1, stream)),
+    }
+    for db in replicas:
+        db.check_status(stream)
+    res["unit"] = "us per call (device, CUDA events)"
+    return res
+
+
 # the other MLA workloads timed by the default run, each a 1-GPU figure of its own
 EXTRA_WORKLOADS = ("prefill_16k", "decode_1m_planted", "mixed_batch")
 
@@ -263,7 +324,25 @@ def run_extra_workload(name, args, dev, stream, sampler):
            "stage_rooflines": {s: roofline_entry(s, stage_avg[s], work, peaks, peak_src, name, decode)
                                for s in ("indexer", "attention")},
            "step_roofline": step_roofline(work, peaks, ms_per_step), "gpu_launches": launches, "clocks": clocks,
+           "selection": "dsa_indexer_topk (fused; stages_ms.indexer holds scores + selection)" if db.prefers_fused()
+           else "dsa_indexer_scores + dsa_topk",
            "config": workload_config(wl, replicas=1, l2="inputs larger than L2 (one device replica)")}
+    # both forms of the first two steps, for the choice between them
+    def t2(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            fn()
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n
+    n2 = max(3, min(50, steps))
+    res["scores_and_selection_ms"] = {
+        "dsa_indexer_scores + dsa_topk": t2(lambda: (db.indexer(stream), db.topk(stream)), n2),
+        "dsa_indexer_topk (fused)": t2(lambda: db.indexer_topk(stream), n2)}
+    db.check_status(stream)
     del db
     torch.cuda.synchronize(dev)
     torch.cuda.empty_cache()
@@ -318,6 +397,8 @@ def run_ours(args, rank, world, local_rank):
     }
     if wl.kind == "mla":
         res["step_roofline"] = step_roofline(work, peaks, ms_per_step)
+    if world == 1 and args.workload == "decode_batch" and not args.no_widened:
+        res["widened"] = time_widened(replicas, stream, dev)
     del replicas
     torch.cuda.synchronize(dev)
     torch.cuda.empty_cache()
@@ -624,6 +705,7 @@ def main():
     ap.add_argument("--extra-workloads", default=",".join(EXTRA_WORKLOADS),
                     help="comma-separated MLA workloads timed after the decode batch at N=1 ('' for none)")
     ap.add_argument("--extra-steps", type=int, default=10)
+    ap.add_argument("--no-widened", action="store_true", help="skip the timing of the decode step's variants")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -688,31 +688,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
 
 // ------------------------------------------------------------------------------------------------ combine
 // out[row, h, :] = sum_s exp(lse_s - lse) o_s,  lse = log sum_s exp(lse_s)   (splits of one row)
+// The splits' lse values are read once into registers (up to kCombineRegSplits of them; more are re-read), so
+// a thread waits on two rounds of loads: the lse values, then all splits' partial outputs at once.
+constexpr int kCombineRegSplits = 8;
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restrict__ part_o,
                                                            const float *__restrict__ part_lse, int splits,
                                                            __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
   pdl_wait();
   pdl_trigger();
   const int row = blockIdx.x, h = blockIdx.y;
+  const float *pl = part_lse + (int64_t)row * splits * kAttH + h;
+  float lreg[kCombineRegSplits];
+#pragma unroll
+  for (int s = 0; s < kCombineRegSplits; ++s) lreg[s] = s < splits ? __ldg(pl + (int64_t)s * kAttH) : -INFINITY;
   float mx = -INFINITY;
-  for (int s = 0; s < splits; ++s) mx = fmaxf(mx, __ldg(part_lse + ((int64_t)row * splits + s) * kAttH + h));
+#pragma unroll
+  for (int s = 0; s < kCombineRegSplits; ++s) mx = fmaxf(mx, lreg[s]);
+  for (int s = kCombineRegSplits; s < splits; ++s) mx = fmaxf(mx, __ldg(pl + (int64_t)s * kAttH));
   float tot = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float l = __ldg(part_lse + ((int64_t)row * splits + s) * kAttH + h);
+#pragma unroll
+  for (int s = 0; s < kCombineRegSplits; ++s)
+    if (s < splits) tot += lreg[s] == -INFINITY ? 0.f : __expf(lreg[s] - mx);
+  for (int s = kCombineRegSplits; s < splits; ++s) {
+    const float l = __ldg(pl + (int64_t)s * kAttH);
     tot += l == -INFINITY ? 0.f : __expf(l - mx);
   }
   const int dv = threadIdx.x * 4;
+  const float *po = part_o + ((int64_t)row * splits * kAttH + h) * kAttDv + dv;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (tot > 0.f) {
-    for (int s = 0; s < splits; ++s) {
-      const float l = __ldg(part_lse + ((int64_t)row * splits + s) * kAttH + h);
+    float4 o[kCombineRegSplits];
+#pragma unroll
+    for (int s = 0; s < kCombineRegSplits; ++s)
+      o[s] = (s < splits && lreg[s] != -INFINITY) ? __ldg(reinterpret_cast<const float4 *>(po + (int64_t)s * kAttH * kAttDv))
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < kCombineRegSplits; ++s) {
+      if (s >= splits || lreg[s] == -INFINITY) continue;
+      const float wgt = __expf(lreg[s] - mx) / tot;
+      acc.x += wgt * o[s].x;
+      acc.y += wgt * o[s].y;
+      acc.z += wgt * o[s].z;
+      acc.w += wgt * o[s].w;
+    }
+    for (int s = kCombineRegSplits; s < splits; ++s) {
+      const float l = __ldg(pl + (int64_t)s * kAttH);
       if (l == -INFINITY) continue;
       const float wgt = __expf(l - mx) / tot;
-      const float4 o = __ldg(reinterpret_cast<const float4 *>(part_o + (((int64_t)row * splits + s) * kAttH + h) * kAttDv + dv));
-      acc.x += wgt * o.x;
-      acc.y += wgt * o.y;
-      acc.z += wgt * o.z;
-      acc.w += wgt * o.w;
+      const float4 os = __ldg(reinterpret_cast<const float4 *>(po + (int64_t)s * kAttH * kAttDv));
+      acc.x += wgt * os.x;
+      acc.y += wgt * os.y;
+      acc.z += wgt * os.z;
+      acc.w += wgt * os.w;
     }
   }
   __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x, acc.y), b1 = __floats2bfloat162_rn(acc.z, acc.w);

@@ -43,6 +43,10 @@ constexpr uint32_t kIdxWSlotBytes = kIdxRows * kIdxHi * 4;       // 1 KB
 // non-zero bins) when the group changes and before a counter could pass 65535 (511 tiles of 128 keys).
 constexpr int kIdxHistBins = 2048;
 constexpr int kIdxHistFlushTiles = 511;
+// Decode batches (one query row per sequence, so row g is sequence g and a group is one row) of up to this
+// many rows are planned inside the main kernel: each CTA scans the rows' tile counts into shared memory,
+// with no plan kernel in front and no chain of dependent plan reads before its first copy.
+constexpr int kIdxInlinePlanMax = 1024;
 
 // ------------------------------------------------------------------------------------------------ plan
 // workspace (after the header): int32 [0] = G, [1] = U, then arrays
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(1024) indexer_plan_kernel(BatchView bv, IdxPla
 // The plan (CTA 0) and, over the whole grid, the zeroing of the rows' leading-digit histograms that the
 // main kernel's epilogue accumulates for the selection step (hist_words u32, a multiple of 4).
 __global__ void __launch_bounds__(1024) indexer_prep_kernel(BatchView bv, IdxPlanView pv, uint32_t *hist,
-                                                            int64_t hist_words) {
+                                                            int64_t hist_words, int do_plan) {
   __shared__ uint32_t tmp[64];
   __shared__ uint32_t s_carry;
   pdl_wait();
@@ -158,7 +162,7 @@ __global__ void __launch_bounds__(1024) indexer_prep_kernel(BatchView bv, IdxPla
   uint4 *h4 = reinterpret_cast<uint4 *>(hist);
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < hist_words / 4; i += (int64_t)gridDim.x * blockDim.x)
     h4[i] = make_uint4(0u, 0u, 0u, 0u);
-  if (blockIdx.x == 0) indexer_plan_body(bv, pv, tmp, s_carry);
+  if (do_plan && blockIdx.x == 0) indexer_plan_body(bv, pv, tmp, s_carry);
 }
 
 // The decode step's cache update fused into its first kernel: the 32 warps append the batch's new tokens
@@ -188,20 +192,25 @@ struct IdxSmem {
 };
 
 // position of unit u: group index and tile within the group
+// (tile_prefix is in global memory, or in shared memory for the in-kernel decode plan: plain loads)
 __device__ __forceinline__ void unit_locate(const int32_t *tile_prefix, int G, int u, int *gi, int *t) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(tile_prefix + mid) <= u) lo = mid; else hi = mid - 1;
+    if (tile_prefix[mid] <= u) lo = mid; else hi = mid - 1;
   }
   *gi = lo;
-  *t = u - __ldg(tile_prefix + lo);
+  *t = u - tile_prefix[lo];
 }
 
+// kHist: the epilogue also counts each row's leading-digit histogram (the fused selection); without it the
+// kernel is compiled with none of that code.
+template <bool kHist>
 __global__ void __launch_bounds__(kIdxThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                   const float *__restrict__ kscale, const float *__restrict__ w, BatchView bv, IdxPlanView pv,
-                  float *__restrict__ scores, int64_t ld, uint32_t *status, uint32_t *__restrict__ hist) {
+                  float *__restrict__ scores, int64_t ld, uint32_t *status, uint32_t *__restrict__ hist,
+                  int inline_plan) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sA = smem;                                             // kIdxStages x 16 KB
@@ -209,7 +218,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   float *sW = (float *)(sB + 2 * kIdxBSlotBytes);                 // 2 x 1 KB
   float *sKS = sW + 2 * (kIdxWSlotBytes / 4);                     // kIdxStages x 128 key scales
   uint32_t *sHist = (uint32_t *)(sKS + kIdxStages * kIdxTile);    // kIdxRows x 2048 16-bit counters
-  IdxSmem *S = (IdxSmem *)(sHist + kIdxRows * (kIdxHistBins / 2));
+  int32_t *sTP = (int32_t *)(sHist + kIdxRows * (kIdxHistBins / 2));   // in-kernel plan: tile prefix
+  IdxSmem *S = (IdxSmem *)(sTP + kIdxInlinePlanMax + 4);
+  __shared__ uint32_t s_scan[64];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -242,7 +253,32 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   // the plan (and the inputs) come from earlier work on the stream
   pdl_wait();
   pdl_trigger();
-  const int G = pv.hdr[0], U = pv.hdr[1];
+  int G, U;
+  const int32_t *tp;
+  if (inline_plan) {
+    // row g = sequence g, one group per row: its tiles cover keys 0 .. seq_lens[g] - 1
+    G = bv.num_seqs;
+    uint32_t carry = 0;
+    for (int base = 0; base < G; base += kIdxThreads) {
+      const int g = base + (int)threadIdx.x;
+      const uint32_t tiles = g < G ? (uint32_t)((__ldg(bv.seq_lens + g) - 1) / kIdxTile + 1) : 0u;
+      uint32_t tot;
+      const uint32_t ex = block_exclusive_scan(tiles, s_scan, &tot);
+      if (g < G) sTP[g] = (int)(carry + ex);
+      carry += tot;
+    }
+    if (threadIdx.x == 0) sTP[G] = (int)carry;
+    __syncthreads();
+    U = (int)carry;
+    tp = sTP;
+  } else {
+    G = pv.hdr[0];
+    U = pv.hdr[1];
+    tp = pv.tile_prefix;
+  }
+  auto g_seq = [&](int g) { return inline_plan ? g : pv.g_seq[g]; };
+  auto g_row0 = [&](int g) { return inline_plan ? g : pv.g_row0[g]; };
+  auto g_nrows = [&](int g) { return inline_plan ? 1 : pv.g_nrows[g]; };
   const int u0 = (int)(((int64_t)blockIdx.x * U) / gridDim.x);
   const int u1 = (int)(((int64_t)(blockIdx.x + 1) * U) / gridDim.x);
 
@@ -262,7 +298,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const int bslot = nbg & 1;
         const uint32_t use = (uint32_t)(nbg >> 1);
         if (!tc::mbar_wait(tc::smem_u32(&S->bempty[bslot]), (use & 1u) ^ 1u, abort, status)) return false;
-        const int row0 = pv.g_row0[gj], nr = pv.g_nrows[gj];
+        const int row0 = g_row0(gj), nr = g_nrows(gj);
         const uint32_t bar = tc::smem_u32(&S->bfull[bslot]);
         tc::mbar_expect_tx(bar, (uint32_t)nr * (kIdxHi * kIdxDi + kIdxHi * 4));
         for (int q = 0; q < nr; ++q) {
@@ -278,8 +314,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       int g_next = 0, g_cur = -1, g_count = 0, g_last = -1;   // warp 0: groups loaded so far
       if (pw == 0) {
         int t0;
-        unit_locate(pv.tile_prefix, G, u0, &g_next, &t0);
-        unit_locate(pv.tile_prefix, G, u1 - 1, &g_last, &t0);
+        unit_locate(tp, G, u0, &g_next, &t0);
+        unit_locate(tp, G, u1 - 1, &g_last, &t0);
       }
       const int mine = (u1 - u0 - pw + 3) / 4;              // tiles of this warp: u0 + pw + 4 m
       for (int mb = 0; mb < mine && ok; mb += 32) {
@@ -288,10 +324,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const int u = u0 + pw + 4 * m;
         int gi = 0, t = 0, blk0 = -1, blk1 = -1;
         if (m < mine) {
-          unit_locate(pv.tile_prefix, G, u, &gi, &t);
-          const int b = pv.g_seq[gi];
+          unit_locate(tp, G, u, &gi, &t);
+          const int b = g_seq(gi);
           const int c0 = __ldg(bv.cu_q + b), nbq = __ldg(bv.cu_q + b + 1) - c0;
-          const int pos_last = __ldg(bv.seq_lens + b) - nbq + (pv.g_row0[gi] - c0) + pv.g_nrows[gi] - 1;
+          const int pos_last = __ldg(bv.seq_lens + b) - nbq + (g_row0(gi) - c0) + g_nrows(gi) - 1;
           const int pages = pos_last / 64 + 1;
           const int32_t *btr = bv.block_table + (int64_t)b * bv.max_blocks_per_seq;
           blk0 = __ldg(btr + 2 * t);
@@ -367,7 +403,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     } else if (warp == 1) {
       // ------------------------------------------------------------------ MMA issuer (whole warp, one elected lane issues)
       int gi, t;
-      unit_locate(pv.tile_prefix, G, u0, &gi, &t);
+      unit_locate(tp, G, u0, &gi, &t);
       int stage = 0, acc = 0, nb_groups = 0, bslot = 0, cur = -1;
       uint32_t phase = 0, acc_phase = 0;
       for (int u = u0; u < u1; ++u) {
@@ -380,7 +416,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         if (!tc::mbar_wait_w(tc::smem_u32(&S->tempty[acc]), acc_phase ^ 1u, abort, status)) break;
         tc::fence_after_sync();
         if (!tc::mbar_wait_w(tc::smem_u32(&S->full[stage]), phase, abort, status)) break;
-        const int nr = pv.g_nrows[gi];
+        const int nr = g_nrows(gi);
         const uint32_t idesc = tc::make_idesc(0, 0, 128, 64 * nr, false, false);
         const uint32_t a0 = tc::smem_u32(sA + stage * kIdxTileBytes);
         const uint32_t b0 = tc::smem_u32(sB + bslot * kIdxBSlotBytes);
@@ -391,11 +427,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         }
         tc::mma_commit_w(tc::smem_u32(&S->empty[stage]));
         tc::mma_commit_w(tc::smem_u32(&S->tfull[acc]));
-        const bool last_of_group = (t + 1 == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) || (u + 1 == u1);
+        const bool last_of_group = (t + 1 == tp[gi + 1] - tp[gi]) || (u + 1 == u1);
         if (last_of_group) tc::mma_commit_w(tc::smem_u32(&S->bempty[bslot]));
         if (++stage == kIdxStages) { stage = 0; phase ^= 1u; }
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-        if (++t == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) { ++gi; t = 0; }
+        if (++t == tp[gi + 1] - tp[gi]) { ++gi; t = 0; }
       }
       // every MMA issued by this thread has completed before TMEM is released
       tc::mma_commit_w(tc::smem_u32(&S->drain));
@@ -409,12 +445,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       // With histograms on, the four warps meet at named barrier 1 around every flush, so the loop never
       // leaves early then: after a timeout the waits return at once and the remaining units pass through
       // without touching TMEM or global memory.
-      if (hist != nullptr) {
+      if constexpr (kHist) {
         for (int j = et; j < kIdxRows * (kIdxHistBins / 2); j += 128) sHist[j] = 0u;
         tc::named_bar_sync(1, 128);
       }
       int gi, t;
-      unit_locate(pv.tile_prefix, G, u0, &gi, &t);
+      unit_locate(tp, G, u0, &gi, &t);
       int acc = 0, nb_groups = 0, bslot = 0, cur = -1, span = 0;
       uint32_t acc_phase = 0;
       int b = 0, row0 = 0, nr = 0, pos0 = 0;
@@ -441,25 +477,25 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       };
       for (int u = u0; u < u1; ++u) {
         if (gi != cur) {
-          if (hist != nullptr && cur >= 0) flush();
+          if (kHist && cur >= 0) flush();
           bslot = nb_groups & 1;
           ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort,
                                                      status)) && ok;
-          if (!ok && hist == nullptr) break;
+          if (!kHist && !ok) break;
           ++nb_groups;
           cur = gi;
-          b = pv.g_seq[gi];
-          row0 = pv.g_row0[gi];
-          nr = pv.g_nrows[gi];
+          b = g_seq(gi);
+          row0 = g_row0(gi);
+          nr = g_nrows(gi);
           const int c0 = __ldg(bv.cu_q + b);
           pos0 = __ldg(bv.seq_lens + b) - (__ldg(bv.cu_q + b + 1) - c0) + (row0 - c0);
-        } else if (hist != nullptr && span == kIdxHistFlushTiles) {
+        } else if (kHist && span == kIdxHistFlushTiles) {
           flush();
         }
         const int s = t * kIdxTile + key_local;
         // the TMEM loads below are warp-collective: the warp takes them together or not at all
         ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->tfull[acc]), acc_phase, abort, status)) && ok;
-        if (!ok && hist == nullptr) break;
+        if (!kHist && !ok) break;
         if (ok) {
           tc::fence_after_sync();
           // the tile's key scales arrived with it; the stage's fill has completed (the MMA consumed it), the
@@ -471,7 +507,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->empty[stage]));
           const float *wq = sW + bslot * (kIdxWSlotBytes / 4);
           const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + acc * 256;
-          for (int q = 0; q < nr; ++q) {
+          uint32_t dig[kIdxRows];             // leading digits of this thread's scores (bit 31: none)
+#pragma unroll
+          for (int q = 0; q < kIdxRows; ++q) {
+            dig[q] = 0x80000000u;
+            if (q >= nr) continue;
             float v0[32], v1[32];
             tc::tmem_ld32(tbase + q * 64, v0);
             tc::tmem_ld32(tbase + q * 64 + 32, v1);
@@ -491,23 +531,30 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             if (s <= pos0 + q) {
               const float sc = (a0 + a1) * ks;
               scores[(int64_t)(row0 + q) * ld + s] = sc;
-              if (hist != nullptr) {
-                const uint32_t d = ordered_key(sc) >> 21;
-                atomicAdd(&sHist[q * (kIdxHistBins / 2) + (d >> 1)], (d & 1u) ? 0x10000u : 1u);
-              }
+              if constexpr (kHist) dig[q] = ordered_key(sc) >> 21;
             }
           }
           tc::fence_before_sync();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->tempty[acc]));
-          const bool last_of_group = (t + 1 == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) || (u + 1 == u1);
+          const bool last_of_group = (t + 1 == tp[gi + 1] - tp[gi]) || (u + 1 == u1);
           if (last_of_group && lane == 0) tc::mbar_arrive(tc::smem_u32(&S->bempty[bslot]));
+          if constexpr (kHist) {
+            // counted after the accumulator and the query rows are handed back (an arrive orders every earlier
+            // memory operation of the warp before it, so adds in front of it would hold the tensor core up)
+#pragma unroll
+            for (int q = 0; q < kIdxRows; ++q)
+              if (dig[q] != 0x80000000u) {
+                const uint32_t addr = tc::smem_u32(&sHist[q * (kIdxHistBins / 2) + (dig[q] >> 1)]);
+                asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"((dig[q] & 1u) ? 0x10000u : 1u) : "memory");
+              }
+          }
         }
         ++span;
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-        if (++t == pv.tile_prefix[gi + 1] - pv.tile_prefix[gi]) { ++gi; t = 0; }
+        if (++t == tp[gi + 1] - tp[gi]) { ++gi; t = 0; }
       }
-      if (hist != nullptr && cur >= 0) flush();
+      if (kHist && cur >= 0) flush();
     }
   }
   tc::fence_before_sync();
@@ -551,7 +598,7 @@ static bool make_rows128_map(CUtensorMap *m, const void *base, uint64_t rows) {
 
 static size_t indexer_tc_smem() {
   return 1024 + kIdxStages * kIdxTileBytes + 2 * kIdxBSlotBytes + 2 * kIdxWSlotBytes + kIdxStages * kIdxTile * 4 +
-         kIdxRows * (kIdxHistBins / 2) * 4 + sizeof(IdxSmem);
+         kIdxRows * (kIdxHistBins / 2) * 4 + (kIdxInlinePlanMax + 4) * 4 + sizeof(IdxSmem);
 }
 
 size_t indexer_hist_bytes(int total_q) { return al256((size_t)total_q * kIdxHistBins * 4); }
@@ -570,6 +617,8 @@ dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t 
     set_error("indexer: cuTensorMapEncodeTiled failed");
     return DSA_ERR_CUDA;
   }
+  const int inline_plan =
+      b->total_q == b->num_seqs && b->max_q_per_seq == 1 && b->num_seqs <= kIdxInlinePlanMax ? 1 : 0;
   if (app != nullptr && hist == nullptr && b->total_q <= kIdxFusedAppendMaxRows) {
     DSA_LAUNCH_PDL("indexer_plan_append_kernel", indexer_plan_append_kernel, dim3(1), dim3(1024), 0, stream, bv, pv,
                    *app, b->total_q, (uint32_t *)ws);
@@ -583,15 +632,22 @@ dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t 
       // the histograms are cleared here, a stream step ahead of the kernel that adds into them
       const int64_t words = (int64_t)b->total_q * kIdxHistBins;
       const int grid = (int)std::min<int64_t>(num_sms, std::max<int64_t>(1, words / (4 * 1024 * 4)));
-      DSA_LAUNCH_PDL("indexer_prep_kernel", indexer_prep_kernel, dim3(grid), dim3(1024), 0, stream, bv, pv, hist, words);
-    } else {
+      DSA_LAUNCH_PDL("indexer_prep_kernel", indexer_prep_kernel, dim3(grid), dim3(1024), 0, stream, bv, pv, hist, words,
+                     inline_plan ? 0 : 1);
+    } else if (!inline_plan) {
       DSA_LAUNCH_PDL("indexer_plan_kernel", indexer_plan_kernel, dim3(1), dim3(1024), 0, stream, bv, pv);
     }
   }
   const size_t smem = indexer_tc_smem();
-  cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  DSA_LAUNCH_PDL("indexer_tc_kernel", indexer_tc_kernel, dim3(num_sms), dim3(kIdxThreads), smem, stream, tm_k, tm_q,
-                 kscale, w, bv, pv, scores, ld, (uint32_t *)ws, hist);
+  if (hist != nullptr) {
+    cudaFuncSetAttribute(indexer_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    DSA_LAUNCH_PDL("indexer_tc_kernel", indexer_tc_kernel<true>, dim3(num_sms), dim3(kIdxThreads), smem, stream, tm_k,
+                   tm_q, kscale, w, bv, pv, scores, ld, (uint32_t *)ws, hist, inline_plan);
+  } else {
+    cudaFuncSetAttribute(indexer_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    DSA_LAUNCH_PDL("indexer_tc_kernel", indexer_tc_kernel<false>, dim3(num_sms), dim3(kIdxThreads), smem, stream, tm_k,
+                   tm_q, kscale, w, bv, pv, scores, ld, (uint32_t *)ws, hist, inline_plan);
+  }
   return DSA_OK;
 }
 

@@ -31,8 +31,8 @@ namespace dsa {
 
 constexpr int kSelThreads = 512;
 constexpr int kSelBins = 2048;
-constexpr int kSelPerThread = 16;                       // consecutive keys per thread per tile (4 x float4)
-constexpr int kSelTile = kSelThreads * kSelPerThread;   // 8192 keys
+constexpr int kSelPerThread = 8;                        // keys per thread per tile (2 x float4)
+constexpr int kSelTile = kSelThreads * kSelPerThread;   // 4096 keys
 
 struct SelArgs {
   const float *scores;
@@ -64,7 +64,8 @@ __device__ __forceinline__ uint32_t sel_cl_ld(const void *p, uint32_t rank) {
 }
 
 // Bin holding the need-th key counted from the top of hist[0..nb) (need >= 1, at most the total).  Returns
-// it in *s_bin and the count of keys in higher bins in *s_above.  Every thread of the block calls this.
+// it in *s_bin and the count of keys in higher bins in *s_above.  Every thread of the block calls this (a
+// block scan over per-thread runs of bins in descending order).
 __device__ void sel_find_bin(const uint32_t *hist, int nb, uint32_t need, uint32_t *tmp, int *s_bin,
                              uint32_t *s_above) {
   const int per = (nb + kSelThreads - 1) / kSelThreads;
@@ -87,30 +88,65 @@ __device__ void sel_find_bin(const uint32_t *hist, int nb, uint32_t need, uint32
   __syncthreads();
 }
 
-// keys of the slice tile starting at `base` (kSelPerThread consecutive per thread); positions past m get
-// valid = false
+// A tile of kSelTile keys is 16 warp segments of 32 x kSelPerThread in position order; in its segment a lane
+// holds the keys at 128 v + 4 lane + j (v < kSelPerThread / 4, j = 0..3), read as coalesced float4 loads.
+// key[4 v + j]; valid bit 4 v + j is clear for positions at or past m.
+__device__ __forceinline__ int sel_elem(int base, int v, int j) {
+  return base + (int)(threadIdx.x >> 5) * (32 * kSelPerThread) + 128 * v + 4 * (int)(threadIdx.x & 31) + j;
+}
 __device__ __forceinline__ void sel_load_tile(const float *src, int m, int base, uint32_t (&key)[kSelPerThread],
                                               uint32_t &valid) {
-  const int i0 = base + threadIdx.x * kSelPerThread;
   valid = 0u;
-  if (i0 + kSelPerThread <= m) {
 #pragma unroll
-    for (int v = 0; v < kSelPerThread / 4; ++v) {
-      const float4 f = __ldg(reinterpret_cast<const float4 *>(src + i0) + v);
+  for (int v = 0; v < kSelPerThread / 4; ++v) {
+    const int i0 = sel_elem(base, v, 0);
+    if (i0 + 4 <= m) {
+      const float4 f = __ldg(reinterpret_cast<const float4 *>(src + i0));
       key[4 * v] = ordered_key(f.x);
       key[4 * v + 1] = ordered_key(f.y);
       key[4 * v + 2] = ordered_key(f.z);
       key[4 * v + 3] = ordered_key(f.w);
-    }
-    valid = 0xFFFFu;
-  } else {
+      valid |= 0xFu << (4 * v);
+    } else {
 #pragma unroll
-    for (int e = 0; e < kSelPerThread; ++e) {
-      const bool in = i0 + e < m;
-      key[e] = in ? ordered_key(__ldg(src + i0 + e)) : 0u;
-      valid |= (in ? 1u : 0u) << e;
+      for (int j = 0; j < 4; ++j) {
+        const bool in = i0 + j < m;
+        key[4 * v + j] = in ? ordered_key(__ldg(src + i0 + j)) : 0u;
+        valid |= (in ? 1u : 0u) << (4 * v + j);
+      }
     }
   }
+}
+
+// Ordered positions of flagged items in a tile laid out as sel_elem describes: flags bit 4 v + j.  Returns, for
+// each v, the count of flagged items before (v, lane, 0) in the tile (pre[v]), and the tile's total; `wsum`
+// holds 32 words of shared scratch.  One __syncthreads inside, one more before wsum is reused.
+__device__ __forceinline__ uint32_t sel_tile_prefix(uint32_t flags, uint32_t (&pre)[kSelPerThread / 4], uint32_t *wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t run = 0u;
+#pragma unroll
+  for (int v = 0; v < kSelPerThread / 4; ++v) {
+    const uint32_t cnt = __popc((flags >> (4 * v)) & 0xFu);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    pre[v] = run + incl - cnt;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) wsum[warp] = run;
+  __syncthreads();
+  uint32_t before = 0u, total = 0u;
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    const uint32_t x = wsum[w];
+    before += w < warp ? x : 0u;
+    total += x;
+  }
+#pragma unroll
+  for (int v = 0; v < kSelPerThread / 4; ++v) pre[v] += before;
+  return total;
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArgs a) {
@@ -130,7 +166,7 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
   const int row = blockIdx.x / (int)C;
   const int tid = threadIdx.x;
   int b;
-  const int n = pos_of_row(a.bv, row, &b) + 1;
+  const int n = pos_of_row_warp(a.bv, row, &b) + 1;
   int32_t *out = a.idx + (int64_t)row * a.k;
   // (every branch on n is taken by the whole cluster)
   if (n <= a.k) {
@@ -145,6 +181,9 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
 
   uint32_t P = 0u, M = 0u, above = 0u, need = (uint32_t)a.k, bin_cnt = (uint32_t)n, local_eq = 0u;
   int shift = 32;
+  // the slice's first tile is read while the threshold digit is found
+  uint32_t key0[kSelPerThread], valid0;
+  sel_load_tile(src, m, 0, key0, valid0);
   if (a.hist != nullptr) {
     const uint32_t *hr = a.hist + (int64_t)row * kSelBins;
     for (int i = tid; i < kSelBins; i += kSelThreads) gh[i] = __ldcg(hr + i);
@@ -211,10 +250,14 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
   // ------------------------------------------------------------------ storing pass: ordered survivors
   uint32_t stored = 0u;                // survivors written so far (block-uniform)
   if (tid == 0) s_flag = 0u;
+  uint32_t kn[kSelPerThread], vn = 0u;  // the next tile, loaded while this one is compacted
 #pragma unroll 1
   for (int base = 0; base < m; base += kSelTile) {
     uint32_t key[kSelPerThread], valid;
-    sel_load_tile(src, m, base, key, valid);
+#pragma unroll
+    for (int e = 0; e < kSelPerThread; ++e) key[e] = base == 0 ? key0[e] : kn[e];
+    valid = base == 0 ? valid0 : vn;
+    if (base + kSelTile < m) sel_load_tile(src, m, base + kSelTile, kn, vn);
     uint32_t keep = 0u, eq = 0u;
 #pragma unroll
     for (int e = 0; e < kSelPerThread; ++e) {
@@ -224,36 +267,43 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
         else if (km == P) eq |= 1u << e;
       }
     }
+    uint32_t pre[kSelPerThread / 4];
     if (full) {
       // equal keys taken in position order: the first `need` of the row
-      uint32_t eq_tot;
-      const uint32_t eq_ex = block_exclusive_scan(__popc(eq), tmp, &eq_tot);
-      uint32_t rank_eq = eq_before + eq_ex;
+      const uint32_t eq_tot = sel_tile_prefix(eq, pre, tmp);
 #pragma unroll
-      for (int e = 0; e < kSelPerThread; ++e)
-        if ((eq >> e) & 1u) {
-          if (rank_eq < need) keep |= 1u << e;
-          ++rank_eq;
-        }
+      for (int v = 0; v < kSelPerThread / 4; ++v) {
+        uint32_t rank_eq = eq_before + pre[v];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if ((eq >> (4 * v + j)) & 1u) {
+            if (rank_eq < need) keep |= 1u << (4 * v + j);
+            ++rank_eq;
+          }
+      }
       eq_before += eq_tot;
+      __syncthreads();
     } else {
       keep |= eq;
     }
-    uint32_t tot;
-    uint32_t off = stored + block_exclusive_scan(__popc(keep), tmp, &tot);
-    const int i0 = base + tid * kSelPerThread;
+    const uint32_t tot = sel_tile_prefix(keep, pre, tmp);
 #pragma unroll
-    for (int e = 0; e < kSelPerThread; ++e)
-      if ((keep >> e) & 1u) {
-        if (off < cap) {
-          skey[off] = key[e];
-          spos[off] = lo + i0 + e;
-        } else {
-          s_flag = 1u;
+    for (int v = 0; v < kSelPerThread / 4; ++v) {
+      uint32_t off = stored + pre[v];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if ((keep >> (4 * v + j)) & 1u) {
+          if (off < cap) {
+            skey[off] = key[4 * v + j];
+            spos[off] = lo + sel_elem(base, v, j);
+          } else {
+            s_flag = 1u;
+          }
+          ++off;
         }
-        ++off;
-      }
+    }
     stored += tot;
+    __syncthreads();
   }
   if (stored > cap) stored = cap;
   __syncthreads();
@@ -264,23 +314,32 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
     if (tid == 0) info[0] = stored;
     tc::cluster_sync();                          // every slice's survivors are in place
     if (r == 0) {
-      uint32_t total = stored;
-      for (uint32_t c = 1; c < C; ++c) {
-        const uint32_t cnt = sel_cl_ld(info, c);
-        const uint32_t take = total + cnt <= cap ? cnt : cap - total;
-        if (take < cnt && tid == 0) set_status(a.status, kStatusBadIndex);
-        const uint32_t kaddr = tc::map_to_rank(tc::smem_u32(skey), c);
-        const uint32_t paddr = tc::map_to_rank(tc::smem_u32(spos), c);
-        for (uint32_t i = tid; i < take; i += kSelThreads) {
-          uint32_t kv, pv;
-          asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(kv) : "r"(kaddr + 4 * i) : "memory");
-          asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(pv) : "r"(paddr + 4 * i) : "memory");
-          skey[total + i] = kv;
-          spos[total + i] = (int32_t)pv;
+      // the other slices' counts, their offsets after this slice's survivors, then every piece in one round
+      uint32_t *offs = lh[0];                    // (free here) offs[c] = first slot of slice c, offs[C] = end
+      if (tid == 0) {
+        uint32_t total = stored;
+        offs[0] = 0u;
+        for (uint32_t c = 1; c < C; ++c) {
+          const uint32_t cnt = sel_cl_ld(info, c);
+          offs[c] = total;
+          total += cnt;
         }
-        total += take;
+        offs[C] = total;
+        if (total > cap) set_status(a.status, kStatusBadIndex);
       }
-      stored = total;
+      __syncthreads();
+      const uint32_t end = min(offs[C], cap);
+      for (uint32_t i = stored + tid; i < end; i += kSelThreads) {
+        uint32_t c = 1;
+        while (c + 1 < C && offs[c + 1] <= i) ++c;
+        const uint32_t j = i - offs[c];
+        uint32_t kv, pv;
+        asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(kv) : "r"(tc::map_to_rank(tc::smem_u32(skey + j), c)) : "memory");
+        asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(pv) : "r"(tc::map_to_rank(tc::smem_u32(spos + j), c)) : "memory");
+        skey[i] = kv;
+        spos[i] = (int32_t)pv;
+      }
+      stored = end;
     }
     tc::cluster_sync();                          // rank 0 has read every other slice
     if (r != 0) return;
@@ -310,38 +369,58 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
     __syncthreads();
   }
   // P is now the k-th key: emit every survivor above it and the first `need` equal to it, in order
+  // survivors in tiles of 16 warp segments of 256, lane l of a segment holding entries 32 e + l (e = 0..7)
   uint32_t written = 0u, eq_seen = 0u;
+  const int lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
 #pragma unroll 1
-  for (uint32_t base = 0; base < stored; base += kSelTile) {
-    const uint32_t i0 = base + tid * kSelPerThread;
-    uint32_t gt = 0u, eq = 0u;
+  for (uint32_t base = 0; base < stored; base += kSelThreads * 8) {
+    const uint32_t i0 = base + (uint32_t)warp * 256u + (uint32_t)lane;
+    uint32_t gtb[8], eqb[8], seg_eq = 0u;
 #pragma unroll
-    for (int e = 0; e < kSelPerThread; ++e) {
-      if (i0 + e < stored) {
-        const uint32_t kv = skey[i0 + e];
-        if (kv > P) gt |= 1u << e;
-        else if (kv == P) eq |= 1u << e;
-      }
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t i = i0 + 32u * e;
+      const uint32_t kv = i < stored ? skey[i] : 0u;
+      gtb[e] = __ballot_sync(0xffffffffu, i < stored && kv > P);
+      eqb[e] = __ballot_sync(0xffffffffu, i < stored && kv == P);
+      seg_eq += __popc(eqb[e]);
     }
-    uint32_t eq_tot;
-    uint32_t rank_eq = eq_seen + block_exclusive_scan(__popc(eq), tmp, &eq_tot);
-    uint32_t sel = gt;
+    // equal keys in position order: the first `need` of all survivors are taken
+    if (lane == 0) tmp[warp] = seg_eq;
+    __syncthreads();
+    uint32_t eq_before_seg = eq_seen, eq_tile = 0u;
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+      eq_before_seg += w < warp ? tmp[w] : 0u;
+      eq_tile += tmp[w];
+    }
+    uint32_t selb[8], seg_sel = 0u, run_eq = eq_before_seg;
 #pragma unroll
-    for (int e = 0; e < kSelPerThread; ++e)
-      if ((eq >> e) & 1u) {
-        if (rank_eq < need) sel |= 1u << e;
-        ++rank_eq;
-      }
-    eq_seen += eq_tot;
-    uint32_t tot;
-    uint32_t off = written + block_exclusive_scan(__popc(sel), tmp, &tot);
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t my_rank = run_eq + __popc(eqb[e] & lt_mask);
+      const bool take = ((eqb[e] >> lane) & 1u) && my_rank < need;
+      selb[e] = gtb[e] | __ballot_sync(0xffffffffu, take);
+      run_eq += __popc(eqb[e]);
+      seg_sel += __popc(selb[e]);
+    }
+    eq_seen += eq_tile;
+    __syncthreads();
+    if (lane == 0) tmp[warp] = seg_sel;
+    __syncthreads();
+    uint32_t off = written, sel_tile = 0u;
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+      off += w < warp ? tmp[w] : 0u;
+      sel_tile += tmp[w];
+    }
 #pragma unroll
-    for (int e = 0; e < kSelPerThread; ++e)
-      if ((sel >> e) & 1u) {
-        if (off < (uint32_t)a.k) out[off] = spos[i0 + e];
-        ++off;
+    for (int e = 0; e < 8; ++e) {
+      if ((selb[e] >> lane) & 1u) {
+        const uint32_t o = off + __popc(selb[e] & lt_mask);
+        if (o < (uint32_t)a.k) out[o] = spos[i0 + 32u * e];
       }
-    written += tot;
+      off += __popc(selb[e]);
+    }
+    written += sel_tile;
+    __syncthreads();
   }
   // a consistent histogram always yields exactly k; pad defensively otherwise
   for (uint32_t j = written + tid; j < (uint32_t)a.k; j += kSelThreads) out[j] = -1;
@@ -356,12 +435,45 @@ static int select_cap(int k) {
   return std::min(cap, 24576);
 }
 
-// CTAs per row: enough to spread few rows over the SMs (two per SM), no slice under 2048 keys, at most 16.
+// CTAs per row: enough to spread few rows over the SMs (half of them busy at most, so rows of a batch with
+// many rows run one CTA each), no slice under 4096 keys, at most 16.  Measured on the decode batch (32 rows of
+// 4K-32K keys): 4 CTAs per row select in about half the time of one.
 static int select_cluster(int T, int max_seq_len, int num_sms) {
   int C = 1;
-  while (C < 16 && (int64_t)T * C * 2 * 2 <= (int64_t)num_sms * 2 && (int64_t)max_seq_len >= (int64_t)C * 2 * 4096)
-    C *= 2;
+  while (C < 16 && (int64_t)T * C * 2 <= (int64_t)num_sms && (int64_t)max_seq_len >= (int64_t)C * 2 * 4096) C *= 2;
   return C;
+}
+
+// Largest cluster (16, 8, 4, 2 or 1 CTAs) the device can place at the largest shared-memory footprint; found
+// once per device (threads racing on the first call compute the same value).
+static int select_max_cluster(int num_sms) {
+  static std::atomic<int> cached[kMaxDevices];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = -1;
+  int c = dev >= 0 ? cached[dev].load(std::memory_order_relaxed) : 0;
+  if (c > 0) return c;
+  const size_t smem = select_smem_bytes(select_cap(16384));
+  cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  for (c = 16; c > 1; c /= 2) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)c);
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = (unsigned)c;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, select_stream_kernel, &cfg) == cudaSuccess && n >= 1) break;
+    cudaGetLastError();
+  }
+  (void)num_sms;
+  if (dev >= 0) cached[dev].store(c, std::memory_order_relaxed);
+  return c;
 }
 
 dsa_status_t select_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx,
@@ -376,40 +488,29 @@ dsa_status_t select_launch(const float *scores, int64_t ld, const dsa_batch_t *b
   a.cap = select_cap(k);
   a.status = status;
   const size_t smem = select_smem_bytes(a.cap);
+  const int C = std::min(select_cluster(b->total_q, b->max_seq_len, num_sms), select_max_cluster(num_sms));
   cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  int C = select_cluster(b->total_q, b->max_seq_len, num_sms);
-  for (;; C /= 2) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(b->total_q * C));
-    cfg.blockDim = dim3(kSelThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = (unsigned)C;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    if (C > 1) {
-      // a cluster that cannot be placed is not launched: fall back to a smaller one
-      int nclusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&nclusters, select_stream_kernel, &cfg) != cudaSuccess || nclusters < 1) {
-        cudaGetLastError();
-        continue;
-      }
-    }
-    const cudaError_t le = cudaLaunchKernelEx(&cfg, select_stream_kernel, a);
-    if (le != cudaSuccess) {
-      set_error("select_stream_kernel: %s", cudaGetErrorString(le));
-      return DSA_ERR_CUDA;
-    }
-    DSA_LAUNCH_CHECK("select_stream_kernel");
-    return DSA_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(b->total_q * C));
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)C;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, select_stream_kernel, a);
+  if (le != cudaSuccess) {
+    set_error("select_stream_kernel: %s", cudaGetErrorString(le));
+    return DSA_ERR_CUDA;
   }
+  DSA_LAUNCH_CHECK("select_stream_kernel");
+  return DSA_OK;
 }
 
 }  // namespace dsa

@@ -181,8 +181,21 @@ class DeviceBatch:
         B.dsa_expand_blocks(self.blk_idx, kb, self.batch, self.idx_blk, stream)
         return self.idx_blk
 
-    def run(self, stream=None, fused=False):
-        """One pass of the path: scores, selection, attention (fused=True: scores and selection in one call)."""
+    # Batches where the fused scores + selection call is the faster form of the first two steps (measured on
+    # one B200): many rows longer than one CTA's shared-memory slice of the plain top-k (the mixed batch's
+    # 57K-65K-candidate chunk rows: 22.3 ms against 26.4 ms).  For decode batches, prefill prompts of up to a few
+    # ten thousand tokens and a single million-token row the two separate calls are faster.
+    FUSED_MIN_ROWS = 1024
+    FUSED_MIN_LEN = 49153
+
+    def prefers_fused(self):
+        return self.wl.total_q >= self.FUSED_MIN_ROWS and self.wl.max_seq_len >= self.FUSED_MIN_LEN
+
+    def run(self, stream=None, fused=None):
+        """One pass of the path: scores, selection, attention.  fused=True takes scores and selection in one
+        call (dsa_indexer_topk), False the two calls; None picks by prefers_fused()."""
+        if fused is None:
+            fused = self.prefers_fused()
         if fused:
             self.indexer_topk(stream)
         else:

@@ -176,7 +176,12 @@ def job_tokens_per_s(tokens_per_rank_step, world, ms_per_step):
     return world * tokens_per_rank_step / (ms_per_step / 1e3)
 
 
-def _time_steps(replicas, stream, steps, warmup, world, dev, sampler=None):
+def _fused_for(db, selection):
+    """Whether a step takes the fused scores + selection call: by the pipeline's shape rule ("auto"), or forced."""
+    return db.prefers_fused() if selection == "auto" else selection == "fused"
+
+
+def _time_steps(replicas, stream, steps, warmup, world, dev, sampler=None, selection="auto"):
     """W untimed warm-up steps, then K steps bracketed by a barrier and a device synchronise, timed with
     CUDA events on the launching stream (per-stage events inside the timed region).  Returns the slowest
     rank's total milliseconds, the per-stage averages, the library launches and the clock summary."""
@@ -187,7 +192,7 @@ def _time_steps(replicas, stream, steps, warmup, world, dev, sampler=None):
     def step(db, ev=None):
         # the first two steps as the pipeline runs them: one fused call for batches where that is faster
         # (its time is then reported under "indexer", "topk" holding the empty interval), else two calls
-        fused = db.prefers_fused()
+        fused = _fused_for(db, selection)
         if ev is not None:
             ev[0].record(stream)
         if fused:
@@ -310,9 +315,9 @@ def run_extra_workload(name, args, dev, stream, sampler):
     work = work_of(wl)
     db = DeviceBatch(wl, device=dev)
     # enough steps for a timed region of about 0.2 s (clock samples under load), at least --extra-steps
-    probe_ms, _, _, _ = _time_steps([db], stream, 1, args.warmup, 1, dev, None)
+    probe_ms, _, _, _ = _time_steps([db], stream, 1, args.warmup, 1, dev, None, args.selection)
     steps = int(min(2000, max(args.extra_steps, math.ceil(200.0 / max(probe_ms, 1e-3)))))
-    total_ms, stage_avg, launches, clocks = _time_steps([db], stream, steps, 1, 1, dev, sampler)
+    total_ms, stage_avg, launches, clocks = _time_steps([db], stream, steps, 1, 1, dev, sampler, args.selection)
     ms_per_step = total_ms / steps
     peaks, peak_src = load_peaks()
     decode = bool(np.all(wl.q_lens == 1))
@@ -324,8 +329,8 @@ def run_extra_workload(name, args, dev, stream, sampler):
            "stage_rooflines": {s: roofline_entry(s, stage_avg[s], work, peaks, peak_src, name, decode)
                                for s in ("indexer", "attention")},
            "step_roofline": step_roofline(work, peaks, ms_per_step), "gpu_launches": launches, "clocks": clocks,
-           "selection": "dsa_indexer_topk (fused; stages_ms.indexer holds scores + selection)" if db.prefers_fused()
-           else "dsa_indexer_scores + dsa_topk",
+           "selection": "dsa_indexer_topk (fused; stages_ms.indexer holds scores + selection)"
+           if _fused_for(db, args.selection) else "dsa_indexer_scores + dsa_topk",
            "config": workload_config(wl, replicas=1, l2="inputs larger than L2 (one device replica)")}
     # both forms of the first two steps, for the choice between them
     def t2(fn, n):
@@ -367,7 +372,8 @@ def run_ours(args, rank, world, local_rank):
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    total_ms, stage_avg, launches, clocks = _time_steps(replicas, stream, args.steps, args.warmup, world, dev, sampler)
+    total_ms, stage_avg, launches, clocks = _time_steps(replicas, stream, args.steps, args.warmup, world, dev, sampler,
+                                                        args.selection)
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(work["tokens"], world, ms_per_step)
 
@@ -394,6 +400,8 @@ def run_ours(args, rank, world, local_rank):
         "config": workload_config(wl, replicas=args.replicas),
         "stages_ms": stage_avg, "roofline": roof, "e2e": e2e, "gpu_launches": int(launches),
         "clocks": clocks, "impl": "ours",
+        "selection": "dsa_indexer_topk (fused; stages_ms.indexer holds scores + selection)"
+        if _fused_for(replicas[0], args.selection) else "dsa_indexer_scores + dsa_topk",
     }
     if wl.kind == "mla":
         res["step_roofline"] = step_roofline(work, peaks, ms_per_step)
@@ -437,8 +445,8 @@ def workload_config(wl, replicas=1, l2=None):
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum per launch) of the dominant kernel from one
 # ncu capture (profiles/), valid only while the kernel's sources are the ones that were captured.
 MEASURED_TRAFFIC = {
-    ("attention", "decode_batch"): {"bytes": 84244992 + 4310784,
-                                    "sources": ("attn_mla_tc.cu", "tc.cuh", "common.cuh"), "sha256_16": "ee6a0cc8aa2fe8fa"},
+    ("attention", "decode_batch"): {"bytes": 84242432 + 3617792,
+                                    "sources": ("attn_mla_tc.cu", "tc.cuh", "common.cuh"), "sha256_16": "f23a2892ed21082a"},
 }
 
 
@@ -493,7 +501,7 @@ def run_e2e(args, wl, db, stream, dev, world):
     def step():
         for h, d in per_step.values():
             d.copy_(h, non_blocking=True)
-        db.run(stream)
+        db.run(stream, fused=_fused_for(db, args.selection))
         out_h.copy_(db.out, non_blocking=True)
         lse_h.copy_(db.lse, non_blocking=True)
 
@@ -601,7 +609,7 @@ def _e2e_overlapped_local(args, wl, replicas, dev):
             s_cmp.wait_event(in_done[j])
             if i >= 2:
                 s_cmp.wait_event(out_done[j])
-            db.run(s_cmp)
+            db.run(s_cmp, fused=_fused_for(db, args.selection))
             cmp_done[j].record(s_cmp)
             s_out.wait_event(cmp_done[j])
             with torch.cuda.stream(s_out):
@@ -706,6 +714,8 @@ def main():
                     help="comma-separated MLA workloads timed after the decode batch at N=1 ('' for none)")
     ap.add_argument("--extra-steps", type=int, default=10)
     ap.add_argument("--no-widened", action="store_true", help="skip the timing of the decode step's variants")
+    ap.add_argument("--selection", default="auto", choices=["auto", "fused", "separate"],
+                    help="scores + selection as one fused call, two calls, or by the pipeline's shape rule")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -181,6 +181,15 @@ def _fused_for(db, selection):
     return db.prefers_fused() if selection == "auto" else selection == "fused"
 
 
+def _run_step(db, stream, args):
+    """One pass of the path through the pipeline (its shape rule picks the selection form unless forced)."""
+    selection = getattr(args, "selection", "auto")
+    if selection == "auto":
+        db.run(stream)
+    else:
+        db.run(stream, fused=selection == "fused")
+
+
 def _time_steps(replicas, stream, steps, warmup, world, dev, sampler=None, selection="auto"):
     """W untimed warm-up steps, then K steps bracketed by a barrier and a device synchronise, timed with
     CUDA events on the launching stream (per-stage events inside the timed region).  Returns the slowest
@@ -501,7 +510,7 @@ def run_e2e(args, wl, db, stream, dev, world):
     def step():
         for h, d in per_step.values():
             d.copy_(h, non_blocking=True)
-        db.run(stream, fused=_fused_for(db, args.selection))
+        _run_step(db, stream, args)
         out_h.copy_(db.out, non_blocking=True)
         lse_h.copy_(db.lse, non_blocking=True)
 
@@ -609,7 +618,7 @@ def _e2e_overlapped_local(args, wl, replicas, dev):
             s_cmp.wait_event(in_done[j])
             if i >= 2:
                 s_cmp.wait_event(out_done[j])
-            db.run(s_cmp, fused=_fused_for(db, args.selection))
+            _run_step(db, s_cmp, args)
             cmp_done[j].record(s_cmp)
             s_out.wait_event(cmp_done[j])
             with torch.cuda.stream(s_out):

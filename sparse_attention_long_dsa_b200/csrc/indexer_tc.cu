@@ -14,12 +14,13 @@
 // per-thread reduction with no shuffles.  A 128-key tile is two 64-token pages fetched by TMA through
 // the block table (128-byte swizzle, the layout the MMA descriptor reads).
 //
-// Warp roles (288 threads, persistent, one CTA per SM):
+// Warp roles (416 threads, persistent, one CTA per SM):
 //   warps 0,6-8  TMA producers: key tiles into an 8-stage ring (round-robin over the four warps); warp 0
 //                also loads the query rows + weights of each row group
 //   warp 1       allocates 512 TMEM columns; lane 0 issues 4 MMAs (K = 32 each) per tile into one of two
 //                256-column accumulators and commits them to the ring / accumulator barriers
-//   warps 2..5   epilogue: tcgen05.ld 64 heads per row, ReLU, weight, sum, key scale, causal store
+//   warps 2..5,  epilogue, two groups taking alternate tiles (one accumulator each): tcgen05.ld 64 heads per
+//   9..12        row, ReLU, weight, sum, key scale, causal store
 // Work units are (row group, key tile) pairs in group order, split evenly over the CTAs; a one-CTA
 // plan kernel enumerates the groups and their tile counts in the workspace first.
 #include <algorithm>
@@ -32,7 +33,8 @@ namespace dsa {
 constexpr int kIdxTile = 128;
 constexpr int kIdxRows = 4;
 constexpr int kIdxStages = 8;
-constexpr int kIdxThreads = 288;                  // warps 0, 6-8 TMA, 1 MMA, 2-5 epilogue
+constexpr int kIdxThreads = 416;                  // warps 0, 6-8 TMA, 1 MMA, 2-5 and 9-12 epilogue
+constexpr int kIdxEpiThreads = 256;               // two epilogue groups of four warps
 constexpr int kIdxHi = 64, kIdxDi = 128;
 constexpr uint32_t kIdxTileBytes = kIdxTile * kIdxDi;         // 16 KB
 constexpr uint32_t kIdxPageBytes = 64 * kIdxDi;               // 8 KB
@@ -227,11 +229,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   if (threadIdx.x == 0) {
     for (int i = 0; i < kIdxStages; ++i) {
       tc::mbar_init(tc::smem_u32(&S->full[i]), 1);
-      tc::mbar_init(tc::smem_u32(&S->empty[i]), 1 + 4);      // MMA commit + 4 epilogue warps (key scales)
+      tc::mbar_init(tc::smem_u32(&S->empty[i]), 1 + 4);      // MMA commit + the tile's 4 epilogue warps (key scales)
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(tc::smem_u32(&S->bfull[i]), 1);
-      tc::mbar_init(tc::smem_u32(&S->bempty[i]), 1 + 4);
+      tc::mbar_init(tc::smem_u32(&S->bempty[i]), 1 + 8);     // MMA commit + both epilogue groups
       tc::mbar_init(tc::smem_u32(&S->tfull[i]), 1);
       tc::mbar_init(tc::smem_u32(&S->tempty[i]), 4);
     }
@@ -283,7 +285,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const int u1 = (int)(((int64_t)(blockIdx.x + 1) * U) / gridDim.x);
 
   if (u0 < u1) {
-    if (warp == 0 || warp >= 6) {
+    if (warp == 0 || (warp >= 6 && warp <= 8)) {
       // ------------------------------------------------------------------ TMA producers (4 warps)
       // Key tiles are spread over four producer warps (a tile's stage is fixed by its position, so each
       // warp owns two of the eight stages): the copy engine takes several warps' copies at once.  Each
@@ -437,31 +439,36 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       tc::mma_commit_w(tc::smem_u32(&S->drain));
       volatile int no_abort = 0;
       tc::mbar_wait_w(tc::smem_u32(&S->drain), 0, &no_abort, status);
-    } else if (warp >= 2 && warp < 6) {
-      // ------------------------------------------------------------------ epilogue
+    } else if ((warp >= 2 && warp < 6) || warp >= 9) {
+      // ------------------------------------------------------------------ epilogue (two groups of 4 warps)
+      // Group eg (warps 2-5: 0, warps 9-12: 1) takes the tiles of even / odd position in the CTA's range, which
+      // are exactly the tiles the MMA accumulates into TMEM accumulator eg: the weighted ReLU sums of two tiles
+      // run at once.  Both groups walk every unit to keep the row-group bookkeeping: each waits for every row
+      // group's query rows and releases them once it is past the group's last tile.
       const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
       const int key_local = quad * 32 + lane;
-      const int et = threadIdx.x - 64;           // 0..127 over the four epilogue warps
-      // With histograms on, the four warps meet at named barrier 1 around every flush, so the loop never
+      const int eg = warp >= 9 ? 1 : 0;
+      const int et = (warp >= 9 ? warp - 5 : warp - 2) * 32 + lane;   // 0..255 over the two groups
+      // With histograms on, the eight warps meet at named barrier 1 around every flush, so the loop never
       // leaves early then: after a timeout the waits return at once and the remaining units pass through
       // without touching TMEM or global memory.
       if constexpr (kHist) {
-        for (int j = et; j < kIdxRows * (kIdxHistBins / 2); j += 128) sHist[j] = 0u;
-        tc::named_bar_sync(1, 128);
+        for (int j = et; j < kIdxRows * (kIdxHistBins / 2); j += kIdxEpiThreads) sHist[j] = 0u;
+        tc::named_bar_sync(1, kIdxEpiThreads);
       }
       int gi, t;
       unit_locate(tp, G, u0, &gi, &t);
-      int acc = 0, nb_groups = 0, bslot = 0, cur = -1, span = 0;
-      uint32_t acc_phase = 0;
+      int nb_groups = 0, bslot = 0, cur = -1, span = 0;
+      uint32_t acc_phase = 0;                    // phase of accumulator eg
       int b = 0, row0 = 0, nr = 0, pos0 = 0;
       bool ok = true;
       // adds this CTA's counts of the current group's rows to their global histograms and clears them
       auto flush = [&]() {
-        tc::named_bar_sync(1, 128);
+        tc::named_bar_sync(1, kIdxEpiThreads);
         for (int q = 0; q < nr; ++q) {
           uint32_t *hg = hist + (int64_t)(row0 + q) * kIdxHistBins;
           uint32_t *hs = sHist + q * (kIdxHistBins / 2);
-          for (int j = et; j < kIdxHistBins / 2; j += 128) {
+          for (int j = et; j < kIdxHistBins / 2; j += kIdxEpiThreads) {
             const uint32_t v = hs[j];
             if (v != 0u) {
               if (ok) {
@@ -472,12 +479,21 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             }
           }
         }
-        tc::named_bar_sync(1, 128);
+        tc::named_bar_sync(1, kIdxEpiThreads);
         span = 0;
       };
+      // this group is done with the current row group's query rows and weights
+      auto release_group = [&]() {
+        __syncwarp();
+        if (lane == 0 && ok) tc::mbar_arrive(tc::smem_u32(&S->bempty[bslot]));
+      };
       for (int u = u0; u < u1; ++u) {
+        const bool mine = ((u - u0) & 1) == eg;
         if (gi != cur) {
-          if (kHist && cur >= 0) flush();
+          if (cur >= 0) {
+            if (kHist) flush();
+            release_group();
+          }
           bslot = nb_groups & 1;
           ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->bfull[bslot]), (uint32_t)(nb_groups >> 1) & 1u, abort,
                                                      status)) && ok;
@@ -492,69 +508,72 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         } else if (kHist && span == kIdxHistFlushTiles) {
           flush();
         }
-        const int s = t * kIdxTile + key_local;
-        // the TMEM loads below are warp-collective: the warp takes them together or not at all
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->tfull[acc]), acc_phase, abort, status)) && ok;
-        if (!kHist && !ok) break;
-        if (ok) {
-          tc::fence_after_sync();
-          // the tile's key scales arrived with it; the stage's fill has completed (the MMA consumed it), the
-          // wait below returns at once and orders the bulk copy before these reads
-          const int stage = (u - u0) % kIdxStages;
-          tc::mbar_wait(tc::smem_u32(&S->full[stage]), (uint32_t)((u - u0) / kIdxStages) & 1u, abort, status);
-          const float ks = sKS[stage * kIdxTile + key_local];
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->empty[stage]));
-          const float *wq = sW + bslot * (kIdxWSlotBytes / 4);
-          const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + acc * 256;
-          uint32_t dig[kIdxRows];             // leading digits of this thread's scores (bit 31: none)
+        if (mine) {
+          const int s = t * kIdxTile + key_local;
+          // the TMEM loads below are warp-collective: the warp takes them together or not at all
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&S->tfull[eg]), acc_phase, abort, status)) && ok;
+          if (!kHist && !ok) break;
+          if (ok) {
+            tc::fence_after_sync();
+            // the tile's key scales arrived with it; the stage's fill has completed (the MMA consumed it), the
+            // wait below returns at once and orders the bulk copy before these reads
+            const int stage = (u - u0) % kIdxStages;
+            tc::mbar_wait(tc::smem_u32(&S->full[stage]), (uint32_t)((u - u0) / kIdxStages) & 1u, abort, status);
+            const float ks = sKS[stage * kIdxTile + key_local];
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->empty[stage]));
+            const float *wq = sW + bslot * (kIdxWSlotBytes / 4);
+            const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + eg * 256;
+            uint32_t dig[kIdxRows];             // leading digits of this thread's scores (bit 31: none)
 #pragma unroll
-          for (int q = 0; q < kIdxRows; ++q) {
-            dig[q] = 0x80000000u;
-            if (q >= nr) continue;
-            float v0[32], v1[32];
-            tc::tmem_ld32(tbase + q * 64, v0);
-            tc::tmem_ld32(tbase + q * 64 + 32, v1);
-            tc::tmem_wait_ld();
-            const float *wr = wq + q * kIdxHi;
-            float a0 = 0.f, a1 = 0.f;
+            for (int q = 0; q < kIdxRows; ++q) {
+              dig[q] = 0x80000000u;
+              if (q >= nr) continue;
+              float v0[32], v1[32];
+              tc::tmem_ld32(tbase + q * 64, v0);
+              tc::tmem_ld32(tbase + q * 64 + 32, v1);
+              tc::tmem_wait_ld();
+              const float *wr = wq + q * kIdxHi;
+              float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int h = 0; h < 32; h += 2) {
-              a0 = fmaf(wr[h], fmaxf(v0[h], 0.f), a0);
-              a1 = fmaf(wr[h + 1], fmaxf(v0[h + 1], 0.f), a1);
-            }
-#pragma unroll
-            for (int h = 0; h < 32; h += 2) {
-              a0 = fmaf(wr[32 + h], fmaxf(v1[h], 0.f), a0);
-              a1 = fmaf(wr[33 + h], fmaxf(v1[h + 1], 0.f), a1);
-            }
-            if (s <= pos0 + q) {
-              const float sc = (a0 + a1) * ks;
-              scores[(int64_t)(row0 + q) * ld + s] = sc;
-              if constexpr (kHist) dig[q] = ordered_key(sc) >> 21;
-            }
-          }
-          tc::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->tempty[acc]));
-          const bool last_of_group = (t + 1 == tp[gi + 1] - tp[gi]) || (u + 1 == u1);
-          if (last_of_group && lane == 0) tc::mbar_arrive(tc::smem_u32(&S->bempty[bslot]));
-          if constexpr (kHist) {
-            // counted after the accumulator and the query rows are handed back (an arrive orders every earlier
-            // memory operation of the warp before it, so adds in front of it would hold the tensor core up)
-#pragma unroll
-            for (int q = 0; q < kIdxRows; ++q)
-              if (dig[q] != 0x80000000u) {
-                const uint32_t addr = tc::smem_u32(&sHist[q * (kIdxHistBins / 2) + (dig[q] >> 1)]);
-                asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"((dig[q] & 1u) ? 0x10000u : 1u) : "memory");
+              for (int h = 0; h < 32; h += 2) {
+                a0 = fmaf(wr[h], fmaxf(v0[h], 0.f), a0);
+                a1 = fmaf(wr[h + 1], fmaxf(v0[h + 1], 0.f), a1);
               }
+#pragma unroll
+              for (int h = 0; h < 32; h += 2) {
+                a0 = fmaf(wr[32 + h], fmaxf(v1[h], 0.f), a0);
+                a1 = fmaf(wr[33 + h], fmaxf(v1[h + 1], 0.f), a1);
+              }
+              if (s <= pos0 + q) {
+                const float sc = (a0 + a1) * ks;
+                scores[(int64_t)(row0 + q) * ld + s] = sc;
+                if constexpr (kHist) dig[q] = ordered_key(sc) >> 21;
+              }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(tc::smem_u32(&S->tempty[eg]));
+            if constexpr (kHist) {
+              // counted after the accumulator is handed back (an arrive orders every earlier memory operation
+              // of the warp before it, so adds in front of it would hold the tensor core up)
+#pragma unroll
+              for (int q = 0; q < kIdxRows; ++q)
+                if (dig[q] != 0x80000000u) {
+                  const uint32_t addr = tc::smem_u32(&sHist[q * (kIdxHistBins / 2) + (dig[q] >> 1)]);
+                  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"((dig[q] & 1u) ? 0x10000u : 1u) : "memory");
+                }
+            }
           }
+          acc_phase ^= 1u;
         }
         ++span;
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         if (++t == tp[gi + 1] - tp[gi]) { ++gi; t = 0; }
       }
-      if (kHist && cur >= 0) flush();
+      if (cur >= 0) {
+        if (kHist) flush();
+        release_group();
+      }
     }
   }
   tc::fence_before_sync();

@@ -3,7 +3,9 @@
 // Selection order: score descending, token position ascending (the lower position wins a tie;
 // -0 == +0).  Scores are compared as order-preserving u32 keys, so the selection is exact.
 // The k-th key T is found digit by digit (11 + 11 + 10 bits) with shared-memory histograms; every
-// key > T is selected plus the lowest-positioned keys == T until k are taken.  The result is
+// key > T is selected plus the lowest-positioned keys == T until k are taken.  The passes stop early once
+// the threshold digit's bin holds exactly the keys still needed (keys are then compared on the digits
+// fixed so far).  The result is
 // written in ascending position order by a block-wide ordered compaction, so no sort is needed.
 //
 // Rows are grouped by row, buffered in shared memory and read with 16-byte vector loads, the
@@ -218,6 +220,9 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
     pmask |= (uint32_t)(nb - 1) << shift;
     k_rem -= s_above;
     __syncthreads();
+    // every key of the threshold bin is taken: no finer digit can change the selection, so the keys are
+    // compared on the digits fixed so far (the same row histogram in every CTA of the cluster: they all stop)
+    if (ghist[s_bin] == k_rem) break;
   }
   const uint32_t T = prefix;
 
@@ -227,7 +232,7 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
   const int tlo = min(m, tid * per), thi = min(m, tlo + per);
   uint32_t gt = 0, eq = 0;
   for (int i = tlo; i < thi; ++i) {
-    uint32_t u = keys[i];
+    uint32_t u = keys[i] & pmask;
     gt += u > T;
     eq += u == T;
   }
@@ -255,7 +260,7 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
   uint32_t off = out_base + gt_before + eq_taken_slice;
   uint32_t e = 0;
   for (int i = tlo; i < thi; ++i) {
-    uint32_t u = keys[i];
+    uint32_t u = keys[i] & pmask;
     bool sel = u > T;
     if (u == T) { sel = e < take_eq; ++e; }
     if (sel && off < (uint32_t)k) out[off++] = lo + i;

@@ -15,9 +15,10 @@
 // Two regimes:
 //   A) n <= C * kTopkSmemCap candidates: a cluster of C CTAs per row (C = 1, 2, 4 or 8: more when there
 //      are few rows, so that the rows fill the GPU, and as many as the longest row needs, at most 2 for
-//      a large batch), each CTA staging one contiguous slice of the row in shared memory.  Every digit pass builds slice histograms, which each CTA sums over the cluster
-//      through distributed shared memory to the same row histogram; the ordered write offsets each
-//      slice by the counts of the slices before it.  One launch.
+//      a large batch), each CTA staging one contiguous slice of the row in shared memory.  Every digit
+//      pass builds slice histograms whose non-zero bins each CTA adds into every CTA's copy of the row
+//      histogram (distributed shared memory atomics, then one cluster barrier); the ordered write offsets
+//      each slice by the counts of the slices before it, stored into the later CTAs.  One launch.
 //   B) longer rows (a million-token decode): the row is split into segments of kTopkSeg keys over
 //      a persistent grid; each digit pass is one launch whose CTAs add segment histograms into a
 //      per-row global histogram, and the last CTA of a row to finish (atomic counter, no waiting)
@@ -120,31 +121,45 @@ __device__ __forceinline__ uint32_t cl_size() {
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
   return r;
 }
-__device__ __forceinline__ void cl_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// u32 at the same shared-memory location in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t cl_ld(const void *p, uint32_t rank) {
-  uint32_t a = (uint32_t)__cvta_generic_to_shared(p), ra, v;
+// red.shared::cluster.add of v to the u32 at the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ void cl_red_add(const void *p, uint32_t rank, uint32_t v) {
+  uint32_t a = (uint32_t)__cvta_generic_to_shared(p), ra;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
-  return v;
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
+}
+__device__ __forceinline__ void cl_st(const void *p, uint32_t rank, uint32_t v) {
+  uint32_t a = (uint32_t)__cvta_generic_to_shared(p), ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
+}
+// (aligned forms: the warp is made converged first, as they require)
+__device__ __forceinline__ void cl_arrive() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cl_wait() {
+  __syncwarp();
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// shared memory of a regime-A CTA: two slice histograms (alternating passes), the row histogram, scan
-// scratch, the slice's counts, then the slice's keys
-constexpr int kTopkSmemFixedU32 = 3 * kRadixBins + 64 + 4;
+// shared memory of a regime-A CTA: the slice histogram, two row histograms (alternating passes), scan scratch,
+// the slices' counts for the ordered write (pairs, up to 16 CTAs), then the slice's keys
+constexpr int kTopkMaxCluster = 16;
+constexpr int kTopkSmemFixedU32 = 3 * kRadixBins + 64 + 2 * kTopkMaxCluster;
 
+// Every access to another CTA's shared memory is a push (an add or a store) issued before a cluster barrier
+// that the receiver waits on: the row histogram of a pass is the sum of the slice histograms' non-zero bins,
+// added into every CTA's copy; the ordered write's offsets come from counts stored into the later CTAs.  No
+// CTA reads a peer's shared memory, so none has to wait for its peers before it exits.
 __global__ void __launch_bounds__(kTopkThreadsA)
 topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, int k,
                       int32_t *__restrict__ idx, TopkWs lw, int register_long) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) uint32_t sm[];
-  uint32_t *hist_s[2] = {sm, sm + kRadixBins};          // this slice, even / odd passes
-  uint32_t *ghist = sm + 2 * kRadixBins;                 // the row (sum over the cluster)
+  uint32_t *hist = sm;                                   // this slice
   uint32_t *tmp = sm + 3 * kRadixBins;
-  uint32_t *cnt = tmp + 64;                              // [0] keys > T, [1] keys == T in this slice
+  uint32_t *cnts = tmp + 64;                             // (keys > T, keys == T) of the slice of each rank
   uint32_t *keys = sm + kTopkSmemFixedU32;
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
@@ -153,7 +168,7 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
   const int row = blockIdx.x / (int)C;
   const int tid = threadIdx.x, bs = blockDim.x;
   int b;
-  const int n = pos_of_row(bv, row, &b) + 1;
+  const int n = pos_of_row_warp(bv, row, &b) + 1;
   int32_t *out = idx + (int64_t)row * k;
 
   // (every branch below depends on n only, so all CTAs of a cluster take it together)
@@ -175,6 +190,11 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
     return;
   }
 
+  // both row histograms start empty before any peer adds into them: the barrier that publishes the clearing
+  // is waited on just before the first push, so the slice load and histogram run meanwhile
+  for (int i = tid; i < 2 * kRadixBins; i += bs) sm[kRadixBins + i] = 0u;
+  if (C > 1) cl_arrive();
+
   // this CTA's slice [lo, lo + m): a multiple of 4 keys long, so 16-byte loads stay aligned
   const int slice = ((n + (int)C - 1) / (int)C + 3) & ~3;
   const int lo = min(n, (int)r * slice), m = min(n, lo + slice) - lo;
@@ -194,7 +214,7 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const int nb = pass == 2 ? 1024 : 2048;
-    uint32_t *hist = hist_s[pass & 1];
+    uint32_t *ghist = sm + kRadixBins * (1 + (pass & 1));   // the row histogram of this pass (even / odd)
     for (int i = tid; i < nb; i += bs) hist[i] = 0u;
     __syncthreads();
     for (int i = tid; i < m; i += bs) {
@@ -203,26 +223,31 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
     }
     __syncthreads();
     if (C > 1) {
-      // every slice histogram of the row is complete (the other parity's buffers were last read before
-      // this barrier, so they may be cleared in the next pass)
-      cl_sync();
+      // add the slice's non-zero bins into every CTA's row histogram; the barrier completes the row histograms
+      if (pass == 0) cl_wait();
       for (int i = tid; i < nb; i += bs) {
-        uint32_t sum = 0u;
-        for (uint32_t c = 0; c < C; ++c) sum += cl_ld(hist + i, c);
-        ghist[i] = sum;
+        const uint32_t v = hist[i];
+        if (v != 0u)
+          for (uint32_t c = 0; c < C; ++c) cl_red_add(ghist + i, c, v);
       }
+      cl_arrive();
+      cl_wait();
     } else {
       for (int i = tid; i < nb; i += bs) ghist[i] = hist[i];
+      __syncthreads();
     }
-    __syncthreads();
     find_threshold_bin(ghist, nb, k_rem, tmp, &s_bin, &s_above);
     prefix |= (uint32_t)s_bin << shift;
     pmask |= (uint32_t)(nb - 1) << shift;
     k_rem -= s_above;
-    __syncthreads();
     // every key of the threshold bin is taken: no finer digit can change the selection, so the keys are
     // compared on the digits fixed so far (the same row histogram in every CTA of the cluster: they all stop)
-    if (ghist[s_bin] == k_rem) break;
+    const bool last = ghist[s_bin] == k_rem;
+    __syncthreads();
+    // this row histogram takes the adds of pass + 2, which peers make only after the next pass's barrier,
+    // which this CTA reaches after clearing it
+    for (int i = tid; i < nb; i += bs) ghist[i] = 0u;
+    if (last) break;
   }
   const uint32_t T = prefix;
 
@@ -241,13 +266,15 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
   const uint32_t gt_before = block_exclusive_scan(gt, tmp, &gt_tot);
   uint32_t out_base = 0u, eq_base = 0u;
   if (C > 1) {
-    if (tid == 0) {
-      cnt[0] = gt_tot;
-      cnt[1] = eq_tot;
+    // this slice's counts go to the CTAs after it
+    if (tid > (int)r && tid < (int)C) {
+      cl_st(cnts + 2 * r, (uint32_t)tid, gt_tot);
+      cl_st(cnts + 2 * r + 1, (uint32_t)tid, eq_tot);
     }
-    cl_sync();
+    cl_arrive();
+    cl_wait();
     for (uint32_t c = 0; c < r; ++c) {
-      const uint32_t g = cl_ld(cnt, c), e = cl_ld(cnt + 1, c);
+      const uint32_t g = cnts[2 * c], e = cnts[2 * c + 1];
       const uint32_t take = k_rem > eq_base ? min(e, k_rem - eq_base) : 0u;
       out_base += g + take;
       eq_base += e;
@@ -265,8 +292,6 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
     if (u == T) { sel = e < take_eq; ++e; }
     if (sel && off < (uint32_t)k) out[off++] = lo + i;
   }
-  // no CTA leaves while another may still read its shared memory
-  if (C > 1) cl_sync();
 }
 
 // ------------------------------------------------------------------------------------------------

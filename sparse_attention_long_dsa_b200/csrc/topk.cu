@@ -108,6 +108,58 @@ __device__ void find_threshold_bin(const uint32_t *hist, int nbins, uint32_t k_r
   __syncthreads();
 }
 
+// The same for a block of at least 32 warps, in two levels: warp w sums the w-th group of nbins / 32 bins
+// from the top, then warp 0 scans the 32 group sums, and scans the chosen group's bins (one or two per lane).
+// Two block barriers.  Needs 1 <= k_rem <= the histogram's total (so one bin qualifies).
+__device__ void find_threshold_bin_w32(const uint32_t *hist, int nbins, uint32_t k_rem, uint32_t *tmp,
+                                       int *s_bin, uint32_t *s_above) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gsz = nbins >> 5;                                  // bins per group: 64 or 32
+  if (warp < 32) {
+    const int g0 = nbins - (warp + 1) * gsz;
+    uint32_t s = 0;
+    for (int j = lane; j < gsz; j += 32) s += hist[g0 + j];
+    s = __reduce_add_sync(0xffffffffu, s);
+    if (lane == 0) tmp[warp] = s;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // groups from the top: lane l holds group l; exactly one group holds the k_rem-th key
+    const uint32_t gs = tmp[lane];
+    uint32_t incl = gs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int gw = __ffs(__ballot_sync(0xffffffffu, incl - gs < k_rem && incl >= k_rem)) - 1;
+    const uint32_t above = __shfl_sync(0xffffffffu, incl - gs, gw);
+    const uint32_t need = k_rem - above;
+    // the group's bins from the top: lane l takes the per = gsz / 32 bins below top - per * l
+    const int per = gsz >> 5;
+    const int hi = nbins - gw * gsz - 1 - per * lane;
+    const uint32_t c0 = hist[hi], c1 = per == 2 ? hist[hi - 1] : 0u;
+    const uint32_t loc = c0 + c1;
+    uint32_t incl2 = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl2, o);
+      if (lane >= o) incl2 += y;
+    }
+    const uint32_t excl2 = incl2 - loc;
+    if (excl2 < need && incl2 >= need) {
+      if (excl2 + c0 >= need) {
+        *s_bin = hi;
+        *s_above = above + excl2;
+      } else {
+        *s_bin = hi - 1;
+        *s_above = above + excl2 + c0;
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // ------------------------------------------------------------------------------------------------
 // Regime A
 // ------------------------------------------------------------------------------------------------
@@ -167,8 +219,24 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
   const uint32_t C = cl_size(), r = cl_rank();
   const int row = blockIdx.x / (int)C;
   const int tid = threadIdx.x, bs = blockDim.x;
-  int b;
-  const int n = pos_of_row_warp(bv, row, &b) + 1;
+  // the row's length: one round of loads for a batch of one query row per sequence (the row is its
+  // sequence: its entries are loaded beside the search's), two otherwise
+  int n;
+  {
+    int sc0 = 0, sc1 = 0, ssl = 0;
+    if (row < bv.num_seqs) {
+      sc0 = __ldg(bv.cu_q + row);
+      sc1 = __ldg(bv.cu_q + row + 1);
+      ssl = __ldg(bv.seq_lens + row);
+    }
+    const int b = seq_of_row_warp(bv.cu_q, bv.num_seqs, row);
+    if (b == row) {
+      n = ssl - (sc1 - sc0) + (row - sc0) + 1;
+    } else {
+      const int c0 = __ldg(bv.cu_q + b), c1 = __ldg(bv.cu_q + b + 1);
+      n = __ldg(bv.seq_lens + b) - (c1 - c0) + (row - c0) + 1;
+    }
+  }
   int32_t *out = idx + (int64_t)row * k;
 
   // (every branch below depends on n only, so all CTAs of a cluster take it together)
@@ -236,7 +304,7 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
       for (int i = tid; i < nb; i += bs) ghist[i] = hist[i];
       __syncthreads();
     }
-    find_threshold_bin(ghist, nb, k_rem, tmp, &s_bin, &s_above);
+    find_threshold_bin_w32(ghist, nb, k_rem, tmp, &s_bin, &s_above);
     prefix |= (uint32_t)s_bin << shift;
     pmask |= (uint32_t)(nb - 1) << shift;
     k_rem -= s_above;
@@ -261,9 +329,12 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
     gt += u > T;
     eq += u == T;
   }
-  uint32_t gt_tot, eq_tot;
-  uint32_t eq_before = block_exclusive_scan(eq, tmp, &eq_tot);
-  const uint32_t gt_before = block_exclusive_scan(gt, tmp, &gt_tot);
+  // both counts in one scan: (gt << 16) | eq never carries, a slice holding at most kTopkSmemCap < 65536 keys
+  uint32_t tot;
+  const uint32_t before = block_exclusive_scan((gt << 16) | eq, tmp, &tot);
+  const uint32_t gt_tot = tot >> 16, eq_tot = tot & 0xFFFFu;
+  uint32_t eq_before = before & 0xFFFFu;
+  const uint32_t gt_before = before >> 16;
   uint32_t out_base = 0u, eq_base = 0u;
   if (C > 1) {
     // this slice's counts go to the CTAs after it

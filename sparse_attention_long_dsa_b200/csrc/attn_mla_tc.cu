@@ -688,8 +688,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
 
 // ------------------------------------------------------------------------------------------------ combine
 // out[row, h, :] = sum_s exp(lse_s - lse) o_s,  lse = log sum_s exp(lse_s)   (splits of one row)
-// The splits' lse values are read once into registers (up to kCombineRegSplits of them; more are re-read), so
-// a thread waits on two rounds of loads: the lse values, then all splits' partial outputs at once.
+// The splits' lse values and partial outputs (up to kCombineRegSplits of each) are loaded in one round; a split
+// with lse = -inf wrote zeros and gets weight 0.  More splits are re-read in a second loop.
 constexpr int kCombineRegSplits = 8;
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restrict__ part_o,
                                                            const float *__restrict__ part_lse, int splits,
@@ -698,9 +698,16 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restri
   pdl_trigger();
   const int row = blockIdx.x, h = blockIdx.y;
   const float *pl = part_lse + (int64_t)row * splits * kAttH + h;
+  const int dv = threadIdx.x * 4;
+  const float *po = part_o + ((int64_t)row * splits * kAttH + h) * kAttDv + dv;
   float lreg[kCombineRegSplits];
+  float4 o[kCombineRegSplits];
 #pragma unroll
-  for (int s = 0; s < kCombineRegSplits; ++s) lreg[s] = s < splits ? __ldg(pl + (int64_t)s * kAttH) : -INFINITY;
+  for (int s = 0; s < kCombineRegSplits; ++s) {
+    lreg[s] = s < splits ? __ldg(pl + (int64_t)s * kAttH) : -INFINITY;
+    o[s] = s < splits ? __ldg(reinterpret_cast<const float4 *>(po + (int64_t)s * kAttH * kAttDv))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   float mx = -INFINITY;
 #pragma unroll
   for (int s = 0; s < kCombineRegSplits; ++s) mx = fmaxf(mx, lreg[s]);
@@ -713,15 +720,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restri
     const float l = __ldg(pl + (int64_t)s * kAttH);
     tot += l == -INFINITY ? 0.f : __expf(l - mx);
   }
-  const int dv = threadIdx.x * 4;
-  const float *po = part_o + ((int64_t)row * splits * kAttH + h) * kAttDv + dv;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (tot > 0.f) {
-    float4 o[kCombineRegSplits];
-#pragma unroll
-    for (int s = 0; s < kCombineRegSplits; ++s)
-      o[s] = (s < splits && lreg[s] != -INFINITY) ? __ldg(reinterpret_cast<const float4 *>(po + (int64_t)s * kAttH * kAttDv))
-                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int s = 0; s < kCombineRegSplits; ++s) {
       if (s >= splits || lreg[s] == -INFINITY) continue;

@@ -221,7 +221,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   float *sKS = sW + 2 * (kIdxWSlotBytes / 4);                     // kIdxStages x 128 key scales
   uint32_t *sHist = (uint32_t *)(sKS + kIdxStages * kIdxTile);    // kIdxRows x 2048 16-bit counters
   int32_t *sTP = (int32_t *)(sHist + kIdxRows * (kIdxHistBins / 2));   // in-kernel plan: tile prefix
-  IdxSmem *S = (IdxSmem *)(sTP + kIdxInlinePlanMax + 4);
+  int32_t *sSL = sTP + kIdxInlinePlanMax + 4;                          // in-kernel plan: sequence lengths
+  IdxSmem *S = (IdxSmem *)(sSL + kIdxInlinePlanMax);
   __shared__ uint32_t s_scan[64];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -263,10 +264,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint32_t carry = 0;
     for (int base = 0; base < G; base += kIdxThreads) {
       const int g = base + (int)threadIdx.x;
-      const uint32_t tiles = g < G ? (uint32_t)((__ldg(bv.seq_lens + g) - 1) / kIdxTile + 1) : 0u;
+      const int sl = g < G ? __ldg(bv.seq_lens + g) : 1;
+      const uint32_t tiles = g < G ? (uint32_t)((sl - 1) / kIdxTile + 1) : 0u;
       uint32_t tot;
       const uint32_t ex = block_exclusive_scan(tiles, s_scan, &tot);
-      if (g < G) sTP[g] = (int)(carry + ex);
+      if (g < G) {
+        sTP[g] = (int)(carry + ex);
+        sSL[g] = sl;
+      }
       carry += tot;
     }
     if (threadIdx.x == 0) sTP[G] = (int)carry;
@@ -328,8 +333,13 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         if (m < mine) {
           unit_locate(tp, G, u, &gi, &t);
           const int b = g_seq(gi);
-          const int c0 = __ldg(bv.cu_q + b), nbq = __ldg(bv.cu_q + b + 1) - c0;
-          const int pos_last = __ldg(bv.seq_lens + b) - nbq + (g_row0(gi) - c0) + g_nrows(gi) - 1;
+          int pos_last;
+          if (inline_plan) {
+            pos_last = sSL[b] - 1;                          // one query row per sequence, at its last position
+          } else {
+            const int c0 = __ldg(bv.cu_q + b), nbq = __ldg(bv.cu_q + b + 1) - c0;
+            pos_last = __ldg(bv.seq_lens + b) - nbq + (g_row0(gi) - c0) + g_nrows(gi) - 1;
+          }
           const int pages = pos_last / 64 + 1;
           const int32_t *btr = bv.block_table + (int64_t)b * bv.max_blocks_per_seq;
           blk0 = __ldg(btr + 2 * t);
@@ -503,8 +513,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           b = g_seq(gi);
           row0 = g_row0(gi);
           nr = g_nrows(gi);
-          const int c0 = __ldg(bv.cu_q + b);
-          pos0 = __ldg(bv.seq_lens + b) - (__ldg(bv.cu_q + b + 1) - c0) + (row0 - c0);
+          if (inline_plan) {
+            pos0 = sSL[b] - 1;
+          } else {
+            const int c0 = __ldg(bv.cu_q + b);
+            pos0 = __ldg(bv.seq_lens + b) - (__ldg(bv.cu_q + b + 1) - c0) + (row0 - c0);
+          }
         } else if (kHist && span == kIdxHistFlushTiles) {
           flush();
         }
@@ -617,7 +631,7 @@ static bool make_rows128_map(CUtensorMap *m, const void *base, uint64_t rows) {
 
 static size_t indexer_tc_smem() {
   return 1024 + kIdxStages * kIdxTileBytes + 2 * kIdxBSlotBytes + 2 * kIdxWSlotBytes + kIdxStages * kIdxTile * 4 +
-         kIdxRows * (kIdxHistBins / 2) * 4 + (kIdxInlinePlanMax + 4) * 4 + sizeof(IdxSmem);
+         kIdxRows * (kIdxHistBins / 2) * 4 + (kIdxInlinePlanMax + 4) * 4 + kIdxInlinePlanMax * 4 + sizeof(IdxSmem);
 }
 
 size_t indexer_hist_bytes(int total_q) { return al256((size_t)total_q * kIdxHistBins * 4); }

@@ -11,15 +11,18 @@
 // the survivors -- keys whose digit is at or above the threshold digit, about k plus the threshold bin --
 // in shared memory, finishes the selection on those, and writes the result.
 //
-// Per row a cluster of C CTAs (C = 1 .. 16) takes contiguous slices.  State shared by the cluster: the
-// fixed key bits (prefix P under mask M), the count `above` of keys strictly above the prefix, the number
-// `need` still to take from the prefix's bin, and that bin's size.  While the survivors would not fit in
-// the capacity, one more streaming pass histograms the next digit (11, 11 then 10 bits) among keys in the
-// bin, summed over the cluster through distributed shared memory.  When every bit is fixed, keys equal to
-// the threshold are kept in position order up to `need`, so the survivors are then exactly k.  The storing
-// pass compacts survivors in position order; rank 0 collects the other slices' survivors after its own,
-// resolves the remaining bits on them and emits every survivor above the threshold plus the first `need`
-// equal ones.  Without a histogram (plain scores) the first pass counts the leading digit itself.
+// Per row a cluster of C CTAs (C = 1 .. 16) takes contiguous slices; every CTA keeps the same selection state
+// (fixed key bits: prefix P under mask M; `above` keys strictly above the prefix; `need` still to take from the
+// prefix's bin of `bin_cnt` keys).  A digit is fixed from a row histogram that every CTA holds a copy of: each
+// CTA adds the non-zero bins of its slice's histogram into every CTA's copy (distributed shared memory
+// atomics, then one cluster barrier).  While the survivors would not fit in the capacity, a counting pass over
+// the slice fixes the next digit (11, 11 then 10 bits).  When every bit is fixed, keys equal to the threshold
+// are kept in position order up to `need` (the slices before take theirs first), so the survivors always fit.
+// The storing pass compacts each slice's survivors in position order; the remaining digits are fixed on the
+// survivors the same way (stopping as soon as the prefix's bin holds exactly the keys still needed); then each
+// slice writes its selected positions, offset by the counts of the slices before it, stored into the later
+// CTAs before a barrier.  No CTA reads another's shared memory.  Without a histogram (plain scores) the first
+// counting pass fixes the leading digit.
 #include <algorithm>
 #include <atomic>
 #include <cstdio>
@@ -30,9 +33,13 @@
 namespace dsa {
 
 constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelBins = 2048;
 constexpr int kSelPerThread = 8;                        // keys per thread per tile (2 x float4)
 constexpr int kSelTile = kSelThreads * kSelPerThread;   // 4096 keys
+constexpr int kSelBatch = 2;                            // tiles whose loads are issued together
+constexpr int kSelVec = kSelPerThread / 4;
+constexpr int kSelMaxCluster = 16;
 
 struct SelArgs {
   const float *scores;
@@ -45,9 +52,9 @@ struct SelArgs {
   uint32_t *status;
 };
 
-// shared memory: survivors (key, position) [cap], two local histograms, the cluster histogram, scan scratch,
-// per-CTA counts read by the other CTAs of the cluster
-constexpr int kSelFixedWords = 3 * kSelBins + 64 + 8;
+// shared memory (u32 words): survivors (key, position) [cap], the slice histogram, two row histograms
+// (alternating passes), scan scratch, the earlier slices' equal-key counts (full case) and final counts
+constexpr int kSelFixedWords = 3 * kSelBins + 64 + kSelMaxCluster + 2 * kSelMaxCluster;
 size_t select_smem_bytes(int cap) { return ((size_t)2 * cap + kSelFixedWords) * 4; }
 
 __device__ __forceinline__ uint32_t sel_cl_nranks() {
@@ -55,35 +62,75 @@ __device__ __forceinline__ uint32_t sel_cl_nranks() {
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
   return r;
 }
-// u32 at the same shared-memory location in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t sel_cl_ld(const void *p, uint32_t rank) {
-  const uint32_t ra = tc::map_to_rank(tc::smem_u32(p), rank);
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
-  return v;
+__device__ __forceinline__ void sel_cl_red_add(const uint32_t *p, uint32_t rank, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(tc::map_to_rank(tc::smem_u32(p), rank)), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sel_cl_st(const uint32_t *p, uint32_t rank, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(tc::map_to_rank(tc::smem_u32(p), rank)), "r"(v) : "memory");
+}
+// split cluster barrier (aligned forms: the warp is made converged first)
+__device__ __forceinline__ void sel_cl_arrive() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void sel_cl_wait() {
+  __syncwarp();
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Bin holding the need-th key counted from the top of hist[0..nb) (need >= 1, at most the total).  Returns
-// it in *s_bin and the count of keys in higher bins in *s_above.  Every thread of the block calls this (a
-// block scan over per-thread runs of bins in descending order).
+// Bin holding the need-th key counted from the top of hist[0..nb) (1 <= need <= the total), and the count of
+// keys in higher bins.  Two levels: warp w sums the w-th group of nb / 16 bins from the top, then warp 0 scans the
+// 16 group sums and the chosen group's bins (nb / 512 per lane, the lane's own ones in order).  Every thread of
+// the block calls it; two block barriers.
 __device__ void sel_find_bin(const uint32_t *hist, int nb, uint32_t need, uint32_t *tmp, int *s_bin,
                              uint32_t *s_above) {
-  const int per = (nb + kSelThreads - 1) / kSelThreads;
-  const int d0 = threadIdx.x * per;                    // position in descending bin order
-  if (threadIdx.x == 0) {                              // (a consistent histogram always overwrites these)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gsz = nb / kSelWarps;                          // 128 or 64
+  if (threadIdx.x == 0) {                                  // (a consistent histogram always overwrites these)
     *s_bin = 0;
     *s_above = 0u;
   }
-  uint32_t local = 0;
-  for (int d = d0; d < d0 + per && d < nb; ++d) local += hist[nb - 1 - d];
-  uint32_t run = block_exclusive_scan(local, tmp, nullptr);
-  for (int d = d0; d < d0 + per && d < nb; ++d) {
-    const uint32_t c = hist[nb - 1 - d];
-    if (run < need && run + c >= need) {
-      *s_bin = nb - 1 - d;
-      *s_above = run;
+  {
+    const int g0 = nb - (warp + 1) * gsz;
+    uint32_t s = 0;
+    for (int j = lane; j < gsz; j += 32) s += hist[g0 + j];
+    s = __reduce_add_sync(0xffffffffu, s);
+    if (lane == 0) tmp[warp] = s;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t gs = lane < kSelWarps ? tmp[lane] : 0u;
+    uint32_t incl = gs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    run += c;
+    const int gw = __ffs(__ballot_sync(0xffffffffu, incl - gs < need && incl >= need)) - 1;
+    const uint32_t above = __shfl_sync(0xffffffffu, incl - gs, gw < 0 ? 0 : gw);
+    const uint32_t want = need - above;
+    const int per = gsz >> 5;                              // 4 or 2 bins per lane, from the group's top down
+    const int hi = nb - (gw < 0 ? 0 : gw) * gsz - 1 - per * lane;
+    uint32_t loc = 0;
+    for (int e = 0; e < per; ++e) loc += hist[hi - e];
+    uint32_t incl2 = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl2, o);
+      if (lane >= o) incl2 += y;
+    }
+    uint32_t run = incl2 - loc;
+    if (gw >= 0 && run < want && incl2 >= want) {
+      for (int e = 0; e < per; ++e) {
+        const uint32_t c = hist[hi - e];
+        if (run + c >= want) {
+          *s_bin = hi - e;
+          *s_above = above + run;
+          break;
+        }
+        run += c;
+      }
+    }
   }
   __syncthreads();
 }
@@ -94,33 +141,47 @@ __device__ void sel_find_bin(const uint32_t *hist, int nb, uint32_t need, uint32
 __device__ __forceinline__ int sel_elem(int base, int v, int j) {
   return base + (int)(threadIdx.x >> 5) * (32 * kSelPerThread) + 128 * v + 4 * (int)(threadIdx.x & 31) + j;
 }
-__device__ __forceinline__ void sel_load_tile(const float *src, int m, int base, uint32_t (&key)[kSelPerThread],
-                                              uint32_t &valid) {
+// Loads are issued for a whole batch of tiles before any value is used (a load followed at once by its use
+// would cost a memory round trip per vector), and a batch's loads are issued before the previous batch is
+// processed.  Positions at or past m read as 0 and are marked invalid at conversion.
+struct SelRaw {
+  float4 f[kSelBatch][kSelVec];
+};
+__device__ __forceinline__ void sel_issue(const float *src, int m, int base, SelRaw &raw) {
+#pragma unroll
+  for (int t = 0; t < kSelBatch; ++t)
+#pragma unroll
+    for (int v = 0; v < kSelVec; ++v) {
+      const int i0 = sel_elem(base + t * kSelTile, v, 0);
+      if (i0 + 4 <= m) {
+        raw.f[t][v] = __ldg(reinterpret_cast<const float4 *>(src + i0));
+      } else {
+        raw.f[t][v].x = i0 < m ? __ldg(src + i0) : 0.f;
+        raw.f[t][v].y = i0 + 1 < m ? __ldg(src + i0 + 1) : 0.f;
+        raw.f[t][v].z = i0 + 2 < m ? __ldg(src + i0 + 2) : 0.f;
+        raw.f[t][v].w = i0 + 3 < m ? __ldg(src + i0 + 3) : 0.f;
+      }
+    }
+}
+__device__ __forceinline__ void sel_convert(const SelRaw &raw, int t, int m, int base, uint32_t (&key)[kSelPerThread],
+                                            uint32_t &valid) {
   valid = 0u;
 #pragma unroll
-  for (int v = 0; v < kSelPerThread / 4; ++v) {
+  for (int v = 0; v < kSelVec; ++v) {
     const int i0 = sel_elem(base, v, 0);
-    if (i0 + 4 <= m) {
-      const float4 f = __ldg(reinterpret_cast<const float4 *>(src + i0));
-      key[4 * v] = ordered_key(f.x);
-      key[4 * v + 1] = ordered_key(f.y);
-      key[4 * v + 2] = ordered_key(f.z);
-      key[4 * v + 3] = ordered_key(f.w);
-      valid |= 0xFu << (4 * v);
-    } else {
+    const float fv[4] = {raw.f[t][v].x, raw.f[t][v].y, raw.f[t][v].z, raw.f[t][v].w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const bool in = i0 + j < m;
-        key[4 * v + j] = in ? ordered_key(__ldg(src + i0 + j)) : 0u;
-        valid |= (in ? 1u : 0u) << (4 * v + j);
-      }
+    for (int j = 0; j < 4; ++j) {
+      const bool in = i0 + j < m;
+      key[4 * v + j] = in ? ordered_key(fv[j]) : 0u;
+      valid |= (in ? 1u : 0u) << (4 * v + j);
     }
   }
 }
 
 // Ordered positions of flagged items in a tile laid out as sel_elem describes: flags bit 4 v + j.  Returns, for
 // each v, the count of flagged items before (v, lane, 0) in the tile (pre[v]), and the tile's total; `wsum`
-// holds 32 words of shared scratch.  One __syncthreads inside, one more before wsum is reused.
+// holds 16 words of shared scratch.  One __syncthreads inside, one more before wsum is reused.
 __device__ __forceinline__ uint32_t sel_tile_prefix(uint32_t flags, uint32_t (&pre)[kSelPerThread / 4], uint32_t *wsum) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t run = 0u;
@@ -139,7 +200,8 @@ __device__ __forceinline__ uint32_t sel_tile_prefix(uint32_t flags, uint32_t (&p
   if (lane == 0) wsum[warp] = run;
   __syncthreads();
   uint32_t before = 0u, total = 0u;
-  for (int w = 0; w < kSelThreads / 32; ++w) {
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
     const uint32_t x = wsum[w];
     before += w < warp ? x : 0u;
     total += x;
@@ -149,26 +211,43 @@ __device__ __forceinline__ uint32_t sel_tile_prefix(uint32_t flags, uint32_t (&p
   return total;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArgs a) {
+__global__ void __launch_bounds__(kSelThreads, 2) select_stream_kernel(const SelArgs a) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) uint32_t sm[];
+  const uint32_t cap = (uint32_t)a.cap;
   uint32_t *skey = sm;
-  int32_t *spos = reinterpret_cast<int32_t *>(sm + a.cap);
-  uint32_t *lh[2] = {sm + 2 * a.cap, sm + 2 * a.cap + kSelBins};
-  uint32_t *gh = sm + 2 * a.cap + 2 * kSelBins;
-  uint32_t *tmp = gh + kSelBins;
-  uint32_t *info = tmp + 64;           // [0] survivors stored, [1] keys equal to the final prefix in this slice
+  int32_t *spos = reinterpret_cast<int32_t *>(sm + cap);
+  uint32_t *lh = sm + 2 * cap;                 // this slice's histogram of the current digit
+  uint32_t *gh0 = lh + kSelBins;               // row histograms, even / odd pushed passes
+  uint32_t *tmp = gh0 + 2 * kSelBins;
+  uint32_t *eq_in = tmp + 64;                  // [c]: equal keys in slice c (full case), stored by CTA c
+  uint32_t *cnt_in = eq_in + kSelMaxCluster;   // [2c], [2c + 1]: (keys > T, keys == T) among slice c's survivors
   __shared__ int s_bin;
   __shared__ uint32_t s_above, s_flag;
 
   const uint32_t C = sel_cl_nranks(), r = tc::cluster_ctarank();
   const int row = blockIdx.x / (int)C;
-  const int tid = threadIdx.x;
-  int b;
-  const int n = pos_of_row_warp(a.bv, row, &b) + 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the row's length: one round of loads for a batch of one query row per sequence (the row is its sequence)
+  int n;
+  {
+    int sc0 = 0, sc1 = 0, ssl = 0;
+    if (row < a.bv.num_seqs) {
+      sc0 = __ldg(a.bv.cu_q + row);
+      sc1 = __ldg(a.bv.cu_q + row + 1);
+      ssl = __ldg(a.bv.seq_lens + row);
+    }
+    const int b = seq_of_row_warp(a.bv.cu_q, a.bv.num_seqs, row);
+    if (b == row) {
+      n = ssl - (sc1 - sc0) + (row - sc0) + 1;
+    } else {
+      const int c0 = __ldg(a.bv.cu_q + b), c1 = __ldg(a.bv.cu_q + b + 1);
+      n = __ldg(a.bv.seq_lens + b) - (c1 - c0) + (row - c0) + 1;
+    }
+  }
   int32_t *out = a.idx + (int64_t)row * a.k;
-  // (every branch on n is taken by the whole cluster)
+  // (every branch on n, on the row histograms and on the selection state is taken by the whole cluster)
   if (n <= a.k) {
     if (r == 0)
       for (int j = tid; j < a.k; j += kSelThreads) out[j] = j < n ? j : -1;
@@ -177,202 +256,245 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
   const int per = ((n + (int)C - 1) / (int)C + 3) & ~3;
   const int lo = min(n, (int)r * per), m = min(n, lo + per) - lo;
   const float *src = a.scores + (int64_t)row * a.ld + lo;
-  const uint32_t cap = (uint32_t)a.cap;
+
+  // both row histograms start empty before any CTA adds into them; the barrier publishing that is waited on
+  // just before the first push
+  for (int i = tid; i < 2 * kSelBins; i += kSelThreads) gh0[i] = 0u;
+  bool wait_pending = false;
+  if (C > 1) {
+    sel_cl_arrive();
+    wait_pending = true;
+  }
+  int pushes = 0;
+  // this slice's histogram lh[0..nb) -> the row histogram (every CTA's copy); returns it
+  auto row_hist = [&](int nb) -> uint32_t * {
+    uint32_t *gh = gh0 + (pushes & 1) * kSelBins;
+    if (C > 1) {
+      if (wait_pending) {
+        sel_cl_wait();
+        wait_pending = false;
+      }
+      for (int i = tid; i < nb; i += kSelThreads) {
+        const uint32_t v = lh[i];
+        if (v != 0u)
+          for (uint32_t c = 0; c < C; ++c) sel_cl_red_add(gh + i, c, v);
+      }
+      sel_cl_arrive();
+      sel_cl_wait();
+    } else {
+      for (int i = tid; i < nb; i += kSelThreads) gh[i] = lh[i];
+      __syncthreads();
+    }
+    ++pushes;
+    return gh;
+  };
+  // done with a row histogram: cleared for the pass after next (peers add into it only after the next barrier)
+  auto release_row_hist = [&](uint32_t *gh, int nb) {
+    __syncthreads();
+    for (int i = tid; i < nb; i += kSelThreads) gh[i] = 0u;
+  };
 
   uint32_t P = 0u, M = 0u, above = 0u, need = (uint32_t)a.k, bin_cnt = (uint32_t)n, local_eq = 0u;
   int shift = 32;
-  // the slice's first tile is read while the threshold digit is found
-  uint32_t key0[kSelPerThread], valid0;
-  sel_load_tile(src, m, 0, key0, valid0);
   if (a.hist != nullptr) {
-    const uint32_t *hr = a.hist + (int64_t)row * kSelBins;
-    for (int i = tid; i < kSelBins; i += kSelThreads) gh[i] = __ldcg(hr + i);
+    // the leading digit from the indexer's row histogram (read by every CTA of the cluster)
+    const uint4 *hr = reinterpret_cast<const uint4 *>(a.hist + (int64_t)row * kSelBins);
+    static_assert(kSelBins == 4 * kSelThreads, "one 16-byte load per thread");
+    reinterpret_cast<uint4 *>(lh)[tid] = __ldcg(hr + tid);
     __syncthreads();
-    sel_find_bin(gh, kSelBins, need, tmp, &s_bin, &s_above);
+    sel_find_bin(lh, kSelBins, need, tmp, &s_bin, &s_above);
     P = (uint32_t)s_bin << 21;
     M = 0xFFE00000u;
     above = s_above;
     need -= s_above;
-    bin_cnt = gh[s_bin];
+    bin_cnt = lh[s_bin];
     shift = 21;
     __syncthreads();
   }
-  // ------------------------------------------------------------------ counting passes (next digit)
-  int pass = 0;
+  // ------------------------------------------------------------------ counting passes over the slice
 #pragma unroll 1
   while (shift > 0 && (shift == 32 || above + bin_cnt > cap)) {
     const int nbits = shift == 10 ? 10 : 11;
     const int nshift = shift - nbits;
     const int nb = 1 << nbits;
-    uint32_t *h = lh[pass & 1];
-    for (int i = tid; i < nb; i += kSelThreads) h[i] = 0u;
+    for (int i = tid; i < nb; i += kSelThreads) lh[i] = 0u;
     __syncthreads();
-    for (int base = 0; base < m; base += kSelTile) {
-      uint32_t key[kSelPerThread], valid;
-      sel_load_tile(src, m, base, key, valid);
+    SelRaw nxt;
+    if (m > 0) sel_issue(src, m, 0, nxt);
+#pragma unroll 1
+    for (int bb = 0; bb < m; bb += kSelBatch * kSelTile) {
+      const SelRaw cur = nxt;
+      if (bb + kSelBatch * kSelTile < m) sel_issue(src, m, bb + kSelBatch * kSelTile, nxt);
 #pragma unroll
-      for (int e = 0; e < kSelPerThread; ++e)
-        if (((valid >> e) & 1u) && (key[e] & M) == P) atomicAdd(&h[(key[e] >> nshift) & (uint32_t)(nb - 1)], 1u);
-    }
-    __syncthreads();
-    if (C > 1) {
-      tc::cluster_sync();
-      for (int i = tid; i < nb; i += kSelThreads) {
-        uint32_t sum = 0u;
-        for (uint32_t c = 0; c < C; ++c) sum += sel_cl_ld(h + i, c);
-        gh[i] = sum;
+      for (int t = 0; t < kSelBatch; ++t) {
+        uint32_t kc[kSelPerThread], vc;
+        sel_convert(cur, t, m, bb + t * kSelTile, kc, vc);
+#pragma unroll
+        for (int e = 0; e < kSelPerThread; ++e)
+          if (((vc >> e) & 1u) && (kc[e] & M) == P) atomicAdd(&lh[(kc[e] >> nshift) & (uint32_t)(nb - 1)], 1u);
       }
-    } else {
-      for (int i = tid; i < nb; i += kSelThreads) gh[i] = h[i];
     }
     __syncthreads();
+    uint32_t *gh = row_hist(nb);
     sel_find_bin(gh, nb, need, tmp, &s_bin, &s_above);
     P |= (uint32_t)s_bin << nshift;
     M |= (uint32_t)(nb - 1) << nshift;
     above += s_above;
     need -= s_above;
     bin_cnt = gh[s_bin];
-    local_eq = h[s_bin];
+    local_eq = lh[s_bin];
     shift = nshift;
-    ++pass;
-    __syncthreads();
+    release_row_hist(gh, nb);
   }
   const bool full = shift == 0;      // P is the exact threshold key; take `need` of the keys equal to it
 
-  // keys equal to the threshold in lower-ranked slices (full case: they come first in position order)
+  // full case: keys equal to the threshold in the slices before this one come first in position order
   uint32_t eq_before = 0u;
   if (full && C > 1) {
-    if (tid == 0) info[1] = local_eq;
-    tc::cluster_sync();
-    for (uint32_t c = 0; c < r; ++c) eq_before += sel_cl_ld(info + 1, c);
+    if (tid > (int)r && tid < (int)C) sel_cl_st(eq_in + r, (uint32_t)tid, local_eq);
+    sel_cl_arrive();
+    sel_cl_wait();
+    for (uint32_t c = 0; c < r; ++c) eq_before += eq_in[c];
   }
 
   // ------------------------------------------------------------------ storing pass: ordered survivors
   uint32_t stored = 0u;                // survivors written so far (block-uniform)
   if (tid == 0) s_flag = 0u;
-  uint32_t kn[kSelPerThread], vn = 0u;  // the next tile, loaded while this one is compacted
+  {
+    SelRaw nxt;
+    if (m > 0) sel_issue(src, m, 0, nxt);
 #pragma unroll 1
-  for (int base = 0; base < m; base += kSelTile) {
-    uint32_t key[kSelPerThread], valid;
+    for (int bb = 0; bb < m; bb += kSelBatch * kSelTile) {
+      // a batch's tiles come from one set of loads; the next batch's loads go out before its first tile
+      const SelRaw cur = nxt;
+      if (bb + kSelBatch * kSelTile < m) sel_issue(src, m, bb + kSelBatch * kSelTile, nxt);
 #pragma unroll
-    for (int e = 0; e < kSelPerThread; ++e) key[e] = base == 0 ? key0[e] : kn[e];
-    valid = base == 0 ? valid0 : vn;
-    if (base + kSelTile < m) sel_load_tile(src, m, base + kSelTile, kn, vn);
-    uint32_t keep = 0u, eq = 0u;
+    for (int t = 0; t < kSelBatch; ++t) {
+      const int base = bb + t * kSelTile;
+      if (base >= m) break;                     // (m is the same for the whole block)
+      uint32_t kc[kSelPerThread], vc;
+      sel_convert(cur, t, m, base, kc, vc);
+      uint32_t keep = 0u, eq = 0u;
 #pragma unroll
-    for (int e = 0; e < kSelPerThread; ++e) {
-      const uint32_t km = key[e] & M;
-      if ((valid >> e) & 1u) {
-        if (km > P) keep |= 1u << e;
-        else if (km == P) eq |= 1u << e;
+      for (int e = 0; e < kSelPerThread; ++e) {
+        const uint32_t km = kc[e] & M;
+        if ((vc >> e) & 1u) {
+          if (km > P) keep |= 1u << e;
+          else if (km == P) eq |= 1u << e;
+        }
       }
-    }
-    uint32_t pre[kSelPerThread / 4];
-    if (full) {
-      // equal keys taken in position order: the first `need` of the row
-      const uint32_t eq_tot = sel_tile_prefix(eq, pre, tmp);
+      uint32_t pre[kSelPerThread / 4];
+      if (full) {
+        // equal keys taken in position order: the first `need` of the row
+        const uint32_t eq_tot = sel_tile_prefix(eq, pre, tmp);
+#pragma unroll
+        for (int v = 0; v < kSelPerThread / 4; ++v) {
+          uint32_t rank_eq = eq_before + pre[v];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if ((eq >> (4 * v + j)) & 1u) {
+              if (rank_eq < need) keep |= 1u << (4 * v + j);
+              ++rank_eq;
+            }
+        }
+        eq_before += eq_tot;
+        __syncthreads();
+      } else {
+        keep |= eq;
+      }
+      const uint32_t tot = sel_tile_prefix(keep, pre, tmp);
 #pragma unroll
       for (int v = 0; v < kSelPerThread / 4; ++v) {
-        uint32_t rank_eq = eq_before + pre[v];
+        uint32_t off = stored + pre[v];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if ((eq >> (4 * v + j)) & 1u) {
-            if (rank_eq < need) keep |= 1u << (4 * v + j);
-            ++rank_eq;
+          if ((keep >> (4 * v + j)) & 1u) {
+            if (off < cap) {
+              skey[off] = kc[4 * v + j];
+              spos[off] = lo + sel_elem(base, v, j);
+            } else {
+              s_flag = 1u;
+            }
+            ++off;
           }
       }
-      eq_before += eq_tot;
+      stored += tot;
       __syncthreads();
-    } else {
-      keep |= eq;
     }
-    const uint32_t tot = sel_tile_prefix(keep, pre, tmp);
-#pragma unroll
-    for (int v = 0; v < kSelPerThread / 4; ++v) {
-      uint32_t off = stored + pre[v];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if ((keep >> (4 * v + j)) & 1u) {
-          if (off < cap) {
-            skey[off] = key[4 * v + j];
-            spos[off] = lo + sel_elem(base, v, j);
-          } else {
-            s_flag = 1u;
-          }
-          ++off;
-        }
     }
-    stored += tot;
-    __syncthreads();
   }
   if (stored > cap) stored = cap;
-  __syncthreads();
   if (s_flag && tid == 0) set_status(a.status, kStatusBadIndex);
 
-  // ------------------------------------------------------------------ rank 0 collects the cluster's survivors
-  if (C > 1) {
-    if (tid == 0) info[0] = stored;
-    tc::cluster_sync();                          // every slice's survivors are in place
-    if (r == 0) {
-      // the other slices' counts, their offsets after this slice's survivors, then every piece in one round
-      uint32_t *offs = lh[0];                    // (free here) offs[c] = first slot of slice c, offs[C] = end
-      if (tid == 0) {
-        uint32_t total = stored;
-        offs[0] = 0u;
-        for (uint32_t c = 1; c < C; ++c) {
-          const uint32_t cnt = sel_cl_ld(info, c);
-          offs[c] = total;
-          total += cnt;
-        }
-        offs[C] = total;
-        if (total > cap) set_status(a.status, kStatusBadIndex);
-      }
-      __syncthreads();
-      const uint32_t end = min(offs[C], cap);
-      for (uint32_t i = stored + tid; i < end; i += kSelThreads) {
-        uint32_t c = 1;
-        while (c + 1 < C && offs[c + 1] <= i) ++c;
-        const uint32_t j = i - offs[c];
-        uint32_t kv, pv;
-        asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(kv) : "r"(tc::map_to_rank(tc::smem_u32(skey + j), c)) : "memory");
-        asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(pv) : "r"(tc::map_to_rank(tc::smem_u32(spos + j), c)) : "memory");
-        skey[i] = kv;
-        spos[i] = (int32_t)pv;
-      }
-      stored = end;
-    }
-    tc::cluster_sync();                          // rank 0 has read every other slice
-    if (r != 0) return;
-  }
-  __syncthreads();
-
-  // ------------------------------------------------------------------ remaining digits on the survivors
+  // ------------------------------------------------------------------ remaining digits, on the survivors
+  // (a slice's survivors hold every key of its slice in the prefix's bin, so their histograms are the slice's)
 #pragma unroll 1
-  while (shift > 0) {
+  while (shift > 0 && bin_cnt != need) {
     const int nbits = shift == 10 ? 10 : 11;
     const int nshift = shift - nbits;
     const int nb = 1 << nbits;
-    uint32_t *h = lh[0];
-    for (int i = tid; i < nb; i += kSelThreads) h[i] = 0u;
+    for (int i = tid; i < nb; i += kSelThreads) lh[i] = 0u;
     __syncthreads();
     for (uint32_t i = tid; i < stored; i += kSelThreads) {
       const uint32_t kv = skey[i];
-      if ((kv & M) == P) atomicAdd(&h[(kv >> nshift) & (uint32_t)(nb - 1)], 1u);
+      if ((kv & M) == P) atomicAdd(&lh[(kv >> nshift) & (uint32_t)(nb - 1)], 1u);
     }
     __syncthreads();
-    sel_find_bin(h, nb, need, tmp, &s_bin, &s_above);
+    uint32_t *gh = row_hist(nb);
+    sel_find_bin(gh, nb, need, tmp, &s_bin, &s_above);
     P |= (uint32_t)s_bin << nshift;
     M |= (uint32_t)(nb - 1) << nshift;
     above += s_above;
     need -= s_above;
+    bin_cnt = gh[s_bin];
     shift = nshift;
-    __syncthreads();
+    release_row_hist(gh, nb);
   }
-  // P is now the k-th key: emit every survivor above it and the first `need` equal to it, in order
-  // survivors in tiles of 16 warp segments of 256, lane l of a segment holding entries 32 e + l (e = 0..7)
-  uint32_t written = 0u, eq_seen = 0u;
-  const int lane = tid & 31, warp = tid >> 5;
+
+  // ------------------------------------------------------------------ ordered write of the selection
+  // Survivors in tiles of 16 warp segments of 256, lane l of a segment holding entries 32 e + l (e = 0..7):
+  // every survivor above the prefix is taken, and the first `need` of the row equal to it (the slices before
+  // this one first).  A first sweep counts this slice's (above, equal) survivors for the later CTAs.
   const uint32_t lt_mask = (1u << lane) - 1u;
+  uint32_t gt_loc = 0u, eq_loc = 0u;
+  for (uint32_t i = tid; i < stored; i += kSelThreads) {
+    const uint32_t km = skey[i] & M;
+    gt_loc += km > P;
+    eq_loc += km == P;
+  }
+  gt_loc = __reduce_add_sync(0xffffffffu, gt_loc);
+  eq_loc = __reduce_add_sync(0xffffffffu, eq_loc);
+  if (lane == 0) {
+    tmp[warp] = gt_loc;
+    tmp[kSelWarps + warp] = eq_loc;
+  }
+  __syncthreads();
+  uint32_t gt_tot = 0u, eq_tot = 0u;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
+    gt_tot += tmp[w];
+    eq_tot += tmp[kSelWarps + w];
+  }
+  uint32_t out_base = 0u, eq_seen = 0u;
+  if (C > 1) {
+    if (wait_pending) {
+      sel_cl_wait();
+      wait_pending = false;
+    }
+    if (tid > (int)r && tid < (int)C) {
+      sel_cl_st(cnt_in + 2 * r, (uint32_t)tid, gt_tot);
+      sel_cl_st(cnt_in + 2 * r + 1, (uint32_t)tid, eq_tot);
+    }
+    sel_cl_arrive();
+    sel_cl_wait();
+    for (uint32_t c = 0; c < r; ++c) {
+      const uint32_t g = cnt_in[2 * c], e = cnt_in[2 * c + 1];
+      out_base += g + (need > eq_seen ? min(e, need - eq_seen) : 0u);
+      eq_seen += e;
+    }
+  }
+  __syncthreads();
+  uint32_t written = out_base;
 #pragma unroll 1
   for (uint32_t base = 0; base < stored; base += kSelThreads * 8) {
     const uint32_t i0 = base + (uint32_t)warp * 256u + (uint32_t)lane;
@@ -380,16 +502,16 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const uint32_t i = i0 + 32u * e;
-      const uint32_t kv = i < stored ? skey[i] : 0u;
-      gtb[e] = __ballot_sync(0xffffffffu, i < stored && kv > P);
-      eqb[e] = __ballot_sync(0xffffffffu, i < stored && kv == P);
+      const uint32_t km = i < stored ? (skey[i] & M) : 0u;
+      gtb[e] = __ballot_sync(0xffffffffu, i < stored && km > P);
+      eqb[e] = __ballot_sync(0xffffffffu, i < stored && km == P);
       seg_eq += __popc(eqb[e]);
     }
-    // equal keys in position order: the first `need` of all survivors are taken
     if (lane == 0) tmp[warp] = seg_eq;
     __syncthreads();
     uint32_t eq_before_seg = eq_seen, eq_tile = 0u;
-    for (int w = 0; w < kSelThreads / 32; ++w) {
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) {
       eq_before_seg += w < warp ? tmp[w] : 0u;
       eq_tile += tmp[w];
     }
@@ -407,7 +529,8 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
     if (lane == 0) tmp[warp] = seg_sel;
     __syncthreads();
     uint32_t off = written, sel_tile = 0u;
-    for (int w = 0; w < kSelThreads / 32; ++w) {
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) {
       off += w < warp ? tmp[w] : 0u;
       sel_tile += tmp[w];
     }
@@ -422,9 +545,11 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(const SelArg
     written += sel_tile;
     __syncthreads();
   }
-  // a consistent histogram always yields exactly k; pad defensively otherwise
-  for (uint32_t j = written + tid; j < (uint32_t)a.k; j += kSelThreads) out[j] = -1;
-  if (written != (uint32_t)a.k && tid == 0) set_status(a.status, kStatusBadIndex);
+  // a consistent histogram always yields exactly k over the row; the last slice pads defensively otherwise
+  if (r == C - 1) {
+    for (uint32_t j = written + tid; j < (uint32_t)a.k; j += kSelThreads) out[j] = -1;
+    if (written != (uint32_t)a.k && tid == 0) set_status(a.status, kStatusBadIndex);
+  }
 }
 
 // ------------------------------------------------------------------------------------------------ host

@@ -160,6 +160,27 @@ __device__ void find_threshold_bin_w32(const uint32_t *hist, int nbins, uint32_t
   __syncthreads();
 }
 
+// keys[0..len) = the ordered keys of src[0..len) (src 16-byte aligned).  Each thread issues up to kV 16-byte
+// loads before it converts any of them: a load followed at once by its use would cost a memory round trip
+// per vector.
+template <int kV>
+__device__ __forceinline__ void stage_keys(const float *__restrict__ src, int len, uint32_t *keys) {
+  const int l4 = len >> 2, bs = blockDim.x;
+  const float4 *src4 = reinterpret_cast<const float4 *>(src);
+  for (int i0 = threadIdx.x; i0 < l4; i0 += kV * bs) {
+    float4 v[kV];
+#pragma unroll
+    for (int q = 0; q < kV; ++q)
+      if (i0 + q * bs < l4) v[q] = __ldg(src4 + i0 + q * bs);
+#pragma unroll
+    for (int q = 0; q < kV; ++q)
+      if (i0 + q * bs < l4)
+        reinterpret_cast<uint4 *>(keys)[i0 + q * bs] =
+            make_uint4(ordered_key(v[q].x), ordered_key(v[q].y), ordered_key(v[q].z), ordered_key(v[q].w));
+  }
+  for (int i = 4 * l4 + threadIdx.x; i < len; i += bs) keys[i] = ordered_key(__ldg(src + i));
+}
+
 // ------------------------------------------------------------------------------------------------
 // Regime A
 // ------------------------------------------------------------------------------------------------
@@ -203,7 +224,7 @@ constexpr int kTopkSmemFixedU32 = 3 * kRadixBins + 64 + 2 * kTopkMaxCluster;
 // that the receiver waits on: the row histogram of a pass is the sum of the slice histograms' non-zero bins,
 // added into every CTA's copy; the ordered write's offsets come from counts stored into the later CTAs.  No
 // CTA reads a peer's shared memory, so none has to wait for its peers before it exits.
-__global__ void __launch_bounds__(kTopkThreadsA)
+__global__ void __launch_bounds__(kTopkThreadsA, 2)
 topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv, int k,
                       int32_t *__restrict__ idx, TopkWs lw, int register_long) {
   pdl_wait();
@@ -266,15 +287,7 @@ topk_rows_smem_kernel(const float *__restrict__ scores, int64_t ld, BatchView bv
   // this CTA's slice [lo, lo + m): a multiple of 4 keys long, so 16-byte loads stay aligned
   const int slice = ((n + (int)C - 1) / (int)C + 3) & ~3;
   const int lo = min(n, (int)r * slice), m = min(n, lo + slice) - lo;
-  const float *src = scores + (int64_t)row * ld + lo;
-  const int m4 = m >> 2;
-  const float4 *src4 = reinterpret_cast<const float4 *>(src);
-  for (int i = tid; i < m4; i += bs) {
-    float4 v = __ldg(src4 + i);
-    uint4 u = make_uint4(ordered_key(v.x), ordered_key(v.y), ordered_key(v.z), ordered_key(v.w));
-    reinterpret_cast<uint4 *>(keys)[i] = u;
-  }
-  for (int i = 4 * m4 + tid; i < m; i += bs) keys[i] = ordered_key(__ldg(src + i));
+  stage_keys<2>(scores + (int64_t)row * ld + lo, m, keys);
   __syncthreads();
 
   uint32_t prefix = 0u, pmask = 0u, k_rem = (uint32_t)k;
@@ -374,7 +387,7 @@ __device__ __forceinline__ bool long_item(const TopkWs &w, const BatchView &bv, 
   *seg = item % w.max_segs;
   *row = w.list[r_i];
   int b;
-  *n = pos_of_row(bv, *row, &b) + 1;
+  *n = pos_of_row_warp(bv, *row, &b) + 1;
   *nseg = (*n + kTopkSeg - 1) / kTopkSeg;
   return *seg < *nseg;
 }
@@ -383,14 +396,7 @@ __device__ __forceinline__ bool long_item(const TopkWs &w, const BatchView &bv, 
 __device__ int stage_segment(const float *__restrict__ scores, int64_t ld, int row, int seg, int n, uint32_t *keys) {
   const int lo = seg * kTopkSeg;
   const int len = min(kTopkSeg, n - lo);
-  const float *src = scores + (int64_t)row * ld + lo;
-  const int l4 = len >> 2;
-  for (int i = threadIdx.x; i < l4; i += blockDim.x) {
-    float4 v = __ldg(reinterpret_cast<const float4 *>(src) + i);
-    reinterpret_cast<uint4 *>(keys)[i] =
-        make_uint4(ordered_key(v.x), ordered_key(v.y), ordered_key(v.z), ordered_key(v.w));
-  }
-  for (int i = 4 * l4 + threadIdx.x; i < len; i += blockDim.x) keys[i] = ordered_key(__ldg(src + i));
+  stage_keys<4>(scores + (int64_t)row * ld + lo, len, keys);
   __syncthreads();
   return len;
 }

@@ -187,9 +187,14 @@ class DeviceBatch:
     # ten thousand tokens and a single million-token row the two separate calls are faster.
     FUSED_MIN_ROWS = 1024
     FUSED_MIN_LEN = 49153
+    FUSED_LONG_ROW = 262144
 
     def prefers_fused(self):
-        return self.wl.total_q >= self.FUSED_MIN_ROWS and self.wl.max_seq_len >= self.FUSED_MIN_LEN
+        # measured on one B200: the fused call wins for big batches of long rows (the mixed batch: 16.7 ms
+        # against 19.9) and for very long rows (one 1M-token decode row: 74.6 us against 83.9); the two calls
+        # win for decode batches of 4K-32K tokens (38.3 us against 46.2) and the 16k prefill (2.56 ms against 3.48)
+        return (self.wl.total_q >= self.FUSED_MIN_ROWS and self.wl.max_seq_len >= self.FUSED_MIN_LEN) or \
+            self.wl.max_seq_len >= self.FUSED_LONG_ROW
 
     def run(self, stream=None, fused=None):
         """One pass of the path: scores, selection, attention.  fused=True takes scores and selection in one

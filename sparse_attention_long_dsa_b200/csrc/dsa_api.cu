@@ -26,7 +26,8 @@ dsa_status_t indexer_tc_launch(const uint8_t *qI, const float *w, const uint8_t 
 size_t indexer_workspace_bytes(int num_seqs, int total_q);
 size_t indexer_hist_bytes(int total_q);
 dsa_status_t select_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx,
-                           const uint32_t *hist, uint32_t *status, cudaStream_t stream, int num_sms);
+                           const uint32_t *hist, uint32_t *status, void *long_ws, cudaStream_t stream, int num_sms);
+size_t select_long_ws_bytes(int total_q, int max_seq_len);
 dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, int k, float softmax_scale,
                              const dsa_batch_t *b, void *out, float *lse, void *ws, bool decode, cudaStream_t stream,
                              int num_sms);
@@ -153,7 +154,8 @@ static bool is_f32_attn(dsa_dtype_t dt, int H, int Dqk, int Dv, const void *v) {
 
 // the fused scores + selection call: the indexer's workspace, then the rows' leading-digit histograms
 static size_t indexer_topk_ws_bytes(const dsa_batch_t *b) {
-  return indexer_workspace_bytes(b->num_seqs, b->total_q) + indexer_hist_bytes(b->total_q);
+  return indexer_workspace_bytes(b->num_seqs, b->total_q) + indexer_hist_bytes(b->total_q) +
+         select_long_ws_bytes(b->total_q, b->max_seq_len);
 }
 
 static size_t attn_ws_bytes(const dsa_batch_t *b, int k, int H, int Dv, bool decode) {
@@ -278,12 +280,17 @@ dsa_status_t dsa_indexer_topk(const void *q_idx, dsa_dtype_t q_dt, const float *
     st = indexer_tc_launch((const uint8_t *)q_idx, w, (const uint8_t *)k_idx_pool, k_scale_pool, b, scores, ld_scores,
                            ws, (cudaStream_t)stream, dev.num_sms, nullptr, hist);
     if (st != DSA_OK) return st;
-    return select_launch(scores, ld_scores, b, k, idx, hist, (uint32_t *)ws, (cudaStream_t)stream, dev.num_sms);
+    void *long_ws = select_long_ws_bytes(b->total_q, b->max_seq_len) > 0
+                        ? (void *)((char *)hist + indexer_hist_bytes(b->total_q))
+                        : nullptr;
+    return select_launch(scores, ld_scores, b, k, idx, hist, (uint32_t *)ws, long_ws, (cudaStream_t)stream,
+                         dev.num_sms);
   }
   // fp32 indexer (CUDA cores): the selection counts the leading digit itself
   st = indexer_simt_launch(q_idx, q_dt, w, k_idx_pool, k_scale_pool, Hi, Di, b, scores, ld_scores, (cudaStream_t)stream);
   if (st != DSA_OK) return st;
-  return select_launch(scores, ld_scores, b, k, idx, nullptr, (uint32_t *)ws, (cudaStream_t)stream, dev.num_sms);
+  return select_launch(scores, ld_scores, b, k, idx, nullptr, (uint32_t *)ws, nullptr, (cudaStream_t)stream,
+                       dev.num_sms);
 }
 
 dsa_status_t dsa_topk_noalloc(const float *scores, int64_t ld_scores, const dsa_batch_t *b, int32_t k,

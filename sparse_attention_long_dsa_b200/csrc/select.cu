@@ -50,7 +50,27 @@ struct SelArgs {
   const uint32_t *hist;    // [T][2048] leading-digit counts of each row's causal keys, or nullptr
   int cap;                 // survivors a CTA can hold (shared memory)
   uint32_t *status;
+  // survivors already collected by select_gather_kernel (one CTA per row then), or nullptr
+  const uint32_t *surv_key;
+  const int32_t *surv_pos;
+  const uint32_t *surv_cnt;
+  int surv_ctas, surv_q;
 };
+
+// Very long rows (a million-token decode): one cluster of CTAs per row would leave most of the GPU idle, so the
+// survivors are first collected by select_gather_kernel over every SM -- each of G CTAs takes one range of the
+// row and keeps, in position order, the keys whose leading digit is at or above the threshold digit, up to
+// kSelSurvQ of them -- and select_stream_kernel (one CTA per row) goes on from those.
+constexpr int kSelLongRow = 262144;     // rows at least this long (in the batch's longest) take the gather
+constexpr int kSelLongMaxRows = 16;     // ... for batches of at most this many rows
+constexpr int kSelLongCtas = 160;       // gather CTAs over the batch (at most; the workspace is sized for it)
+constexpr int kSelSurvQ = 512;          // survivors one gather CTA keeps (a range holding more: the row is streamed)
+
+size_t select_long_ws_bytes(int total_q, int max_seq_len) {
+  if (max_seq_len < kSelLongRow || total_q > kSelLongMaxRows || total_q < 1) return 0;
+  const size_t slots = (size_t)kSelLongCtas * kSelSurvQ;
+  return (slots * 8 + 255) / 256 * 256 + ((size_t)kSelLongCtas * 4 + 255) / 256 * 256;
+}
 
 // shared memory (u32 words): survivors (key, position) [cap], the slice histogram, two row histograms
 // (alternating passes), scan scratch, the earlier slices' equal-key counts (full case) and final counts
@@ -211,7 +231,101 @@ __device__ __forceinline__ uint32_t sel_tile_prefix(uint32_t flags, uint32_t (&p
   return total;
 }
 
-__global__ void __launch_bounds__(kSelThreads, 2) select_stream_kernel(const SelArgs a) {
+// the row's length: one round of loads for a batch of one query row per sequence (the row is its sequence)
+__device__ __forceinline__ int sel_row_len(const BatchView &bv, int row) {
+  int sc0 = 0, sc1 = 0, ssl = 0;
+  if (row < bv.num_seqs) {
+    sc0 = __ldg(bv.cu_q + row);
+    sc1 = __ldg(bv.cu_q + row + 1);
+    ssl = __ldg(bv.seq_lens + row);
+  }
+  const int b = seq_of_row_warp(bv.cu_q, bv.num_seqs, row);
+  if (b == row) return ssl - (sc1 - sc0) + (row - sc0) + 1;
+  const int c0 = __ldg(bv.cu_q + b), c1 = __ldg(bv.cu_q + b + 1);
+  return __ldg(bv.seq_lens + b) - (c1 - c0) + (row - c0) + 1;
+}
+
+struct GatherArgs {
+  const float *scores;
+  int64_t ld;
+  BatchView bv;
+  int k;
+  const uint32_t *hist;
+  uint32_t *surv_key;      // [T][G][kSelSurvQ]
+  int32_t *surv_pos;
+  uint32_t *surv_cnt;      // [T][G]: survivors of each range (more than kSelSurvQ: not all kept)
+  int G;
+};
+
+__global__ void __launch_bounds__(kSelThreads, 1) select_gather_kernel(const GatherArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ __align__(16) uint32_t lh[kSelBins];
+  __shared__ uint32_t tmp[64];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above;
+  const int row = blockIdx.x / a.G, g = blockIdx.x % a.G;
+  const int tid = threadIdx.x;
+  const int n = sel_row_len(a.bv, row);
+  if (n <= a.k) return;                                    // (the selection writes such rows itself)
+  const int per = ((n + a.G - 1) / a.G + 3) & ~3;
+  const int lo = min(n, g * per), m = min(n, lo + per) - lo;
+  const float *src = a.scores + (int64_t)row * a.ld + lo;
+  // the threshold digit, as the selection will find it
+  const uint4 *hr = reinterpret_cast<const uint4 *>(a.hist + (int64_t)row * kSelBins);
+  reinterpret_cast<uint4 *>(lh)[tid] = __ldcg(hr + tid);
+  __syncthreads();
+  if (tid == 0) {
+    s_bin = 0;
+    s_above = 0u;
+  }
+  sel_find_bin(lh, kSelBins, (uint32_t)a.k, tmp, &s_bin, &s_above);
+  const uint32_t P = (uint32_t)s_bin << 21, M = 0xFFE00000u;
+  uint32_t *sk = a.surv_key + ((int64_t)row * a.G + g) * kSelSurvQ;
+  int32_t *sp = a.surv_pos + ((int64_t)row * a.G + g) * kSelSurvQ;
+  uint32_t stored = 0u;
+  SelRaw nxt;
+  if (m > 0) sel_issue(src, m, 0, nxt);
+#pragma unroll 1
+  for (int bb = 0; bb < m; bb += kSelBatch * kSelTile) {
+    const SelRaw cur = nxt;
+    if (bb + kSelBatch * kSelTile < m) sel_issue(src, m, bb + kSelBatch * kSelTile, nxt);
+#pragma unroll
+    for (int t = 0; t < kSelBatch; ++t) {
+      const int base = bb + t * kSelTile;
+      if (base >= m) break;                                // (m is the same for the whole block)
+      uint32_t kc[kSelPerThread], vc;
+      sel_convert(cur, t, m, base, kc, vc);
+      uint32_t keep = 0u;
+#pragma unroll
+      for (int e = 0; e < kSelPerThread; ++e)
+        if (((vc >> e) & 1u) && (kc[e] & M) >= P) keep |= 1u << e;
+      uint32_t pre[kSelPerThread / 4];
+      const uint32_t tot = sel_tile_prefix(keep, pre, tmp);
+#pragma unroll
+      for (int v = 0; v < kSelPerThread / 4; ++v) {
+        uint32_t off = stored + pre[v];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if ((keep >> (4 * v + j)) & 1u) {
+            if (off < (uint32_t)kSelSurvQ) {
+              sk[off] = kc[4 * v + j];
+              sp[off] = lo + sel_elem(base, v, j);
+            }
+            ++off;
+          }
+      }
+      stored += tot;
+      __syncthreads();
+    }
+  }
+  if (tid == 0) a.surv_cnt[row * a.G + g] = stored;
+}
+
+// kGathered: the survivors may come from select_gather_kernel (an instance of its own, so that the code for it
+// costs the other launches no registers)
+template <bool kGathered>
+__global__ void __launch_bounds__(kSelThreads, kGathered ? 1 : 2) select_stream_kernel(const SelArgs a) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) uint32_t sm[];
@@ -311,9 +425,59 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_stream_kernel(const Sel
     shift = 21;
     __syncthreads();
   }
+  // survivors collected over the whole GPU (one CTA per row here): every range's list, in range order, is the
+  // row's survivors in position order -- when every range kept all of its own and they add up
+  bool gathered = false;
+  uint32_t stored = 0u;                // survivors in shared memory (block-uniform)
+  if (kGathered && a.surv_cnt != nullptr && shift == 21 && above + bin_cnt <= cap) {
+    const int G = a.surv_ctas;
+    const uint32_t c = tid < G ? __ldcg(a.surv_cnt + row * G + tid) : 0u;
+    const bool fits = __syncthreads_and(c <= (uint32_t)a.surv_q) != 0;
+    uint32_t tot;
+    const uint32_t off = block_exclusive_scan(c, tmp, &tot);
+    if (fits && tot == above + bin_cnt) {
+      uint32_t *offs = lh;                     // offs[g]: first survivor of range g in the row's list
+      if (tid < G) offs[tid] = off;
+      __syncthreads();
+      // thread t copies entries t, t + 512, ... of the concatenated lists, finding each entry's range by a binary
+      // search over the offsets; a batch of entries' loads all go out before any is stored
+      constexpr int kCopy = 4;
+      const uint32_t *gk0 = a.surv_key + (int64_t)row * G * a.surv_q;
+      const int32_t *gp0 = a.surv_pos + (int64_t)row * G * a.surv_q;
+      for (uint32_t i0 = tid; i0 < tot; i0 += kCopy * kSelThreads) {
+        uint32_t kv[kCopy];
+        int32_t pv[kCopy];
+#pragma unroll
+        for (int q = 0; q < kCopy; ++q) {
+          const uint32_t i = i0 + q * kSelThreads;
+          if (i < tot) {
+            int lo_g = 0, hi_g = G - 1;              // last range whose offset is <= i
+            while (lo_g < hi_g) {
+              const int mid = (lo_g + hi_g + 1) >> 1;
+              if (offs[mid] <= i) lo_g = mid; else hi_g = mid - 1;
+            }
+            const int64_t src_i = (int64_t)lo_g * a.surv_q + (i - offs[lo_g]);
+            kv[q] = __ldcg(gk0 + src_i);
+            pv[q] = __ldcg(gp0 + src_i);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < kCopy; ++q) {
+          const uint32_t i = i0 + q * kSelThreads;
+          if (i < tot) {
+            skey[i] = kv[q];
+            spos[i] = pv[q];
+          }
+        }
+      }
+      stored = tot;
+      gathered = true;
+    }
+    __syncthreads();
+  }
   // ------------------------------------------------------------------ counting passes over the slice
 #pragma unroll 1
-  while (shift > 0 && (shift == 32 || above + bin_cnt > cap)) {
+  while (!gathered && shift > 0 && (shift == 32 || above + bin_cnt > cap)) {
     const int nbits = shift == 10 ? 10 : 11;
     const int nshift = shift - nbits;
     const int nb = 1 << nbits;
@@ -358,9 +522,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_stream_kernel(const Sel
   }
 
   // ------------------------------------------------------------------ storing pass: ordered survivors
-  uint32_t stored = 0u;                // survivors written so far (block-uniform)
   if (tid == 0) s_flag = 0u;
-  {
+  if (!gathered) {
     SelRaw nxt;
     if (m > 0) sel_issue(src, m, 0, nxt);
 #pragma unroll 1
@@ -578,8 +741,8 @@ static int select_max_cluster(int num_sms) {
   int c = dev >= 0 ? cached[dev].load(std::memory_order_relaxed) : 0;
   if (c > 0) return c;
   const size_t smem = select_smem_bytes(select_cap(16384));
-  cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaFuncSetAttribute(select_stream_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaFuncSetAttribute(select_stream_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   for (c = 16; c > 1; c /= 2) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)c);
@@ -593,7 +756,7 @@ static int select_max_cluster(int num_sms) {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, select_stream_kernel, &cfg) == cudaSuccess && n >= 1) break;
+    if (cudaOccupancyMaxActiveClusters(&n, select_stream_kernel<false>, &cfg) == cudaSuccess && n >= 1) break;
     cudaGetLastError();
   }
   (void)num_sms;
@@ -602,7 +765,7 @@ static int select_max_cluster(int num_sms) {
 }
 
 dsa_status_t select_launch(const float *scores, int64_t ld, const dsa_batch_t *b, int k, int32_t *idx,
-                           const uint32_t *hist, uint32_t *status, cudaStream_t stream, int num_sms) {
+                           const uint32_t *hist, uint32_t *status, void *long_ws, cudaStream_t stream, int num_sms) {
   SelArgs a{};
   a.scores = scores;
   a.ld = ld;
@@ -613,8 +776,32 @@ dsa_status_t select_launch(const float *scores, int64_t ld, const dsa_batch_t *b
   a.cap = select_cap(k);
   a.status = status;
   const size_t smem = select_smem_bytes(a.cap);
-  const int C = std::min(select_cluster(b->total_q, b->max_seq_len, num_sms), select_max_cluster(num_sms));
-  cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  int C = std::min(select_cluster(b->total_q, b->max_seq_len, num_sms), select_max_cluster(num_sms));
+  if (hist != nullptr && long_ws != nullptr && select_long_ws_bytes(b->total_q, b->max_seq_len) > 0) {
+    // very long rows: the survivors are collected over every SM first, then one CTA per row goes on
+    GatherArgs ga{};
+    ga.scores = scores;
+    ga.ld = ld;
+    ga.bv = a.bv;
+    ga.k = k;
+    ga.hist = hist;
+    ga.G = std::max(1, std::min(num_sms, kSelLongCtas) / b->total_q);
+    const size_t slots = (size_t)kSelLongCtas * kSelSurvQ;
+    ga.surv_key = (uint32_t *)long_ws;
+    ga.surv_pos = (int32_t *)((uint32_t *)long_ws + slots);
+    ga.surv_cnt = (uint32_t *)((char *)long_ws + (slots * 8 + 255) / 256 * 256);
+    DSA_LAUNCH_PDL("select_gather_kernel", select_gather_kernel, dim3(b->total_q * ga.G), dim3(kSelThreads), 0, stream,
+                   ga);
+    a.surv_key = ga.surv_key;
+    a.surv_pos = ga.surv_pos;
+    a.surv_cnt = ga.surv_cnt;
+    a.surv_ctas = ga.G;
+    a.surv_q = kSelSurvQ;
+    C = 1;
+  }
+  const bool gathered = a.surv_cnt != nullptr;
+  cudaFuncSetAttribute(gathered ? select_stream_kernel<true> : select_stream_kernel<false>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(b->total_q * C));
   cfg.blockDim = dim3(kSelThreads);
@@ -629,7 +816,8 @@ dsa_status_t select_launch(const float *scores, int64_t ld, const dsa_batch_t *b
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t le = cudaLaunchKernelEx(&cfg, select_stream_kernel, a);
+  const cudaError_t le = gathered ? cudaLaunchKernelEx(&cfg, select_stream_kernel<true>, a)
+                                  : cudaLaunchKernelEx(&cfg, select_stream_kernel<false>, a);
   if (le != cudaSuccess) {
     set_error("select_stream_kernel: %s", cudaGetErrorString(le));
     return DSA_ERR_CUDA;

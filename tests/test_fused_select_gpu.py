@@ -119,3 +119,40 @@ def test_fused_mixed_batch_full_size_grid():
     _check_rows_vs_oracle(wl, db, rows)
     # every row against dsa_topk over the same scores
     assert torch.equal(db.idx, _separate_idx(db))
+
+
+def test_fused_long_rows_gather_matches_separate_calls():
+    """Rows of 256K candidates or more in a batch of at most 16 rows: the survivors are collected over every SM
+    (one range per CTA) before one CTA per row finishes the selection."""
+    wl = W.make_workload("fused_long", kind="mla", seed=208, seq_lens=[300000, 270000, 5000], q_lens=[1, 1, 1],
+                         topk=2048, attention=False)
+    db = _fused(wl)
+    assert torch.equal(db.idx, _separate_idx(db))
+
+
+def test_fused_long_row_with_clustered_top_keys():
+    """A 300,000-token row whose 2048 best keys sit at its start: a gathering range keeps at most a fixed number
+    of survivors, so the range holding them overflows and the selection streams the row itself."""
+    wl = W.make_workload("fused_cluster", kind="mla", seed=207, seq_lens=[300000], q_lens=[1], topk=2048,
+                         planted_k=2048, attention=False)
+    n, P = 300000, wl.kI_pool.shape[1]
+    pos = np.arange(n)
+    phys = wl.block_table[0, pos // P].astype(np.int64) * P + pos % P
+    order = np.concatenate([wl.planted, np.setdiff1d(pos, wl.planted)])     # planted keys first
+    kflat = wl.kI_pool.reshape(-1, wl.kI_pool.shape[-1])
+    kflat[phys] = kflat[phys][order]
+    sflat = wl.kS_pool.reshape(-1)
+    sflat[phys] = sflat[phys][order]
+    db = _fused(wl)
+    assert np.array_equal(db.idx[0].cpu().numpy(), np.arange(2048))
+    assert torch.equal(db.idx, _separate_idx(db))
+
+
+def test_fused_long_row_all_equal_scores():
+    """Every score 0 on a 300,000-token row: the threshold bin holds the whole row, past the survivor capacity,
+    so the gathered survivors are not used and the selection resolves every key bit by counting passes."""
+    wl = W.make_workload("fused_long_ties", kind="mla", seed=209, seq_lens=[300000], q_lens=[1], topk=2048,
+                         attention=False)
+    wl.w = np.zeros_like(wl.w)
+    db = _fused(wl)
+    assert np.array_equal(db.idx[0].cpu().numpy(), np.arange(2048))

@@ -688,9 +688,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttThreads, 1)
 
 // ------------------------------------------------------------------------------------------------ combine
 // out[row, h, :] = sum_s exp(lse_s - lse) o_s,  lse = log sum_s exp(lse_s)   (splits of one row)
-// The splits' lse values and partial outputs (up to kCombineRegSplits of each) are loaded in one round; a split
-// with lse = -inf wrote zeros and gets weight 0.  More splits are re-read in a second loop.
+// Up to kCombineRegSplits splits: their lse values and partial outputs are loaded in one round.  More splits (a
+// single long row spread over many CTA pairs): every split's lse goes to shared memory (one load per thread)
+// and the partial outputs come in batches of kCombineRegSplits, each batch's loads issued before the previous
+// batch is summed.  Either way the sums run over the splits in order; a split with lse = -inf wrote zeros and
+// gets weight 0.
 constexpr int kCombineRegSplits = 8;
+constexpr int kCombineMaxSplits = 128;           // >= the largest split count (74 CTA pairs)
+__device__ __forceinline__ void combine_issue(const float *po, int splits, int s0, float4 (&o)[kCombineRegSplits]) {
+#pragma unroll
+  for (int j = 0; j < kCombineRegSplits; ++j)
+    o[j] = s0 + j < splits ? __ldg(reinterpret_cast<const float4 *>(po + (int64_t)(s0 + j) * kAttH * kAttDv))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+__global__ void __launch_bounds__(128) attn_combine_many_kernel(const float *__restrict__ part_o,
+                                                                const float *__restrict__ part_lse, int splits,
+                                                                __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+  __shared__ float s_l[kCombineMaxSplits];
+  pdl_wait();
+  pdl_trigger();
+  const int row = blockIdx.x, h = blockIdx.y;
+  const float *pl = part_lse + (int64_t)row * splits * kAttH + h;
+  const int dv = threadIdx.x * 4;
+  const float *po = part_o + ((int64_t)row * splits * kAttH + h) * kAttDv + dv;
+  {
+    float4 nxt[kCombineRegSplits];
+    combine_issue(po, splits, 0, nxt);
+    for (int s = threadIdx.x; s < splits; s += blockDim.x) s_l[s] = __ldg(pl + (int64_t)s * kAttH);
+    __syncthreads();
+    float mx = -INFINITY;
+    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, s_l[s]);
+    float tot = 0.f;
+    for (int s = 0; s < splits; ++s) tot += s_l[s] == -INFINITY ? 0.f : __expf(s_l[s] - mx);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tot > 0.f) {
+      for (int s0 = 0; s0 < splits; s0 += kCombineRegSplits) {
+        float4 cur[kCombineRegSplits];
+#pragma unroll
+        for (int j = 0; j < kCombineRegSplits; ++j) cur[j] = nxt[j];
+        if (s0 + kCombineRegSplits < splits) combine_issue(po, splits, s0 + kCombineRegSplits, nxt);
+#pragma unroll
+        for (int j = 0; j < kCombineRegSplits; ++j) {
+          const int s = s0 + j;
+          if (s >= splits || s_l[s] == -INFINITY) continue;
+          const float wgt = __expf(s_l[s] - mx) / tot;
+          acc.x += wgt * cur[j].x;
+          acc.y += wgt * cur[j].y;
+          acc.z += wgt * cur[j].z;
+          acc.w += wgt * cur[j].w;
+        }
+      }
+    }
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x, acc.y), b1 = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 w;
+    w.x = *reinterpret_cast<uint32_t *>(&b0);
+    w.y = *reinterpret_cast<uint32_t *>(&b1);
+    *reinterpret_cast<uint2 *>(out + ((int64_t)row * kAttH + h) * kAttDv + dv) = w;
+    if (lse && threadIdx.x == 0) lse[(int64_t)row * kAttH + h] = tot > 0.f ? mx + __logf(tot) : -INFINITY;
+  }
+}
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restrict__ part_o,
                                                            const float *__restrict__ part_lse, int splits,
                                                            __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
@@ -860,8 +916,14 @@ dsa_status_t attn_mla_launch(const void *q, const void *kv, const int32_t *idx, 
   const int pairs = std::min(max_pairs, units);
   DSA_LAUNCH_PDL("attn_mla_kernel", attn_mla_kernel, dim3(2 * pairs), dim3(kAttThreads), smem, stream, tm_q, tm_kv, a);
   if (a.splits > 1) {
-    DSA_LAUNCH_PDL("attn_combine_kernel", attn_combine_kernel, dim3(a.T, kAttH), dim3(128), 0, stream,
-                   (const float *)a.part_o, (const float *)a.part_lse, a.splits, (__nv_bfloat16 *)out, lse);
+    if (a.splits <= kCombineRegSplits) {
+      DSA_LAUNCH_PDL("attn_combine_kernel", attn_combine_kernel, dim3(a.T, kAttH), dim3(128), 0, stream,
+                     (const float *)a.part_o, (const float *)a.part_lse, a.splits, (__nv_bfloat16 *)out, lse);
+    } else {
+      static_assert(kAttPairsForSplits <= kCombineMaxSplits, "every split's lse fits in shared memory");
+      DSA_LAUNCH_PDL("attn_combine_many_kernel", attn_combine_many_kernel, dim3(a.T, kAttH), dim3(128), 0, stream,
+                     (const float *)a.part_o, (const float *)a.part_lse, a.splits, (__nv_bfloat16 *)out, lse);
+    }
   }
   return DSA_OK;
 }

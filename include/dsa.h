@@ -160,9 +160,11 @@ DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, const dsa_
  * order-preserving key per row (a 2048-bin histogram in the workspace), so the selection starts from the
  * threshold digit and reads each row's scores once, keeping only the keys at or above it.  The f32 indexer
  * takes the same selection kernel, which then counts the leading digit itself first.
- * Workspace: dsa_workspace_size(DSA_OP_INDEXER_TOPK) (the indexer's plus 8 KB per query row); its status
- * word also reports a selection that ran past its shared-memory capacity (DSA_ERR_DEVICE_CHECK; cannot
- * happen with a histogram written by this call). */
+ * Batches of at most 16 rows whose longest row has 262,144 candidates or more first gather each row's
+ * survivors (keys at or above the threshold digit) over all SMs, then finish one row per CTA.
+ * Workspace: dsa_workspace_size(DSA_OP_INDEXER_TOPK) (the indexer's plus 8 KB per query row, plus 640 KB of
+ * survivor slots for such long-row batches); its status word also reports a selection that ran past its
+ * shared-memory capacity (DSA_ERR_DEVICE_CHECK; cannot happen with a histogram written by this call). */
 DSA_API dsa_status_t dsa_indexer_topk(const void *q_idx, dsa_dtype_t q_dt, const float *w, const void *k_idx_pool,
                                       dsa_dtype_t k_dt, const float *k_scale_pool, int32_t Hi, int32_t Di,
                                       const dsa_batch_t *b, int32_t k, float *scores, int64_t ld_scores, int32_t *idx,

@@ -253,3 +253,17 @@ def test_fused_append_validates_before_launch():
             B.dsa_indexer_scores_append(a["kv_new"], BF, a["k_new"], a["k_new_dt"], a["kv_pool"], P, F8, P, P, F8, P,
                                         a["Hi"], 128, b, P, a["ld"], P, a["ws_bytes"], 0)
         assert e.value.status == status, over
+
+
+def test_fused_selection_workspace_holds_the_gather_buffers_for_long_rows():
+    """dsa_indexer_topk on a batch of at most 16 rows whose longest row has 262,144 candidates or more also
+    gathers each row's survivors over the SMs first: its workspace then holds 160 slots of 512 (key, position)
+    pairs and their counts, and only then."""
+    gather = 160 * 512 * 8 + 768            # pairs (256-byte rounded) + 160 counts (rounded to 768)
+    def ws(total_q, max_seq_len):
+        b = _batch(num_seqs=total_q, total_q=total_q, max_q_per_seq=1, max_seq_len=max_seq_len,
+                   max_blocks_per_seq=(max_seq_len + 63) // 64)
+        return B.dsa_workspace_size(B.DSA_OP_INDEXER_TOPK, b, 2048)
+    assert ws(1, 262144) - ws(1, 262143) == gather
+    assert ws(16, 1 << 20) - ws(16, 262143) == gather
+    assert ws(17, 1 << 20) == ws(17, 262143)               # more rows: one cluster per row, no gather

@@ -22,7 +22,8 @@
 // survivors the same way (stopping as soon as the prefix's bin holds exactly the keys still needed); then each
 // slice writes its selected positions, offset by the counts of the slices before it, stored into the later
 // CTAs before a barrier.  No CTA reads another's shared memory.  Without a histogram (plain scores) the first
-// counting pass fixes the leading digit.
+// counting pass fixes the leading digit.  Very long rows in small batches collect their survivors over every SM
+// first (select_gather_kernel, below), and one CTA per row goes on from them.
 #include <algorithm>
 #include <atomic>
 #include <cstdio>
@@ -658,6 +659,15 @@ __global__ void __launch_bounds__(kSelThreads, kGathered ? 1 : 2) select_stream_
   }
   __syncthreads();
   uint32_t written = out_base;
+  // every key of the prefix's bin is taken (the usual end of the digit passes): when every survivor of this slice
+  // is above or in the bin, the survivors are the slice's output as they stand, in position order
+  const bool all_eq = bin_cnt == need;
+  if (all_eq && gt_tot + eq_tot == stored) {
+    for (uint32_t i = tid; i < stored; i += kSelThreads)
+      if (out_base + i < (uint32_t)a.k) out[out_base + i] = spos[i];
+    written = out_base + stored;
+    stored = 0u;                                        // (nothing left for the general write below)
+  }
 #pragma unroll 1
   for (uint32_t base = 0; base < stored; base += kSelThreads * 8) {
     const uint32_t i0 = base + (uint32_t)warp * 256u + (uint32_t)lane;

@@ -154,9 +154,11 @@ __global__ void __launch_bounds__(kAttPlanThreads) attn_plan_kernel(const int32_
   pdl_wait();
   pdl_trigger();
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int b;
-  pos_of_row(bv, row, &b);
-  const int seq_len = __ldg(bv.seq_lens + b);
+  // the row's sequence length: the warp-wide search, with the entry of sequence `row` loaded beside it (a batch
+  // of one query row per sequence, where the row is its sequence, needs no second round)
+  const int spec = row < bv.num_seqs ? __ldg(bv.seq_lens + row) : 0;
+  const int b = seq_of_row_warp(bv.cu_q, bv.num_seqs, row);
+  const int seq_len = b == row ? spec : __ldg(bv.seq_lens + b);
   int last = -1;
   bool bad = false;
   const int32_t *ir = idx + (int64_t)row * k;

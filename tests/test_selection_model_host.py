@@ -11,8 +11,9 @@ each slice then writes every survivor above the prefix and the row's first `need
 counts of the slices before it.  The GPU tests check the kernel itself against the oracle; this checks that the
 steps compose to the top-k's definition (score descending, position ascending; -0 == +0) under ties, all-equal
 rows, signed zeros, tiny magnitudes, keys that differ only in their last bits, small capacities that force every
-counting pass, and 1 to 16 slices.  (Dropping the last digit pass, taking one equal key too many or halving a
-digit's bins each fail it.)
+counting pass, and 1 to 16 slices.  (Dropping the last digit pass, taking one equal key too many, halving a
+digit's bins or offsetting a slice by all of the earlier slices' equal keys each fail it.)  The decode top-k
+(`topk_rows_smem_kernel`) is checked the same way.
 """
 import numpy as np
 import pytest
@@ -102,6 +103,8 @@ def _rows(seed):
     for n in (5, 100, 2049, 3000, 9000, 20000):
         yield rng.standard_normal(n).astype(np.float32)
         yield rng.integers(-3, 4, n).astype(np.float32)                 # heavy ties
+        yield rng.integers(0, n // 300 + 2, n).astype(np.float32)       # ~300 keys per level: a tied threshold
+                                                                         # with keys above it in every slice
         yield np.zeros(n, np.float32)                                    # all equal
         z = np.zeros(n, np.float32)
         z[::2] = -0.0                                                    # signed zeros tie
@@ -121,3 +124,50 @@ def test_selection_steps_reproduce_the_topk_definition(k):
         got = _select(s, k, C, cap, use_hist=bool(t % 2))
         exp = oracle.topk_row(s.astype(np.float64), k)
         assert np.array_equal(got, exp), f"case {t}: n={s.size} k={k} C={C} cap={cap}"
+
+
+def _topk_slices(scores, k, C):
+    """The steps of `topk_rows_smem_kernel` (a row in C slices of a cluster): 11-, 11- and 10-bit digits, each
+    chosen from the sum of the slices' histograms of the keys matching the prefix; the passes stop as soon as the
+    threshold bin holds exactly the keys still needed, and the keys are then compared on the digits fixed so far;
+    each slice writes its keys above the threshold and its share of the row's first keys equal to it, in position
+    order, offset by the slices before it."""
+    n = scores.size
+    keys = _okey(scores)
+    if n <= k:
+        return np.array([j if j < n else -1 for j in range(k)], np.int32)
+    per = ((n + C - 1) // C + 3) & ~3
+    slices = [(min(n, r * per), min(n, min(n, r * per) + per)) for r in range(C)]
+    prefix = pmask = 0
+    k_rem = k
+    for shift, nb in ((21, 2048), (10, 2048), (0, 1024)):
+        hist = sum(np.bincount(((keys[lo:hi][(keys[lo:hi] & pmask) == prefix] >> shift) & (nb - 1)).astype(np.int64),
+                               minlength=nb) for lo, hi in slices)
+        d, ab = _find_bin(hist, k_rem)
+        prefix, pmask, k_rem = prefix | (d << shift), pmask | ((nb - 1) << shift), k_rem - ab
+        if hist[d] == k_rem:
+            break
+    out = np.full(k, -1, np.int32)
+    counts = [(int(((keys[lo:hi] & pmask) > prefix).sum()), int(((keys[lo:hi] & pmask) == prefix).sum()))
+              for lo, hi in slices]
+    for r, (lo, hi) in enumerate(slices):
+        out_base = eq_base = 0
+        for g, e in counts[:r]:
+            out_base += g + (min(e, k_rem - eq_base) if k_rem > eq_base else 0)
+            eq_base += e
+        km = keys[lo:hi] & pmask
+        eq = km == prefix
+        take = (km > prefix) | (eq & (eq_base + np.cumsum(eq) - 1 < k_rem))
+        sel = np.arange(lo, hi)[take]
+        out[out_base: out_base + sel.size] = sel[: max(0, k - out_base)]
+    return out
+
+
+@pytest.mark.parametrize("k", [1, 7, 100, 2048])
+def test_topk_slice_steps_reproduce_the_topk_definition(k):
+    rng = np.random.default_rng(2000 + k)
+    for t, s in enumerate(_rows(k + 1)):
+        C = int(rng.choice([1, 2, 4, 8]))
+        got = _topk_slices(s, k, C)
+        exp = oracle.topk_row(s.astype(np.float64), k)
+        assert np.array_equal(got, exp), f"case {t}: n={s.size} k={k} C={C}"

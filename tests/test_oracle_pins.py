@@ -543,3 +543,20 @@ def test_reuse_of_the_same_step_is_idempotent():
         cands = oracle.reuse_candidates(sel, pos + 1, pos)
         got = oracle.candidate_topk(oracle.candidate_scores_row(wl, row, cands), cands, 16)
         assert np.array_equal(np.sort(got[got >= 0]), sel[sel >= 0])
+
+
+def test_reuse_empty_slots_score_minus_infinity_and_are_never_chosen():
+    """An earlier selection's -1 slots carry no token: they score -inf, so even when every real candidate
+    scores below zero (a negative indexer weight) none of them is passed over for an empty slot."""
+    # one head, one active dim, weight -1: token s has key (s + 1, 0), so I[s] = -ReLU(s + 1) = -(s + 1)
+    case = _single_row_case(qI=[[1.0, 0.0]], kI=[[s + 1.0, 0.0] for s in range(6)], w=[-1.0])
+    assert oracle.indexer_scores_row(case, 0).tolist() == [-1.0, -2.0, -3.0, -4.0, -5.0, -6.0]
+    # an earlier selection {0, 2} with two empty slots, made at 4 tokens; the query sits at position 5
+    cands = oracle.reuse_candidates(np.array([0, 2, -1, -1]), 4, 5)
+    assert cands.tolist() == [0, 2, -1, -1, 4, 5]
+    sc = oracle.candidate_scores_row(case, 0, cands)
+    assert sc.tolist() == [-1.0, -3.0, -np.inf, -np.inf, -5.0, -6.0]
+    # k = 4: the four real candidates, in slot order
+    assert oracle.candidate_topk(sc, cands, 4).tolist() == [0, 2, 4, 5]
+    # k = 3: the three best (-1, -3, -5)
+    assert oracle.candidate_topk(sc, cands, 3).tolist() == [0, 2, 4]

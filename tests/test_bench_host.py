@@ -38,3 +38,40 @@ def test_step_roofline_tensor_and_hbm_bound():
     work["attention"]["bytes"] = 29e9
     r = bench.step_roofline(work, peaks, 60.0)
     assert r["bound"] == "hbm" and r["t_roof_us"] == pytest.approx(30e3) and r["frac"] == pytest.approx(0.5)
+
+
+def _csrc_copy(tmp_path, edit=None):
+    """A copy of the attention kernel's sources under tmp_path (laid out like the package), one file edited."""
+    import shutil
+    d = tmp_path / "sparse_attention_long_dsa_b200" / "csrc"
+    d.mkdir(parents=True)
+    src = os.path.join(bench.ROOT, "sparse_attention_long_dsa_b200", "csrc")
+    for f in ("attn_mla_tc.cu", "tc.cuh", "common.cuh"):
+        shutil.copy(os.path.join(src, f), d / f)
+    if edit is not None:
+        f, old, new = edit
+        text = (d / f).read_text()
+        assert text.count(old) == 1, old
+        (d / f).write_text(text.replace(old, new))
+    return str(tmp_path)
+
+
+@pytest.mark.parametrize("edit,kept", [
+    (None, True),
+    # the combine kernels and their launch, and the plan kernel, are launches of their own
+    (("attn_mla_tc.cu", "constexpr int kCombineRegSplits = 8;", "constexpr int kCombineRegSplits = 4;"), True),
+    (("attn_mla_tc.cu", "constexpr int kAttPlanThreads = 256;", "constexpr int kAttPlanThreads = 128;"), True),
+    # the kernel's declarations, its body, its launch and the shared headers decide its traffic
+    (("attn_mla_tc.cu", "constexpr int kAttNBuf = 3;", "constexpr int kAttNBuf = 2;"), False),
+    (("attn_mla_tc.cu", "const int pairs = std::min(max_pairs, units);", "const int pairs = max_pairs;"), False),
+    (("attn_mla_tc.cu", "// ------------------------------------------------------------------------------------------------ main",
+      "// main"), False),                                                            # a marker gone
+])
+def test_measured_traffic_follows_the_captured_kernel(tmp_path, monkeypatch, edit, kept):
+    rec = bench.MEASURED_TRAFFIC[("attention", "decode_batch")]
+    assert bench.measured_traffic("attention", "decode_batch") in (rec["bytes"], None)
+    base = bench.traffic_key(rec["regions"])
+    monkeypatch.setattr(bench, "ROOT", _csrc_copy(tmp_path, edit))
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, ("attention", "decode_batch"), dict(rec, sha256_16=base))
+    assert (bench.measured_traffic("attention", "decode_batch") == rec["bytes"]) == kept
+    assert bench.measured_traffic("attention", "prefill_16k") is None                # no capture recorded

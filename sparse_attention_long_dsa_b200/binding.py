@@ -108,10 +108,19 @@ def _check(status: int, where: str):
 
 
 def _ptr(t) -> Optional[int]:
+    """Address of a tensor's data, or an integer address passed through.  A tensor must be a dense CUDA tensor:
+    the kernels read and write its bytes in the layout include/dsa.h gives, so a host tensor would hand them a
+    host address and a strided view would be read as if it were dense."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise DSAError(DSA_ERR_INVALID_ARG, "argument",
+                       f"a {tuple(t.shape)} tensor on {t.device}; the library takes device memory")
+    if not t.is_contiguous():
+        raise DSAError(DSA_ERR_INVALID_ARG, "argument",
+                       f"a strided {tuple(t.shape)} tensor (strides {tuple(t.stride())}); the library takes dense arrays")
     return t.data_ptr()
 
 

@@ -267,3 +267,29 @@ def test_fused_selection_workspace_holds_the_gather_buffers_for_long_rows():
     assert ws(1, 262144) - ws(1, 262143) == gather
     assert ws(16, 1 << 20) - ws(16, 262143) == gather
     assert ws(17, 1 << 20) == ws(17, 262143)               # more rows: one cluster per row, no gather
+
+
+def test_binding_rejects_host_and_strided_tensors_before_the_library():
+    """A host tensor would give the kernels a host address and a strided view would be read as dense: the
+    binding refuses both before anything reaches the library (nothing is launched)."""
+    import torch
+    b = _batch()
+    n0 = B.dsa_launch_count()
+    with pytest.raises(B.DSAError, match="device memory") as e:
+        B.dsa_topk(torch.zeros(4, 128), 128, b, 16, 1 << 20, 1 << 21, 1 << 20, 0)
+    assert e.value.status == B.DSA_ERR_INVALID_ARG
+
+    class _StridedCuda:                                   # stands in for a CUDA view (no device here)
+        is_cuda = True
+        shape = (4, 128)
+
+        def is_contiguous(self):
+            return False
+
+        def stride(self):
+            return (1, 4)
+
+    with pytest.raises(B.DSAError, match="dense") as e:
+        B.dsa_topk(_StridedCuda(), 128, b, 16, 1 << 20, 1 << 21, 1 << 20, 0)
+    assert e.value.status == B.DSA_ERR_INVALID_ARG
+    assert B.dsa_launch_count() == n0

@@ -170,7 +170,9 @@ DSA_API dsa_status_t dsa_indexer_topk(const void *q_idx, dsa_dtype_t q_dt, const
                                       const dsa_batch_t *b, int32_t k, float *scores, int64_t ld_scores, int32_t *idx,
                                       void *ws, size_t ws_bytes, void *stream);
 
-/* Allocation-free top-k.  There is no counterpart in the pages: this entry point exists for callers
+/* Allocation-free top-k: the selection of dsa_topk ("Day-0 Adaptation for LLMs ...", III.1: top-k over
+ * long sequences; decode sketch idx = topk(score, k)) with arguments and output as there, but no
+ * workspace.  The source pages have no allocation-free variant; this entry point exists for callers
  * that cannot allocate device memory for a workspace -- code that runs where cudaMalloc is not allowed
  * or not wanted (a plugin or custom operator handed only a stream, a framework whose memory is owned
  * by its own pool, a latency-critical path that must not trigger an allocation and its implicit device

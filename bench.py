@@ -172,6 +172,49 @@ def slowest_rank_ms(ms, world, device):
     return ms
 
 
+# a timed region whose clock record shows one of these is not a valid number: it is measured once more
+REJECTED_CLOCK_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+# reasons that explain an SM clock below its maximum (kept, noted in the record)
+POWER_CLOCK_REASONS = ("sw_power_cap", "hw_power_brake_slowdown")
+
+
+def clocks_rejected(clocks):
+    """Whether a timed region's clock record invalidates its number: a hardware or thermal slowdown was active,
+    or the median SM clock sat below 80 % of its maximum with no power-cap reason to explain it (a clock left
+    locked).  A missing record (no NVML) rejects nothing."""
+    if not clocks or clocks.get("sm_mhz") is None:
+        return False
+    reasons = clocks.get("reasons") or []
+    if any(r in REJECTED_CLOCK_REASONS for r in reasons):
+        return True
+    mx = clocks.get("sm_max_mhz")
+    return bool(mx) and clocks["sm_mhz"] < 0.8 * mx and not any(r in POWER_CLOCK_REASONS for r in reasons)
+
+
+def any_rank(flag, world, device):
+    """True on every rank when it is true on one (MAX all-reduce; a no-op on one rank), so that all ranks take
+    the same timed regions."""
+    if world > 1:
+        import torch
+        t = torch.tensor([1.0 if flag else 0.0], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return bool(t.item() > 0)
+    return bool(flag)
+
+
+def _time_steps_checked(replicas, stream, steps, warmup, world, dev, sampler, selection):
+    """_time_steps, measured once more when the clock record of the timed region rejects it (on any rank); the
+    record then keeps the first region's clocks under `rejected_first`."""
+    res = _time_steps(replicas, stream, steps, warmup, world, dev, sampler, selection)
+    if any_rank(clocks_rejected(res[3]), world, dev):
+        first = res[3]
+        res = _time_steps(replicas, stream, steps, warmup, world, dev, sampler, selection)
+        clocks = dict(res[3] or {})
+        clocks["rejected_first"] = first
+        res = (res[0], res[1], res[2], clocks)
+    return res
+
+
 def job_tokens_per_s(tokens_per_rank_step, world, ms_per_step):
     """Whole-job throughput under weak scaling: every rank processes its own batch of the same shape."""
     return world * tokens_per_rank_step / (ms_per_step / 1e3)
@@ -341,7 +384,7 @@ def run_extra_workload(name, args, dev, stream, sampler):
     # enough steps for a timed region of about 0.2 s (clock samples under load), at least --extra-steps
     probe_ms, _, _, _ = _time_steps([db], stream, 1, args.warmup, 1, dev, None, args.selection)
     steps = int(min(2000, max(args.extra_steps, math.ceil(200.0 / max(probe_ms, 1e-3)))))
-    total_ms, stage_avg, launches, clocks = _time_steps([db], stream, steps, 1, 1, dev, sampler, args.selection)
+    total_ms, stage_avg, launches, clocks = _time_steps_checked([db], stream, steps, 1, 1, dev, sampler, args.selection)
     ms_per_step = total_ms / steps
     peaks, peak_src = load_peaks()
     decode = bool(np.all(wl.q_lens == 1))
@@ -396,8 +439,8 @@ def run_ours(args, rank, world, local_rank):
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    total_ms, stage_avg, launches, clocks = _time_steps(replicas, stream, args.steps, args.warmup, world, dev, sampler,
-                                                        args.selection)
+    total_ms, stage_avg, launches, clocks = _time_steps_checked(replicas, stream, args.steps, args.warmup, world, dev,
+                                                                sampler, args.selection)
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(work["tokens"], world, ms_per_step)
 

@@ -75,3 +75,39 @@ def test_measured_traffic_follows_the_captured_kernel(tmp_path, monkeypatch, edi
     monkeypatch.setitem(bench.MEASURED_TRAFFIC, ("attention", "decode_batch"), dict(rec, sha256_16=base))
     assert (bench.measured_traffic("attention", "decode_batch") == rec["bytes"]) == kept
     assert bench.measured_traffic("attention", "prefill_16k") is None                # no capture recorded
+
+
+@pytest.mark.parametrize("clocks,rejected", [
+    (None, False),                                                                   # no NVML: nothing to judge
+    ({"sm_mhz": None, "sm_max_mhz": 1965, "reasons": []}, False),
+    ({"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": []}, False),
+    ({"sm_mhz": 1330.0, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]}, False),     # power cap: kept, noted
+    ({"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": ["hw_slowdown"]}, True),
+    ({"sm_mhz": 1800.0, "sm_max_mhz": 1965, "reasons": ["sw_thermal_slowdown"]}, True),
+    ({"sm_mhz": 1500.0, "sm_max_mhz": 1965, "reasons": ["sw_power_cap", "hw_thermal_slowdown"]}, True),
+    ({"sm_mhz": 1100.0, "sm_max_mhz": 1965, "reasons": []}, True),                   # well below max, no reason
+    ({"sm_mhz": 1700.0, "sm_max_mhz": 1965, "reasons": []}, False),
+])
+def test_clock_record_rejection(clocks, rejected):
+    assert bench.clocks_rejected(clocks) == rejected
+
+
+def test_rejected_timed_region_is_measured_once_more(monkeypatch):
+    records = [{"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": ["hw_slowdown"]},
+               {"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": ["hw_slowdown"]},
+               {"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": []}]
+    calls = []
+
+    def fake(replicas, stream, steps, warmup, world, dev, sampler, selection):
+        calls.append(len(calls))
+        return 10.0 + len(calls), {"attention": 1.0}, 6, records[len(calls) - 1]
+
+    monkeypatch.setattr(bench, "_time_steps", fake)
+    ms, stages, launches, clocks = bench._time_steps_checked(None, None, 1, 3, 1, "cpu", None, "auto")
+    # once more, not more: the second region is reported (still rejected: the record says so)
+    assert len(calls) == 2 and ms == 12.0 and launches == 6
+    assert clocks["reasons"] == ["hw_slowdown"] and clocks["rejected_first"] == records[0]
+    calls.clear()
+    records[0] = records[2]
+    ms, _, _, clocks = bench._time_steps_checked(None, None, 1, 3, 1, "cpu", None, "auto")
+    assert len(calls) == 1 and ms == 11.0 and "rejected_first" not in clocks

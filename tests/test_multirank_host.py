@@ -35,8 +35,20 @@ def _rank_main(rank, world, port, results):
         shapes = torch.tensor([wl.total_q, wl.num_seqs, int(wl.seq_lens.sum())], dtype=torch.int64)
         gathered = [torch.zeros_like(shapes) for _ in range(world)]
         dist.all_gather(gathered, shapes)
+        # a clock record that rejects rank 0's timed region re-measures on every rank (same collectives)
+        calls = []
+
+        def fake_time_steps(replicas, stream, steps, warmup, world_, dev, sampler, selection):
+            calls.append(1)
+            throttled = rank == 0 and len(calls) == 1
+            return 1.0, {}, 0, {"sm_mhz": 1965.0, "sm_max_mhz": 1965,
+                                "reasons": ["hw_thermal_slowdown"] if throttled else []}
+
+        bench._time_steps = fake_time_steps
+        checked = bench._time_steps_checked(None, None, 1, 1, world, "cpu", None, "auto")
         results[rank] = {"job_ms": job_ms, "value": value, "seq_lens": wl.seq_lens.tolist(),
-                         "shapes": [g.tolist() for g in gathered]}
+                         "shapes": [g.tolist() for g in gathered], "timed_regions": len(calls),
+                         "rejected_first": checked[3].get("rejected_first")}
     finally:
         dist.destroy_process_group()
 
@@ -63,6 +75,10 @@ def test_two_gloo_ranks_slowest_rank_time_and_weak_scaling_value():
     assert res[0]["shapes"][0][:2] == res[0]["shapes"][1][:2] == [32, 32]
     assert res[0]["seq_lens"] != res[1]["seq_lens"]
     assert np.all(np.asarray(res[0]["seq_lens"]) >= 4096) and np.all(np.asarray(res[1]["seq_lens"]) <= 32768)
+    # rank 0's throttled region was measured again on both ranks; rank 0 keeps the rejected record
+    assert res[0]["timed_regions"] == res[1]["timed_regions"] == 2
+    assert res[0]["rejected_first"]["reasons"] == ["hw_thermal_slowdown"]
+    assert res[1]["rejected_first"]["reasons"] == []
 
 
 # ----------------------------------------------------------------------------- overlapped e2e leg

@@ -544,7 +544,7 @@ def traffic_key(regions):
     import hashlib
     m = hashlib.sha256()
     for f, start, end, incl in regions:
-        with open(os.path.join(ROOT, "sparse_attention_long_dsa_b200", "csrc", f)) as fh:
+        with open(os.path.join(ROOT, "sparse_attention_long_dsa_b200", "csrc", f), encoding="utf-8") as fh:
             m.update(_source_region(fh.read(), start, end, incl).encode())
     return m.hexdigest()[:16]
 
@@ -555,7 +555,7 @@ def measured_traffic(stage, workload):
         return None
     try:
         key = traffic_key(rec["regions"])
-    except StopIteration:          # a region's marker line is gone: the sources are not the captured ones
+    except (StopIteration, OSError, UnicodeDecodeError):   # a marker line or a file is gone: not the captured sources
         return None
     return rec["bytes"] if key == rec["sha256_16"] else None
 

@@ -826,7 +826,9 @@ def main():
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+        # ranks meet first after drawing their workloads (tens of seconds each, drawn at the same time); a
+        # collective left waiting longer than this ends with an error instead of holding the GPUs
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
         if args.impl == "reference":

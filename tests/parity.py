@@ -120,3 +120,55 @@ def compare_rows(case, db, rows, check_out=True):
             o, l = oracle.sparse_attention_row(case, r, gi[r])      # attention on the GPU's own index set
             check_attention(case, r, go[r], gl[r], o, l)
     return ref
+
+
+def candidates_per_row(case):
+    """n(row) = pos(row) + 1 for every query row (a sequence's rows are its last q_len tokens)."""
+    b = case.row_seq()
+    first = np.asarray(case.cu_q[:-1], np.int64)[b]
+    q_len = np.asarray(case.q_lens, np.int64)[b]
+    return np.asarray(case.seq_lens, np.int64)[b] - q_len + (np.arange(case.total_q) - first) + 1
+
+
+def check_topk_every_row(case, scores, idx, rows_per_chunk=256):
+    """The selection of every row against properties that fix the top-k of the given scores exactly: min(n, k)
+    entries, ascending, in [0, n), -1 only after them; no unselected score above the smallest selected one; and
+    among the keys tied at that score, the selected ones before the unselected ones (ties go to the lower
+    position; -0 and +0 compare equal).  `scores` [T, ld] and `idx` [T, k] are torch tensors on any device (the
+    GPU's own scores: the rule is checked on the values the selection saw); rows go in chunks to bound memory."""
+    import torch
+    n_all = candidates_per_row(case)
+    T, k = idx.shape
+    dev = idx.device
+    for r0 in range(0, T, rows_per_chunk):
+        r1 = min(T, r0 + rows_per_chunk)
+        n = torch.as_tensor(n_all[r0:r1], device=dev)
+        L = int(n_all[r0:r1].max())
+        pos = torch.arange(L, device=dev)
+        live = pos[None, :] < n[:, None]
+        S = torch.where(live, scores[r0:r1, :L].float(), torch.tensor(float("-inf"), device=dev))
+        I = idx[r0:r1].long()
+        valid = I >= 0
+        want = torch.clamp(n, max=k)
+        where = f"rows {r0}..{r1 - 1}"
+        assert torch.equal(valid.sum(1), want), f"{where}: wrong number of selected positions"
+        assert torch.equal(valid, torch.arange(k, device=dev)[None, :] < want[:, None]), f"{where}: -1 inside"
+        assert bool((I < n[:, None]).all()), f"{where}: a position past the row's candidates"
+        assert bool(((I[:, 1:] > I[:, :-1]) | ~valid[:, 1:]).all()), f"{where}: positions not ascending"
+        # how often each position is selected (the -1 entries land in a spare column L)
+        cnt = torch.zeros((r1 - r0, L + 1), dtype=torch.int32, device=dev)
+        cnt.scatter_add_(1, torch.where(valid, I, torch.full_like(I, L)), torch.ones_like(I, dtype=torch.int32))
+        assert bool((cnt[:, :L] <= 1).all()), f"{where}: a position selected twice"
+        sel = cnt[:, :L] > 0
+        full = n <= k                                          # every candidate selected: nothing to rank
+        inf = torch.tensor(float("inf"), device=dev)
+        tau = torch.where(sel, S, inf).min(1).values
+        unsel = live & ~sel
+        top_out = torch.where(unsel, S, -inf).max(1).values
+        bad = ~full & (top_out > tau)
+        assert not bool(bad.any()), f"{where}: an unselected score above the threshold (row {r0 + int(bad.nonzero()[0])})"
+        tied = S == tau[:, None]
+        last_sel = torch.where(sel & tied, pos[None, :], torch.full_like(pos, -1)[None, :]).max(1).values
+        first_out = torch.where(unsel & tied, pos[None, :], torch.full_like(pos, L)[None, :]).min(1).values
+        bad = ~full & (last_sel > first_out)
+        assert not bool(bad.any()), f"{where}: a tie at the threshold went to a higher position (row {r0 + int(bad.nonzero()[0])})"

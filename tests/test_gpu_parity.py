@@ -2,14 +2,15 @@
 
 Small cases run every row and span several tiles plus ragged tails; the five full-size
 workloads run in the same launch configuration the benchmark times and are checked on
-sampled rows (rows are independent, so a sampled row is a complete check of that row).
+sampled rows (rows are independent, so a sampled row is a complete check of that row), and every row's
+selection against the top-k's defining properties on the GPU's own scores.
 """
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from parity import check_attention, compare_rows, sample_rows
+from parity import check_attention, check_topk_every_row, compare_rows, sample_rows
 from sparse_attention_long_dsa_b200 import binding as B
 from sparse_attention_long_dsa_b200 import workloads as W
 from sparse_attention_long_dsa_b200.pipeline import DeviceBatch
@@ -196,12 +197,14 @@ def test_decode_batch(grid):
     wl = W.decode_batch(grid=grid)
     db = _run(wl)
     compare_rows(wl, db, sample_rows(wl, extra=4))
+    check_topk_every_row(wl, db.scores, db.idx)
 
 
 def test_prefill_16k():
     wl = W.prefill_16k()
     db = _run(wl)
     compare_rows(wl, db, sample_rows(wl, extra=24))
+    check_topk_every_row(wl, db.scores, db.idx)
 
 
 def test_decode_1m_planted():
@@ -210,6 +213,7 @@ def test_decode_1m_planted():
     got = db.idx.cpu().numpy()[0]
     assert np.array_equal(got, wl.planted.astype(np.int32)), "GPU top-k is not the planted set"
     compare_rows(wl, db, [0])
+    check_topk_every_row(wl, db.scores, db.idx)
 
 
 def test_mixed_batch():
@@ -217,6 +221,7 @@ def test_mixed_batch():
     db = _run(wl)
     assert not db.decode
     compare_rows(wl, db, sample_rows(wl, extra=16))
+    check_topk_every_row(wl, db.scores, db.idx)
 
 
 # --------------------------------------------------------------------------------------- ABI on device

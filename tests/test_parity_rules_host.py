@@ -141,3 +141,72 @@ def test_attention_rule_mean_relative_bound():
     parity.check_attention(case, 0, small, l, small, l)
     with pytest.raises(AssertionError, match="mean-rel"):
         parity.check_attention(case, 0, small * 1.02, l, small, l)
+
+
+def _scored_case(tied):
+    """A 4-row case, its scores (garbage past each row's candidates, as the kernels leave them) and the
+    oracle's selection of every row."""
+    import torch
+    case = W.make_workload("rows", kind="f32", seed=93, seq_lens=[300, 150, 20], q_lens=[2, 2, 1], topk=32,
+                           H=3, Dqk=16, Dv=12, Hi=2, Di=8)
+    rng = np.random.default_rng(94 if tied else 95)
+    ld = 304
+    sc = (rng.integers(-2, 3, (case.total_q, ld)) if tied else rng.standard_normal((case.total_q, ld))).astype(np.float32)
+    if tied:
+        sc[0, ::7] = -0.0                                                       # -0 ties +0
+    n = parity.candidates_per_row(case)
+    idx = np.stack([oracle.topk_row(sc[r, : n[r]].astype(np.float64), case.topk) for r in range(case.total_q)])
+    sc[np.arange(ld)[None, :] >= n[:, None]] = 1e30                            # never read
+    return case, torch.from_numpy(sc), torch.from_numpy(idx), n
+
+
+def test_candidates_per_row_by_hand():
+    case, _, _, n = _scored_case(False)
+    assert n.tolist() == [299, 300, 149, 150, 20]
+
+
+@pytest.mark.parametrize("tied", [False, True])
+def test_every_row_rule_accepts_the_definition(tied):
+    case, sc, idx, _ = _scored_case(tied)
+    for chunk in (1, 2, 256):
+        parity.check_topk_every_row(case, sc, idx, rows_per_chunk=chunk)
+
+
+def test_every_row_rule_rejects_planted_errors():
+    import torch
+    case, sc, idx, n = _scored_case(True)
+    k = case.topk
+    r = 2                                                                         # 149 candidates, k = 32
+    s = sc[r, : n[r]].double().numpy()
+    sel = idx[r].numpy()
+    tau = s[sel].min()
+    out = np.setdiff1d(np.arange(n[r]), sel)
+
+    def planted(fn):
+        bad = idx.clone()
+        fn(bad[r])
+        with pytest.raises(AssertionError):
+            parity.check_topk_every_row(case, sc, bad)
+
+    lower = out[s[out] < tau][0]                       # a key strictly below the threshold
+    tied_out = out[s[out] == tau]                      # keys tied at the threshold left out (higher positions)
+    last_tied_in = sel[s[sel] == tau].max()
+    assert tied_out.size and tied_out.min() > last_tied_in
+
+    def swap(row, old, new):
+        v = row.numpy()
+        v[v == old] = new
+        v.sort()
+
+    planted(lambda row: swap(row, sel[np.argmin(s[sel])], lower))                # below the threshold
+    planted(lambda row: swap(row, last_tied_in, tied_out.max()))                 # tie to a higher position
+    planted(lambda row: row.__setitem__(k - 1, -1))                              # one short
+    planted(lambda row: row.__setitem__(0, -1))                                  # -1 first
+    planted(lambda row: row.__setitem__(k - 1, int(n[r])))                       # past the candidates
+    planted(lambda row: row.__setitem__(1, int(row[0])))                         # one position twice
+    planted(lambda row: row.copy_(torch.flip(row, [0])))                         # descending
+    # a row with fewer candidates than k must select all of them
+    bad = idx.clone()
+    bad[4, 19] = -1
+    with pytest.raises(AssertionError):
+        parity.check_topk_every_row(case, sc, bad)

@@ -1,6 +1,6 @@
 """The seeded input generator (no GPU): the same seed gives the same arrays whatever the number of host
-threads that draw them, different seeds give different draws, and the decode-batch recipe has the shapes and
-ranges it is documented with."""
+threads that draw them, different seeds give different draws, the decode-batch recipe has the shapes and
+ranges it is documented with, and the other recipes hand the generator their documented configurations."""
 import numpy as np
 
 from sparse_attention_long_dsa_b200 import workloads as W
@@ -40,3 +40,31 @@ def test_decode_batch_recipe():
     # w ~ N(0, 1/64): sample standard deviation near 1/8
     assert abs(float(np.std(wl.w)) - 0.125) < 0.01
     assert np.all(wl.kS_pool > 0)
+
+
+def _recipe(monkeypatch, fn, **kw):
+    """The arguments a workload recipe hands to make_workload (nothing is drawn)."""
+    got = {}
+    monkeypatch.setattr(W, "make_workload", lambda name, **a: got.update(a, name=name) or got)
+    fn(**kw)
+    return got
+
+
+def test_other_recipes(monkeypatch):
+    t = _recipe(monkeypatch, W.tiny_f32)
+    assert (t["kind"], list(t["seq_lens"]), list(t["q_lens"]), t["topk"]) == ("f32", [256], [256], 32)
+    assert (t["H"], t["Dqk"], t["Dv"], t["Hi"], t["Di"]) == (4, 64, 64, 2, 32)
+    assert t["shuffle"] is False and t["w_dist"] == "uniform" and t["seed"] == 20260001
+    p = _recipe(monkeypatch, W.prefill_16k)
+    assert (p["kind"], list(p["seq_lens"]), list(p["q_lens"]), p["topk"]) == ("mla", [16384], [16384], 2048)
+    p4 = _recipe(monkeypatch, W.prefill_4k)
+    assert (list(p4["seq_lens"]), list(p4["q_lens"]), p4["topk"]) == ([4096], [4096], 2048)
+    d = _recipe(monkeypatch, W.decode_1m_planted)
+    assert (list(d["seq_lens"]), list(d["q_lens"]), d["topk"], d["planted_k"]) == ([1 << 20], [1], 2048, 2048)
+    m = _recipe(monkeypatch, W.mixed_batch)
+    sl, ql = np.asarray(m["seq_lens"]), np.asarray(m["q_lens"])
+    assert m["kind"] == "mla" and m["topk"] == 2048 and sl.size == ql.size == 18
+    assert np.all(ql[:16] == 1) and np.all((sl[:16] >= 8192) & (sl[:16] <= 131072))
+    # two chunks of 8192 rows: positions 57,344..65,535 of 65,536-token sequences (the chunk's KV is cached)
+    assert list(ql[16:]) == [8192, 8192] and list(sl[16:]) == [65536, 65536]
+    assert list(sl[16:] - ql[16:]) == [57344, 57344]

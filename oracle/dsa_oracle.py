@@ -66,7 +66,7 @@ routines, brute force).
 from __future__ import annotations
 
 import math
-from typing import Iterable, Optional, Sequence
+from typing import Iterable, Sequence
 
 import numpy as np
 
@@ -350,11 +350,9 @@ def combine(parts: Sequence, lses: Sequence):
 # whole path, row by row
 # ----------------------------------------------------------------------------
 
-def run_rows(case, rows: Iterable[int], idx_override: Optional[dict] = None,
-             want_scores: bool = True, want_attention: bool = True) -> dict:
-    """Scores, top-k and attention of the given query rows.  `idx_override[row]` replaces
-    the oracle's own selection for the attention step (conditional parity on another
-    implementation's index set)."""
+def run_rows(case, rows: Iterable[int], want_scores: bool = True, want_attention: bool = True) -> dict:
+    """Scores, top-k and attention of the given query rows (attention on another implementation's index set
+    is `sparse_attention_row` called with that set)."""
     res = {}
     for row in rows:
         row = int(row)
@@ -364,8 +362,7 @@ def run_rows(case, rows: Iterable[int], idx_override: Optional[dict] = None,
             r["scores"] = sc
         r["idx"] = topk_row(sc, case.topk)
         if want_attention:
-            idx = r["idx"] if idx_override is None or row not in idx_override else idx_override[row]
-            r["out"], r["lse"] = sparse_attention_row(case, row, idx)
+            r["out"], r["lse"] = sparse_attention_row(case, row, r["idx"])
         res[row] = r
     return res
 
